@@ -1,0 +1,164 @@
+/*
+ * attn_sink.h -- C ABI of the B200 (sm_100a) sink-attention library, libattn_sink.so.
+ *
+ * The operation (Huawei CANN ops-transformer "flash_attn" doc, section "Function",
+ * the formula after "After adding sink"):
+ *
+ *     S   = scale * Q K^T                       per (sequence, q head)
+ *     m   = max(sink, max_j S_j)
+ *     out = sum_j e^{S_j - m} V_j / (sum_j e^{S_j - m} + e^{sink - m})
+ *
+ * sink is a per-q-head fp32 logit in post-scale units.  It is the learnable softmax
+ * offset of slime's learnable_softmax_attention.py (module docstring: an appended
+ * logit column, equivalently softmax(S) * sigmoid(lse - offset)) and softmax_n of the
+ * Flash-Attention-Softmax-N README with sink = log n.  A NULL sink means -inf, i.e.
+ * plain softmax attention.
+ *
+ * Conventions shared by every entry point
+ *   - Layout: packed THD, row-major, contiguous.
+ *       q   [total_q, num_heads_q,  head_dim_qk]
+ *       k   [total_k, num_heads_kv, head_dim_qk]
+ *       v   [total_k, num_heads_kv, head_dim_v ]
+ *       out [total_q, num_heads_q,  head_dim_v ]
+ *       lse [num_heads_q, total_q] fp32   (CANN doc, softmax_lse note: (Q_N, Q_T) for TND)
+ *       sink [num_heads_q] fp32
+ *     Sequence b owns q rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and k/v rows
+ *     [cu_seqlens_k[b], cu_seqlens_k[b+1]); both arrays are int32 [batch + 1], start
+ *     at 0, never decrease, end at total_q / total_k (slime wrapper docstring; CANN doc,
+ *     "SeqLengths Parameter Group").  Zero-length sequences are allowed.
+ *   - GQA: num_heads_q % num_heads_kv == 0; q head h reads kv head
+ *     h / (num_heads_q / num_heads_kv) (CANN doc, "Common Parameter Group").
+ *   - Masking: query row i of a sequence with sq queries and sk keys sits at key
+ *     position i + (sk - sq) (bottom-right alignment, PyTorch issue #108108,
+ *     "Proposal").  It sees key j iff  pos - window_left <= j <= pos + window_right,
+ *     where -1 means unbounded (slime wrapper docstring "window_size"; CANN doc,
+ *     "Mask Parameter Group") and causal sets window_right = min(window_right, 0).
+ *     A row that sees no key outputs 0 (issue #108108) and has lse = -inf.
+ *   - lse is the vanilla log-sum-exp of the visible scaled scores, natural log,
+ *     WITHOUT the sink (CANN doc, softmax_lse formula).
+ *   - dtype: ATTN_SINK_BF16 (bf16 q/k/v/out/dout/dq/dk/dv, fp32 accumulation, outputs
+ *     rounded once to nearest-even) or ATTN_SINK_FP32 (fp32 everywhere, no tensor cores).
+ *   - Supported head dims: head_dim_qk in {64, 128}; head_dim_v in {32, 64, 128}.
+ *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace).  The
+ *     library never allocates, frees or synchronises; every pointer except `params`
+ *     is a device pointer and must be 16-byte aligned.  Calls are asynchronous on
+ *     `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *   - Errors: the return value is an attn_sink_status.  Arguments the host can see
+ *     are validated before anything is launched (ATTN_SINK_ERR_INVALID_ARG,
+ *     ATTN_SINK_ERR_UNSUPPORTED, ATTN_SINK_ERR_WORKSPACE); a failed launch returns
+ *     ATTN_SINK_ERR_CUDA.  The contents of cu_seqlens are the caller's contract (as in
+ *     the CANN doc's "Declaration"): they are not read on the host.  Kernels that wait
+ *     on on-chip barriers give every wait an iteration limit; a wait that runs out
+ *     sets a bit in a per-device status word and the kernel returns early, leaving
+ *     the outputs undefined.  attn_sink_get_device_status() reads and clears it.
+ */
+#ifndef ATTN_SINK_H
+#define ATTN_SINK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { ATTN_SINK_BF16 = 0, ATTN_SINK_FP32 = 1 } attn_sink_dtype;
+
+typedef enum {
+  ATTN_SINK_OK = 0,
+  ATTN_SINK_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, ... */
+  ATTN_SINK_ERR_UNSUPPORTED = 2,   /* head dims / dtype outside the supported set     */
+  ATTN_SINK_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required      */
+  ATTN_SINK_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed            */
+  ATTN_SINK_ERR_TIMEOUT = 5        /* device status: a bounded on-chip wait ran out   */
+} attn_sink_status;
+
+/* Problem description shared by the three entry points (plain struct, by pointer). */
+typedef struct {
+  int batch;            /* B > 0: number of sequences                                  */
+  int total_q;          /* rows of q / out (> 0); decode: must equal batch             */
+  int total_k;          /* rows of k / v (> 0)                                         */
+  int max_seqlen_q;     /* >= every sequence's query length (decode: 1)                */
+  int max_seqlen_k;     /* >= every sequence's key length                              */
+  int num_heads_q;      /* Hq > 0                                                      */
+  int num_heads_kv;     /* Hkv > 0, Hq % Hkv == 0                                      */
+  int head_dim_qk;      /* 64 or 128                                                   */
+  int head_dim_v;       /* 32, 64 or 128                                               */
+  float softmax_scale;  /* multiplies QK^T; finite.  The slime wrapper's default is
+                           1/sqrt(head_dim_qk); here the caller passes it explicitly   */
+  int causal;           /* nonzero: bottom-right causal                                */
+  int window_left;      /* >= -1; -1 = unbounded                                       */
+  int window_right;     /* >= -1; -1 = unbounded                                       */
+  attn_sink_dtype dtype;
+} attn_sink_params;
+
+/* Opaque stream handle: pass a cudaStream_t. */
+typedef void* attn_sink_stream_t;
+
+/*
+ * Forward (CANN doc, "Function" formula and softmax_lse formula; slime
+ * learnable_softmax_flash_attn_varlen).  Writes out [total_q, Hq, dv] (dtype) and, when
+ * `lse` is not NULL, lse [Hq, total_q] fp32.  sink may be NULL (= -inf).  The workspace
+ * may be NULL when attn_sink_fwd_workspace_size() returns 0.
+ */
+int attn_sink_fwd(const attn_sink_params* params, const void* q, const void* k, const void* v,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
+                  void* out, float* lse, void* workspace, size_t workspace_bytes,
+                  attn_sink_stream_t stream);
+
+/*
+ * Backward of the forward above for the loss sum(dout * out) (the gradient the slime
+ * class docstring describes: dS = P * s * (D - s * di) with s = sigmoid(lse - sink),
+ * and d_offset = -sum_i (dout_i . out_vanilla_i) s_i (1 - s_i)).
+ * Inputs: q, k, v, the forward's out and lse (lse REQUIRED), dout [total_q, Hq, dv].
+ * Outputs (all overwritten): dq [total_q, Hq, dk], dk [total_k, Hkv, dk],
+ * dv [total_k, Hkv, dv] (dtype; dk / dv sum over the q heads of each group) and
+ * dsink [Hq] fp32 (may be NULL when sink is NULL or not wanted).
+ */
+int attn_sink_bwd(const attn_sink_params* params, const void* q, const void* k, const void* v,
+                  const void* out, const void* dout, const float* lse,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
+                  void* dq, void* dk, void* dv, float* dsink, void* workspace,
+                  size_t workspace_bytes, attn_sink_stream_t stream);
+
+/*
+ * Decode: one query per sequence, q [batch, Hq, dk] (cu_seqlens_q = 0, 1, ..., batch is
+ * implied; total_q == batch, max_seqlen_q == 1).  K/V are packed with cu_seqlens_k.
+ * The keys of each (sequence, kv head) are cut into num_splits chunks (0 = choose
+ * automatically), each chunk produces (max, sum, unnormalised output) without the sink,
+ * and a merge combines them and applies the sink exactly once (CANN doc, softmax_lse
+ * note on combining partial results).  Writes out [batch, Hq, dv] and, when not NULL,
+ * lse [Hq, batch].  The workspace holds the partials.  fp32 problems are computed
+ * without splitting.
+ */
+int attn_sink_decode(const attn_sink_params* params, const void* q, const void* k, const void* v,
+                     const int32_t* cu_seqlens_k, const float* sink, int num_splits, void* out,
+                     float* lse, void* workspace, size_t workspace_bytes,
+                     attn_sink_stream_t stream);
+
+/* Workspace bytes each entry point needs for `params` (0 = none; SIZE_MAX = params invalid). */
+size_t attn_sink_fwd_workspace_size(const attn_sink_params* params);
+size_t attn_sink_bwd_workspace_size(const attn_sink_params* params);
+size_t attn_sink_decode_workspace_size(const attn_sink_params* params, int num_splits);
+
+/* The split count attn_sink_decode uses for num_splits == 0. */
+int attn_sink_decode_num_splits(const attn_sink_params* params);
+
+/* Static text for a status code. */
+const char* attn_sink_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's status word.
+ * Returns ATTN_SINK_OK, ATTN_SINK_ERR_TIMEOUT (a bounded wait ran out) or
+ * ATTN_SINK_ERR_CUDA.  *bits (if not NULL) receives the raw word.
+ */
+int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+int attn_sink_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_SINK_H */

@@ -1,0 +1,258 @@
+// Host side of the C ABI declared in include/attn_sink.h: argument validation, workspace
+// layout, kernel dispatch and the per-device status word.  No allocation, no
+// synchronisation (except attn_sink_get_device_status, which exists to synchronise).
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/attn_sink.h"
+#include "launch.h"
+
+using namespace attn_sink;
+
+namespace {
+
+// Bits set by kernels whose bounded waits ran out (kStatusTimeout).
+__device__ unsigned int g_status_word;
+
+constexpr int kMaxDevices = 64;
+unsigned* g_status_ptr[kMaxDevices];
+
+unsigned* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool dims_supported(int dk, int dv) {
+  return (dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128);
+}
+
+int validate_params(const attn_sink_params* p, bool decode) {
+  if (!p) return ATTN_SINK_ERR_INVALID_ARG;
+  if (p->dtype != ATTN_SINK_BF16 && p->dtype != ATTN_SINK_FP32) return ATTN_SINK_ERR_UNSUPPORTED;
+  if (p->batch <= 0 || p->total_q <= 0 || p->total_k <= 0) return ATTN_SINK_ERR_INVALID_ARG;
+  if (p->num_heads_q <= 0 || p->num_heads_kv <= 0) return ATTN_SINK_ERR_INVALID_ARG;
+  if (p->num_heads_q % p->num_heads_kv != 0) return ATTN_SINK_ERR_INVALID_ARG;
+  if (p->max_seqlen_q < 1 || p->max_seqlen_k < 1) return ATTN_SINK_ERR_INVALID_ARG;
+  if (p->max_seqlen_q > p->total_q || p->max_seqlen_k > p->total_k) return ATTN_SINK_ERR_INVALID_ARG;
+  if (p->window_left < -1 || p->window_right < -1) return ATTN_SINK_ERR_INVALID_ARG;
+  if (!isfinite(p->softmax_scale)) return ATTN_SINK_ERR_INVALID_ARG;
+  if (!dims_supported(p->head_dim_qk, p->head_dim_v)) return ATTN_SINK_ERR_UNSUPPORTED;
+  if (decode && (p->total_q != p->batch || p->max_seqlen_q != 1)) return ATTN_SINK_ERR_INVALID_ARG;
+  return ATTN_SINK_OK;
+}
+
+void effective_window(const attn_sink_params* p, int& left, int& right) {
+  left = p->window_left < 0 ? kUnbounded : p->window_left;
+  right = p->window_right < 0 ? kUnbounded : p->window_right;
+  if (p->causal && right > 0) right = 0;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? ATTN_SINK_OK : ATTN_SINK_ERR_CUDA; }
+
+// workspace layout of the backward
+struct BwdLayout {
+  size_t D, lse_tot, dq_acc, total;
+};
+BwdLayout bwd_layout(const attn_sink_params* p) {
+  BwdLayout l{};
+  const size_t rows = (size_t)p->num_heads_q * p->total_q;
+  l.D = 0;
+  l.lse_tot = align_up(l.D + rows * 4, 256);
+  l.dq_acc = align_up(l.lse_tot + rows * 4, 256);
+  size_t end = l.dq_acc;
+  if (p->dtype == ATTN_SINK_BF16) end += (size_t)p->total_q * p->num_heads_q * p->head_dim_qk * 4;
+  l.total = align_up(end, 256);
+  return l;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+int decode_auto_splits(const attn_sink_params* p) {
+  const int group = p->num_heads_q / p->num_heads_kv;
+  const long long units = (long long)p->num_heads_kv * ((group + 15) / 16);
+  const long long target = 4LL * sm_count();
+  long long chunk = (long long)p->total_k * units / target;
+  if (chunk < 256) chunk = 256;
+  if (chunk > 2048) chunk = 2048;
+  chunk = (chunk + 63) / 64 * 64;
+  long long splits = (p->max_seqlen_k + chunk - 1) / chunk;
+  if (splits < 1) splits = 1;
+  if (splits > 1024) splits = 1024;
+  return (int)splits;
+}
+
+size_t decode_ws(const attn_sink_params* p, int splits) {
+  if (p->dtype != ATTN_SINK_BF16) return 0;
+  const size_t rows = (size_t)p->batch * p->num_heads_q * splits;
+  return align_up(rows * p->head_dim_v * 4, 256) + align_up(rows * 2 * 4, 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_sink_version(void) { return 0x000100; }
+
+const char* attn_sink_status_string(int status) {
+  switch (status) {
+    case ATTN_SINK_OK: return "ok";
+    case ATTN_SINK_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_SINK_ERR_UNSUPPORTED: return "unsupported dtype or head dims";
+    case ATTN_SINK_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_SINK_ERR_CUDA: return "CUDA error";
+    case ATTN_SINK_ERR_TIMEOUT: return "a bounded on-chip wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t attn_sink_fwd_workspace_size(const attn_sink_params* p) {
+  if (validate_params(p, false) != ATTN_SINK_OK) return SIZE_MAX;
+  return 0;
+}
+
+size_t attn_sink_bwd_workspace_size(const attn_sink_params* p) {
+  if (validate_params(p, false) != ATTN_SINK_OK) return SIZE_MAX;
+  return bwd_layout(p).total;
+}
+
+int attn_sink_decode_num_splits(const attn_sink_params* p) {
+  if (validate_params(p, true) != ATTN_SINK_OK) return -1;
+  return decode_auto_splits(p);
+}
+
+size_t attn_sink_decode_workspace_size(const attn_sink_params* p, int num_splits) {
+  if (validate_params(p, true) != ATTN_SINK_OK || num_splits < 0) return SIZE_MAX;
+  return decode_ws(p, num_splits == 0 ? decode_auto_splits(p) : num_splits);
+}
+
+int attn_sink_fwd(const attn_sink_params* p, const void* q, const void* k, const void* v,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
+                  void* out, float* lse, void* workspace, size_t workspace_bytes,
+                  attn_sink_stream_t stream) {
+  int st = validate_params(p, false);
+  if (st != ATTN_SINK_OK) return st;
+  if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !out) return ATTN_SINK_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
+  if ((lse && !aligned16(lse)) || (sink && !aligned16(sink))) return ATTN_SINK_ERR_INVALID_ARG;
+  (void)workspace;
+  (void)workspace_bytes;
+  FwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
+  a.out = out; a.lse = lse;
+  a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
+  a.max_sq = p->max_seqlen_q; a.max_sk = p->max_seqlen_k;
+  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
+  a.scale = p->softmax_scale;
+  effective_window(p, a.left, a.right);
+  a.status = status_ptr();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dt = p->dtype == ATTN_SINK_FP32 ? 1 : 0;
+  if (dt == 0 && fwd_sm100_supported(a, dt)) return from_cuda(launch_fwd_sm100(a, s));
+  return from_cuda(launch_fwd_simt(a, dt, s));
+}
+
+int attn_sink_bwd(const attn_sink_params* p, const void* q, const void* k, const void* v,
+                  const void* out, const void* dout, const float* lse,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
+                  void* dq, void* dk, void* dv, float* dsink, void* workspace,
+                  size_t workspace_bytes, attn_sink_stream_t stream) {
+  int st = validate_params(p, false);
+  if (st != ATTN_SINK_OK) return st;
+  if (!q || !k || !v || !out || !dout || !lse || !cu_seqlens_q || !cu_seqlens_k || !dq || !dk || !dv)
+    return ATTN_SINK_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, out, dout, (const void*)lse, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
+  if ((sink && !aligned16(sink)) || (dsink && !aligned16(dsink))) return ATTN_SINK_ERR_INVALID_ARG;
+  const BwdLayout lay = bwd_layout(p);
+  if (!workspace || workspace_bytes < lay.total || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  BwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.lse = lse;
+  a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
+  a.grad_q = dq; a.grad_k = dk; a.grad_v = dv; a.dsink = dsink;
+  a.D = reinterpret_cast<float*>(ws + lay.D);
+  a.lse_tot = reinterpret_cast<float*>(ws + lay.lse_tot);
+  a.dq_acc = p->dtype == ATTN_SINK_BF16 ? reinterpret_cast<float*>(ws + lay.dq_acc) : nullptr;
+  a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
+  a.max_sq = p->max_seqlen_q; a.max_sk = p->max_seqlen_k;
+  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
+  a.scale = p->softmax_scale;
+  effective_window(p, a.left, a.right);
+  a.status = status_ptr();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dt = p->dtype == ATTN_SINK_FP32 ? 1 : 0;
+  if (dt == 0 && bwd_sm100_supported(a, dt)) return from_cuda(launch_bwd_sm100(a, s));
+  return from_cuda(launch_bwd_simt(a, dt, s));
+}
+
+int attn_sink_decode(const attn_sink_params* p, const void* q, const void* k, const void* v,
+                     const int32_t* cu_seqlens_k, const float* sink, int num_splits, void* out,
+                     float* lse, void* workspace, size_t workspace_bytes,
+                     attn_sink_stream_t stream) {
+  int st = validate_params(p, true);
+  if (st != ATTN_SINK_OK) return st;
+  if (num_splits < 0) return ATTN_SINK_ERR_INVALID_ARG;
+  if (!q || !k || !v || !cu_seqlens_k || !out) return ATTN_SINK_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
+  if ((lse && !aligned16(lse)) || (sink && !aligned16(sink))) return ATTN_SINK_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int left, right;
+  effective_window(p, left, right);
+  if (p->dtype == ATTN_SINK_FP32) {
+    FwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.cu_q = nullptr; a.cu_k = cu_seqlens_k; a.sink = sink;
+    a.out = out; a.lse = lse;
+    a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
+    a.max_sq = 1; a.max_sk = p->max_seqlen_k;
+    a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
+    a.scale = p->softmax_scale; a.left = left; a.right = right;
+    a.status = status_ptr();
+    return from_cuda(launch_fwd_simt(a, 1, s));
+  }
+  const int splits = num_splits == 0 ? decode_auto_splits(p) : num_splits;
+  const size_t need = decode_ws(p, splits);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
+  const size_t rows = (size_t)p->batch * p->num_heads_q * splits;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  DecodeArgs a{};
+  a.q = q; a.k = k; a.v = v; a.cu_k = cu_seqlens_k; a.sink = sink; a.out = out; a.lse = lse;
+  a.part_o = reinterpret_cast<float*>(ws);
+  a.part_ml = reinterpret_cast<float*>(ws + align_up(rows * p->head_dim_v * 4, 256));
+  a.batch = p->batch; a.total_k = p->total_k; a.max_sk = p->max_seqlen_k;
+  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
+  a.splits = splits; a.scale = p->softmax_scale; a.left = left; a.right = right;
+  a.status = status_ptr();
+  return from_cuda(launch_decode_split(a, s));
+}
+
+int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits) {
+  unsigned* sp = status_ptr();
+  if (!sp) return ATTN_SINK_ERR_CUDA;
+  unsigned host = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&host, sp, sizeof(unsigned), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_SINK_ERR_CUDA;
+  if (cudaMemsetAsync(sp, 0, sizeof(unsigned), s) != cudaSuccess) return ATTN_SINK_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_SINK_ERR_CUDA;
+  if (bits) *bits = host;
+  return host ? ATTN_SINK_ERR_TIMEOUT : ATTN_SINK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,316 @@
+// Sink-attention backward on the CUDA cores (fp32 problems and uncovered head dims),
+// plus the preprocess pass every backward uses.
+//
+// Gradient of the sink forward for the loss sum(dout * out).  With the forward's vanilla
+// lse and lse_tot = logaddexp(lse, sink), the sink-normalised probabilities are
+// P_ij = e^{S_ij - lse_tot_i} and the sink's share is p_sink_i = e^{sink - lse_tot_i}.
+// Then D_i = dout_i . out_i, dS = P * (dout V^T - D), dq = scale dS K, dk = scale dS^T Q,
+// dv = P^T dout and dsink = -sum_i p_sink_i D_i.  slime's learnable_softmax_attention.py
+// states the same gradient as dS = P_van * s * (D - s * di) with s = sigmoid(lse - offset)
+// (class docstring) and d_offset = -sum (dout . out_van) s (1 - s) (``backward``);
+// P = s P_van and D = s di make the two forms equal.
+#include "common.cuh"
+
+namespace attn_sink {
+namespace {
+
+__device__ __forceinline__ float logaddexp(float a, float b) {
+  if (a == kNegInf) return b;
+  if (b == kNegInf) return a;
+  const float mx = fmaxf(a, b);
+  return mx + log1pf(__expf(-fabsf(a - b)));
+}
+
+// --- preprocess: D, lse_tot and dsink ------------------------------------------------
+// grid (ceil(total_q / 64), hq), 256 threads: each warp handles 8 rows of one head.
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
+  const int h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* out = static_cast<const T*>(a.out);
+  const T* dout = static_cast<const T*>(a.dout);
+  const float sink = a.sink ? a.sink[h] : kNegInf;
+  float ds_acc = 0.f;
+  for (int rr = 0; rr < 8; ++rr) {
+    const long long i = ((long long)blockIdx.x * 8 + warp) * 8 + rr;
+    if (i >= a.total_q) break;
+    const long long base = (i * a.hq + h) * a.dv;
+    float d = 0.f;
+    for (int c = lane; c < a.dv; c += 32) d = fmaf(to_float(out[base + c]), to_float(dout[base + c]), d);
+    d = warp_sum(d);
+    const float lse = a.lse[(long long)h * a.total_q + i];
+    const float lt = logaddexp(lse, sink);
+    if (lane == 0) {
+      a.D[(long long)h * a.total_q + i] = d;
+      a.lse_tot[(long long)h * a.total_q + i] = lt;
+    }
+    if (sink != kNegInf && lt != kNegInf) ds_acc -= __expf(sink - lt) * d;
+  }
+  __shared__ float red[8];
+  if (lane == 0) red[warp] = ds_acc;
+  __syncthreads();
+  if (threadIdx.x == 0 && a.dsink) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += red[w];
+    atomicAdd(a.dsink + h, s);
+  }
+}
+
+// --- dK / dV: key-stationary -----------------------------------------------------------
+// grid (ceil(max_sk / 8), hkv, batch), 4 warps x 2 keys.  Each block owns its keys for
+// one kv head and loops over every q head of the group, so no atomics are needed.
+constexpr int kKeysPerWarp = 2;
+constexpr int kWarps = 4;
+constexpr int kBlockKeys = kKeysPerWarp * kWarps;
+constexpr int kTile = 32;
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(kWarps * 32) bwd_dkdv_simt_kernel(const BwdArgs a) {
+  constexpr int KPL = DK / 32, VPL = DV / 32;
+  __shared__ float s_k[kBlockKeys][DK];
+  __shared__ float s_v[kBlockKeys][DV];
+  __shared__ float s_q[kTile][DK + 1];
+  __shared__ float s_do[kTile][DV + 1];
+  __shared__ float s_lt[kTile], s_D[kTile];
+
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
+  const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
+  const long long j0 = (long long)blockIdx.x * kBlockKeys;
+  if (j0 >= sk) return;
+  const int group = a.hq / a.hkv;
+  const T* q = static_cast<const T*>(a.q);
+  const T* kp = static_cast<const T*>(a.k);
+  const T* vp = static_cast<const T*>(a.v);
+  const T* dout = static_cast<const T*>(a.dout);
+
+  for (int idx = threadIdx.x; idx < kBlockKeys * DK; idx += blockDim.x) {
+    const int j = idx / DK, c = idx % DK;
+    s_k[j][c] = (j0 + j < sk) ? to_float(kp[((k0 + j0 + j) * a.hkv + g) * DK + c]) : 0.f;
+  }
+  for (int idx = threadIdx.x; idx < kBlockKeys * DV; idx += blockDim.x) {
+    const int j = idx / DV, c = idx % DV;
+    s_v[j][c] = (j0 + j < sk) ? to_float(vp[((k0 + j0 + j) * a.hkv + g) * DV + c]) : 0.f;
+  }
+  const long long j_last = (j0 + kBlockKeys < sk ? j0 + kBlockKeys : sk) - 1;
+  long long lo0, hi0, lo1, hi1;
+  key_query_range(j0, sq, sk, a.left, a.right, lo0, hi0);
+  key_query_range(j_last, sq, sk, a.left, a.right, lo1, hi1);
+  const long long lo = lo0 < lo1 ? lo0 : lo1;
+  const long long hi = hi0 > hi1 ? hi0 : hi1;
+
+  float dk_acc[kKeysPerWarp][KPL], dv_acc[kKeysPerWarp][VPL];
+#pragma unroll
+  for (int kk = 0; kk < kKeysPerWarp; ++kk) {
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) dk_acc[kk][c] = 0.f;
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) dv_acc[kk][c] = 0.f;
+  }
+
+  for (int hh = 0; hh < group; ++hh) {
+    const int h = g * group + hh;
+    for (long long t0 = lo; t0 < hi; t0 += kTile) {
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < kTile * DK; idx += blockDim.x) {
+        const int i = idx / DK, c = idx % DK;
+        s_q[i][c] = (t0 + i < hi) ? to_float(q[((q0 + t0 + i) * a.hq + h) * DK + c]) : 0.f;
+      }
+      for (int idx = threadIdx.x; idx < kTile * DV; idx += blockDim.x) {
+        const int i = idx / DV, c = idx % DV;
+        s_do[i][c] = (t0 + i < hi) ? to_float(dout[((q0 + t0 + i) * a.hq + h) * DV + c]) : 0.f;
+      }
+      if (threadIdx.x < kTile) {
+        const long long i = t0 + threadIdx.x;
+        s_lt[threadIdx.x] = (i < hi) ? a.lse_tot[(long long)h * a.total_q + q0 + i] : 0.f;
+        s_D[threadIdx.x] = (i < hi) ? a.D[(long long)h * a.total_q + q0 + i] : 0.f;
+      }
+      __syncthreads();
+      const long long i = t0 + lane;
+#pragma unroll
+      for (int kk = 0; kk < kKeysPerWarp; ++kk) {
+        const int jl = warp * kKeysPerWarp + kk;
+        const long long j = j0 + jl;
+        if (j >= sk) continue;  // warp-uniform
+        const bool vis = (i < hi) && visible(i, j, sq, sk, a.left, a.right);
+        float p = 0.f, ds = 0.f;
+        if (vis) {
+          float s = 0.f, dp = 0.f;
+#pragma unroll 8
+          for (int c = 0; c < DK; ++c) s = fmaf(s_q[lane][c], s_k[jl][c], s);
+#pragma unroll 8
+          for (int c = 0; c < DV; ++c) dp = fmaf(s_do[lane][c], s_v[jl][c], dp);
+          p = __expf(s * a.scale - s_lt[lane]);
+          ds = p * (dp - s_D[lane]);
+        }
+#pragma unroll 4
+        for (int ii = 0; ii < kTile; ++ii) {
+          const float pi = __shfl_sync(0xffffffffu, p, ii);
+          const float dsi = __shfl_sync(0xffffffffu, ds, ii);
+#pragma unroll
+          for (int c = 0; c < VPL; ++c) dv_acc[kk][c] = fmaf(pi, s_do[ii][lane + 32 * c], dv_acc[kk][c]);
+#pragma unroll
+          for (int c = 0; c < KPL; ++c) dk_acc[kk][c] = fmaf(dsi, s_q[ii][lane + 32 * c], dk_acc[kk][c]);
+        }
+      }
+    }
+  }
+
+  T* dk = static_cast<T*>(a.grad_k);
+  T* dv = static_cast<T*>(a.grad_v);
+#pragma unroll
+  for (int kk = 0; kk < kKeysPerWarp; ++kk) {
+    const long long j = j0 + warp * kKeysPerWarp + kk;
+    if (j >= sk) continue;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c)
+      dk[((k0 + j) * a.hkv + g) * DK + lane + 32 * c] = from_float<T>(dk_acc[kk][c] * a.scale);
+#pragma unroll
+    for (int c = 0; c < VPL; ++c)
+      dv[((k0 + j) * a.hkv + g) * DV + lane + 32 * c] = from_float<T>(dv_acc[kk][c]);
+  }
+}
+
+// --- dQ: query-stationary ------------------------------------------------------------------
+constexpr int kRowsPerWarp = 2;
+constexpr int kBlockRows = kRowsPerWarp * kWarps;
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(kWarps * 32) bwd_dq_simt_kernel(const BwdArgs a) {
+  constexpr int KPL = DK / 32;
+  __shared__ float s_q[kBlockRows][DK];
+  __shared__ float s_do[kBlockRows][DV];
+  __shared__ float s_k[kTile][DK + 1];
+  __shared__ float s_v[kTile][DV + 1];
+
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
+  const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
+  const long long r0 = (long long)blockIdx.x * kBlockRows;
+  if (r0 >= sq) return;
+  const int g = h / (a.hq / a.hkv);
+  const T* q = static_cast<const T*>(a.q);
+  const T* kp = static_cast<const T*>(a.k);
+  const T* vp = static_cast<const T*>(a.v);
+  const T* dout = static_cast<const T*>(a.dout);
+
+  for (int idx = threadIdx.x; idx < kBlockRows * DK; idx += blockDim.x) {
+    const int r = idx / DK, c = idx % DK;
+    s_q[r][c] = (r0 + r < sq) ? to_float(q[((q0 + r0 + r) * a.hq + h) * DK + c]) : 0.f;
+  }
+  for (int idx = threadIdx.x; idx < kBlockRows * DV; idx += blockDim.x) {
+    const int r = idx / DV, c = idx % DV;
+    s_do[r][c] = (r0 + r < sq) ? to_float(dout[((q0 + r0 + r) * a.hq + h) * DV + c]) : 0.f;
+  }
+  float lt[kRowsPerWarp], Dr[kRowsPerWarp], acc[kRowsPerWarp][KPL];
+#pragma unroll
+  for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+    const long long i = r0 + warp * kRowsPerWarp + rr;
+    lt[rr] = (i < sq) ? a.lse_tot[(long long)h * a.total_q + q0 + i] : 0.f;
+    Dr[rr] = (i < sq) ? a.D[(long long)h * a.total_q + q0 + i] : 0.f;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) acc[rr][c] = 0.f;
+  }
+  const long long r_last = (r0 + kBlockRows < sq ? r0 + kBlockRows : sq) - 1;
+  long long lo0, hi0, lo1, hi1;
+  row_key_range(r0, sq, sk, a.left, a.right, lo0, hi0);
+  row_key_range(r_last, sq, sk, a.left, a.right, lo1, hi1);
+  const long long lo = lo0 < lo1 ? lo0 : lo1;
+  const long long hi = hi0 > hi1 ? hi0 : hi1;
+
+  for (long long t0 = lo; t0 < hi; t0 += kTile) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < kTile * DK; idx += blockDim.x) {
+      const int j = idx / DK, c = idx % DK;
+      s_k[j][c] = (t0 + j < hi) ? to_float(kp[((k0 + t0 + j) * a.hkv + g) * DK + c]) : 0.f;
+    }
+    for (int idx = threadIdx.x; idx < kTile * DV; idx += blockDim.x) {
+      const int j = idx / DV, c = idx % DV;
+      s_v[j][c] = (t0 + j < hi) ? to_float(vp[((k0 + t0 + j) * a.hkv + g) * DV + c]) : 0.f;
+    }
+    __syncthreads();
+    const long long j = t0 + lane;
+#pragma unroll
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+      const int r = warp * kRowsPerWarp + rr;
+      const long long i = r0 + r;
+      if (i >= sq) continue;
+      const bool vis = (j < hi) && visible(i, j, sq, sk, a.left, a.right);
+      float ds = 0.f;
+      if (vis) {
+        float s = 0.f, dp = 0.f;
+#pragma unroll 8
+        for (int c = 0; c < DK; ++c) s = fmaf(s_q[r][c], s_k[lane][c], s);
+#pragma unroll 8
+        for (int c = 0; c < DV; ++c) dp = fmaf(s_do[r][c], s_v[lane][c], dp);
+        const float p = __expf(s * a.scale - lt[rr]);
+        ds = p * (dp - Dr[rr]);
+      }
+#pragma unroll 4
+      for (int jj = 0; jj < kTile; ++jj) {
+        const float dsj = __shfl_sync(0xffffffffu, ds, jj);
+#pragma unroll
+        for (int c = 0; c < KPL; ++c) acc[rr][c] = fmaf(dsj, s_k[jj][lane + 32 * c], acc[rr][c]);
+      }
+    }
+  }
+  T* dq = static_cast<T*>(a.grad_q);
+#pragma unroll
+  for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+    const long long i = r0 + warp * kRowsPerWarp + rr;
+    if (i >= sq) continue;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c)
+      dq[((q0 + i) * a.hq + h) * DK + lane + 32 * c] = from_float<T>(acc[rr][c] * a.scale);
+  }
+}
+
+// Every key row of every sequence is written by the dk/dv pass (zeros where no query sees
+// it) and every query row by the dq pass, so no output needs clearing first.
+template <typename T, int DK, int DV>
+cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
+  cudaError_t e;
+  dim3 g1((a.max_sk + kBlockKeys - 1) / kBlockKeys, a.hkv, a.batch);
+  bwd_dkdv_simt_kernel<T, DK, DV><<<g1, kWarps * 32, 0, s>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  dim3 g2((a.max_sq + kBlockRows - 1) / kBlockRows, a.hq, a.batch);
+  bwd_dq_simt_kernel<T, DK, DV><<<g2, kWarps * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch_dims(const BwdArgs& a, cudaStream_t s) {
+#define ATTN_SINK_BWD_CASE(DK_, DV_) \
+  if (a.dk == DK_ && a.dv == DV_) return launch_typed<T, DK_, DV_>(a, s);
+  ATTN_SINK_BWD_CASE(64, 32)
+  ATTN_SINK_BWD_CASE(64, 64)
+  ATTN_SINK_BWD_CASE(64, 128)
+  ATTN_SINK_BWD_CASE(128, 32)
+  ATTN_SINK_BWD_CASE(128, 64)
+  ATTN_SINK_BWD_CASE(128, 128)
+#undef ATTN_SINK_BWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s) {
+  cudaError_t e;
+  if (a.dsink && (e = cudaMemsetAsync(a.dsink, 0, sizeof(float) * a.hq, s)) != cudaSuccess) return e;
+  dim3 grid((a.total_q + 63) / 64, a.hq);
+  if (dtype == 1)
+    bwd_preprocess_kernel<float><<<grid, 256, 0, s>>>(a);
+  else
+    bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_simt(const BwdArgs& a, int dtype, cudaStream_t s) {
+  cudaError_t e = launch_bwd_preprocess(a, dtype, s);
+  if (e != cudaSuccess) return e;
+  return dtype == 1 ? dispatch_dims<float>(a, s) : dispatch_dims<__nv_bfloat16>(a, s);
+}
+
+}  // namespace attn_sink

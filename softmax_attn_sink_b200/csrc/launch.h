@@ -1,0 +1,85 @@
+// Internal launcher interface between the C-ABI host code and the kernels.
+// Not part of the public ABI (that is include/attn_sink.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace attn_sink {
+
+// A window side at or above this value is unbounded.
+constexpr int kUnbounded = 1 << 30;
+
+// Bits of the per-device status word.
+constexpr unsigned kStatusTimeout = 1u;
+
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* cu_q;   // nullptr in decode mode: sequence b owns exactly q row b
+  const int32_t* cu_k;
+  const float* sink;     // nullptr = -inf
+  void* out;
+  float* lse;            // may be nullptr
+  int batch, total_q, total_k, max_sq, max_sk, hq, hkv, dk, dv;
+  float scale;
+  int left, right;       // effective window (causal folded into right), kUnbounded = none
+  unsigned* status;
+};
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* out;
+  const void* dout;
+  const float* lse;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const float* sink;
+  void* grad_q;          // dq [total_q, hq, dk]
+  void* grad_k;          // dk [total_k, hkv, dk]
+  void* grad_v;          // dv [total_k, hkv, dv]
+  float* dsink;          // may be nullptr
+  float* D;              // workspace [hq, total_q]: rowsum(dout * out)
+  float* lse_tot;        // workspace [hq, total_q]: logaddexp(lse, sink)
+  float* dq_acc;         // workspace [total_q, hq, dk] fp32 (tensor-core path only)
+  int batch, total_q, total_k, max_sq, max_sk, hq, hkv, dk, dv;
+  float scale;
+  int left, right;
+  unsigned* status;
+};
+
+struct DecodeArgs {
+  const void* q;         // [batch, hq, dk]
+  const void* k;
+  const void* v;
+  const int32_t* cu_k;
+  const float* sink;
+  void* out;             // [batch, hq, dv]
+  float* lse;            // [hq, batch] or nullptr
+  float* part_o;         // workspace [batch, hq, splits, dv]
+  float* part_ml;        // workspace [batch, hq, splits, 2] (max, sum)
+  int batch, total_k, max_sk, hq, hkv, dk, dv, splits;
+  float scale;
+  int left, right;
+  unsigned* status;
+};
+
+// dtype: 0 = bf16, 1 = fp32.  Each returns cudaSuccess or the launch error.
+cudaError_t launch_fwd_simt(const FwdArgs& a, int dtype, cudaStream_t s);
+bool fwd_sm100_supported(const FwdArgs& a, int dtype);
+cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s);
+
+// D, lse_tot and dsink (dsink cleared first); shared by both backward paths.
+cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_bwd_simt(const BwdArgs& a, int dtype, cudaStream_t s);
+bool bwd_sm100_supported(const BwdArgs& a, int dtype);
+cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s);
+
+cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
+bool decode_split_supported(int dk, int dv, int dtype);
+
+}  // namespace attn_sink

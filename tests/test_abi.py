@@ -1,0 +1,116 @@
+"""The C ABI: the library loads, exports every function include/attn_sink.h declares, and
+rejects bad arguments on the host before touching the GPU.  CPU only (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import softmax_attn_sink_b200 as sab
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_sink.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_sink_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = sab.lib()
+    declared = _declared_functions()
+    assert "attn_sink_fwd" in declared and "attn_sink_bwd" in declared and "attn_sink_decode" in declared
+    for name in declared:
+        assert hasattr(L, name), f"{name} declared in attn_sink.h but not exported"
+    assert set(sab._SYMBOLS) <= set(declared)
+
+
+def test_params_struct_matches_header_field_order():
+    text = open(HEADER).read()
+    body = re.search(r"typedef struct \{(.*?)\} attn_sink_params;", text, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\b([a-z_]+)\s*[;,]", body)
+    assert names == [f[0] for f in sab.AttnSinkParams._fields_]
+
+
+def test_status_strings_and_version():
+    L = sab.lib()
+    assert L.attn_sink_status_string(0) == b"ok"
+    assert b"workspace" in L.attn_sink_status_string(3)
+    assert L.attn_sink_status_string(99) == b"unknown status"
+    assert L.attn_sink_version() == 0x000100
+
+
+def _params(**kw):
+    base = dict(batch=2, total_q=64, total_k=64, max_seqlen_q=32, max_seqlen_k=32, num_heads_q=8,
+                num_heads_kv=2, head_dim_qk=128, head_dim_v=128, softmax_scale=0.088,
+                causal=True, window_left=-1, window_right=-1, dtype=sab.ATTN_SINK_BF16)
+    base.update(kw)
+    return sab.make_params(**base)
+
+
+SIZE_MAX = ctypes.c_size_t(-1).value
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(num_heads_kv=3), 1), (dict(batch=0), 1), (dict(total_q=0), 1),
+    (dict(head_dim_qk=96), 2), (dict(head_dim_v=256), 2), (dict(dtype=7), 2),
+    (dict(window_left=-2), 1), (dict(softmax_scale=float("inf")), 1),
+    (dict(max_seqlen_q=0), 1), (dict(max_seqlen_k=65), 1),
+])
+def test_invalid_params_rejected_on_host(bad, status):
+    L = sab.lib()
+    p = _params(**bad)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    st = L.attn_sink_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, None, None, 0, None)
+    assert st == status
+    assert L.attn_sink_fwd_workspace_size(ctypes.byref(p)) == SIZE_MAX
+
+
+def test_null_and_misaligned_pointers_rejected():
+    L = sab.lib()
+    p = _params()
+    a = 1 << 20
+    assert L.attn_sink_fwd(ctypes.byref(p), None, a, a, a, a, None, a, None, None, 0, None) == 1
+    assert L.attn_sink_fwd(ctypes.byref(p), a + 2, a, a, a, a, None, a, None, None, 0, None) == 1
+    assert L.attn_sink_bwd(ctypes.byref(p), a, a, a, a, a, None, a, a, None, a, a, a, None,
+                           None, 0, None) == 1  # lse is required
+
+
+def test_bwd_workspace_is_required_and_sized():
+    L = sab.lib()
+    p = _params()
+    need = L.attn_sink_bwd_workspace_size(ctypes.byref(p))
+    # D + lse_tot (fp32 [Hq, T_q] each) + fp32 dQ accumulator [T_q, Hq, dk]
+    assert need >= 2 * 8 * 64 * 4 + 64 * 8 * 128 * 4
+    a = 1 << 20
+    st = L.attn_sink_bwd(ctypes.byref(p), a, a, a, a, a, a, a, a, None, a, a, a, None, a, need - 256, None)
+    assert st == 3
+    st = L.attn_sink_bwd(ctypes.byref(p), a, a, a, a, a, a, a, a, None, a, a, a, None, None, 0, None)
+    assert st == 3
+
+
+def test_decode_params_and_workspace():
+    L = sab.lib()
+    p = _params(total_q=2, max_seqlen_q=1, total_k=40000, max_seqlen_k=30000)
+    n = L.attn_sink_decode_num_splits(ctypes.byref(p))
+    assert 1 <= n <= 1024
+    ws = L.attn_sink_decode_workspace_size(ctypes.byref(p), 0)
+    assert ws == L.attn_sink_decode_workspace_size(ctypes.byref(p), n)
+    assert ws >= 2 * 8 * n * (128 + 2) * 4
+    # decode needs total_q == batch and max_seqlen_q == 1
+    bad = _params(total_q=3, max_seqlen_q=1)
+    assert L.attn_sink_decode_workspace_size(ctypes.byref(bad), 0) == SIZE_MAX
+    a = 1 << 20
+    assert L.attn_sink_decode(ctypes.byref(p), a, a, a, a, None, -1, a, None, None, 0, None) == 1
+    assert L.attn_sink_decode(ctypes.byref(p), a, a, a, a, None, 4, a, None, None, 0, None) == 3
+
+
+def test_python_binding_requires_cuda_tensors():
+    import torch
+    q = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        sab.attn_sink_fwd(q, q, q, cu, cu, 4, 4)

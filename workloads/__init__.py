@@ -36,11 +36,18 @@ import numpy as np
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    bits = x.view(np.uint32).astype(np.uint64)
-    bits = ((bits + 0x7FFF + ((bits >> 16) & 1)) >> 16) << 16
-    return bits.astype(np.uint32).view(np.float32)
+    """Round finite float32 values to the nearest bf16 (ties to even); returns float32.
+
+    Works on the bit pattern in place: add 0x7FFF plus the lowest kept bit, then clear the
+    16 dropped bits.  For finite inputs the sum cannot overflow 32 bits."""
+    out = np.array(x, dtype=np.float32, copy=True, order="C")
+    bits = out.view(np.uint32)
+    lsb = bits >> 16
+    lsb &= 1
+    lsb += 0x7FFF
+    bits += lsb
+    bits &= np.uint32(0xFFFF0000)
+    return out
 
 
 @dataclass
