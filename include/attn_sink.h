@@ -136,6 +136,30 @@ int attn_sink_decode(const attn_sink_params* params, const void* q, const void* 
                      float* lse, void* workspace, size_t workspace_bytes,
                      attn_sink_stream_t stream);
 
+/*
+ * Decode that allocates nothing and takes no workspace.  None of the pages this library
+ * follows has a counterpart: it exists for callers that cannot allocate device memory
+ * (a plugin or custom-op host that passes only the call's tensors and offers no
+ * allocator, a process whose device memory is all held by another framework's pool, or a
+ * latency-critical loop that must not allocate).  Same arguments, results and kernels as
+ * attn_sink_decode, minus the workspace: the chunk partials live in a fixed 16 MiB
+ * device array inside the library, present on every GPU that loads the library until the
+ * process exits.  No cudaMalloc, cudaFree or other allocating routine is called.
+ *   - num_splits == 0 picks the automatic split count, lowered until the partials fit in
+ *     16 MiB; an explicit num_splits whose partials need more than 16 MiB, or a problem
+ *     that does not fit even with one split, returns ATTN_SINK_ERR_WORKSPACE before any
+ *     launch.
+ *   - The first call on each device looks up the array's device address (a
+ *     cudaGetSymbolAddress with that device current) and caches it; make that first call
+ *     before capturing any stream.
+ *   - All calls share the one array and it keeps the last call's contents.  Nothing in
+ *     it has to start at zero (each call writes every slot it later reads), but calls
+ *     whose kernels overlap on the GPU race on it: order them on one stream.
+ */
+int attn_sink_decode_noalloc(const attn_sink_params* params, const void* q, const void* k,
+                             const void* v, const int32_t* cu_seqlens_k, const float* sink,
+                             int num_splits, void* out, float* lse, attn_sink_stream_t stream);
+
 /* Workspace bytes each entry point needs for `params` (0 = none; SIZE_MAX = params invalid). */
 size_t attn_sink_fwd_workspace_size(const attn_sink_params* params);
 size_t attn_sink_bwd_workspace_size(const attn_sink_params* params);
