@@ -1,9 +1,431 @@
-// Tensor-core (tcgen05) sink-attention backward for sm_100a.
-#include "common.cuh"
+// Sink-attention backward on the sm_100a tensor cores (bf16 in, fp32 accumulation).
+//
+// Gradient of the sink forward for the loss sum(dout * out).  With lse_tot =
+// logaddexp(lse, sink) (from the preprocess pass) the probabilities are
+// P_ij = e^{S_ij - lse_tot_i}; then dS = P * (dout V^T - D) with D_i = dout_i . out_i,
+// dq = scale dS K, dk = scale dS^T Q, dv = P^T dout.  slime's learnable_softmax_attention.py
+// writes the same gradient as dS = P_van * s * (D - s * di) with s = sigmoid(lse - offset)
+// (class docstring); P = s P_van and D_i = s di make the two forms equal.
+//
+// One CTA owns a 128-key tile of one (sequence, kv head) and loops over every q head of
+// the GQA group and every 128-query tile that can see those keys, so dK and dV
+// accumulate in TMEM with no atomics.  Per query tile t:
+//   S^T  = K Q^T        (M = keys, N = queries)        -> TMEM R0
+//   dP^T = V dout^T                                    -> TMEM R1
+//   compute warps (thread = key row): P^T = 2^{S^T scale log2e - lse_tot log2e} (masked),
+//     dS^T = P^T (dP^T - D); P^T as bf16 back into R0 (TMEM A operand), dS^T as bf16 into
+//     a 128-byte-swizzled shared tile
+//   dV += P^T dout      (A = P^T from TMEM, B = dout MN-major)
+//   dK += dS^T Q        (A = dS^T K-major from shared memory, B = Q MN-major)
+//   dQ_t = dS K         (A = the same dS^T tile read MN-major, B = K MN-major) -> TMEM R1
+//   dQ warps (thread = query row) read dQ_t and add scale * dQ_t into an fp32 workspace
+//     with vector atomics; a final pass converts it to bf16.
+// TMEM columns: dK [0,128) dV [128,256) R0 [256,384) R1 [384,512).
+// The next tile's S^T overwrites R0, which the dV MMA reads as P^T: the MMA thread waits
+// for a commit of that dV MMA first (it is issued ahead of dK and dQ, so the tensor pipe
+// stays busy meanwhile).  All mbarrier waits are bounded.
+#include <cuda.h>
+
+#include "sm100_ptx.cuh"
 
 namespace attn_sink {
 
-bool bwd_sm100_supported(const BwdArgs&, int) { return false; }
-cudaError_t launch_bwd_sm100(const BwdArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBN = 128;  // keys per CTA
+constexpr int kBM = 128;  // queries per inner tile
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColDK = 0, kColDV = 128, kColR0 = 256, kColR1 = 384;
+
+template <int DK, int DV>
+struct BLayout {
+  static constexpr int KH = DK / 64, VH = DV / 64;
+  static constexpr int kHalf = 128 * 128;                  // 128 rows x 128 bytes
+  static constexpr int kKBytes = KH * kHalf, kVBytes = VH * kHalf;
+  static constexpr int kQBytes = KH * kHalf, kOBytes = VH * kHalf;
+  static constexpr int kDSBytes = 2 * kHalf;               // 128 keys x 128 queries bf16
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKBytes;
+  static constexpr int kOffQ = kOffV + kVBytes;            // 2 stages
+  static constexpr int kOffO = kOffQ + 2 * kQBytes;        // 2 stages (dout)
+  static constexpr int kOffDS = kOffO + 2 * kOBytes;
+  static constexpr int kOffBar = kOffDS + kDSBytes;
+  static constexpr int kNumBars = 12;
+  static constexpr int kOffSlot = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffSlot + 16 + 1024;
+};
+
+struct BBars {
+  uint32_t base;
+  __device__ __forceinline__ uint32_t kv_full() const { return base; }
+  __device__ __forceinline__ uint32_t qd_full(int s) const { return base + 8u * (1 + s); }
+  __device__ __forceinline__ uint32_t qd_empty(int s) const { return base + 8u * (3 + s); }
+  __device__ __forceinline__ uint32_t sdp_full() const { return base + 8u * 5; }
+  __device__ __forceinline__ uint32_t compute_done() const { return base + 8u * 6; }
+  __device__ __forceinline__ uint32_t dv_done() const { return base + 8u * 7; }
+  __device__ __forceinline__ uint32_t dq_full() const { return base + 8u * 8; }
+  __device__ __forceinline__ uint32_t dq_free() const { return base + 8u * 9; }
+  __device__ __forceinline__ uint32_t ds_free() const { return base + 8u * 10; }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * 11; }
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do) {
+  using L = BLayout<DK, DV>;
+  extern __shared__ unsigned char smem_raw[];
+
+  // ---- work unit: key tile nt of (sequence b, kv head g); tile 0 (most queries) first --
+  const int g = blockIdx.x, b = blockIdx.y, nt = blockIdx.z;
+  const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
+  const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
+  const long long n0 = (long long)nt * kBN;
+  if (n0 >= sk) return;
+  const int group = a.hq / a.hkv;
+  const long long nkeys = (sk - n0 < kBN) ? sk - n0 : kBN;
+  long long qlo, qhi, qlo1, qhi1;
+  key_query_range(n0, sq, sk, a.left, a.right, qlo, qhi);
+  key_query_range(n0 + nkeys - 1, sq, sk, a.left, a.right, qlo1, qhi1);
+  qhi = qhi1;  // query ranges move right with the key, so the union is [qlo(first), qhi(last))
+  const int n_m = qhi > qlo ? (int)((qhi - qlo + kBM - 1) / kBM) : 0;
+  const int T = n_m * group;
+
+  const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
+  const uint32_t sK = base_u32 + L::kOffK, sV = base_u32 + L::kOffV, sQ = base_u32 + L::kOffQ,
+                 sO = base_u32 + L::kOffO, sDS = base_u32 + L::kOffDS;
+  const BBars bar{base_u32 + L::kOffBar};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar.kv_full(), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar.qd_full(s), 1);
+      mbar_init(bar.qd_empty(s), 1);
+    }
+    mbar_init(bar.sdp_full(), 1);
+    mbar_init(bar.compute_done(), 4);
+    mbar_init(bar.dv_done(), 1);
+    mbar_init(bar.dq_full(), 1);
+    mbar_init(bar.dq_free(), 4);
+    mbar_init(bar.ds_free(), 1);
+    mbar_init(bar.drain(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto head_of = [&](int t) { return g * group + t / n_m; };
+  auto qbase_of = [&](int t) { return qlo + (long long)(t % n_m) * kBM; };
+
+  if (warp == 0) {
+    // ================================ TMA producer ======================================
+    if (lane == 0 && T > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(bar.kv_full(), L::kKBytes + L::kVBytes);
+      for (int hf = 0; hf < L::KH; ++hf)
+        tma_load_3d(sK + hf * L::kHalf, &tm_k, bar.kv_full(), hf * 64, g, (int)(k0 + n0));
+      for (int hf = 0; hf < L::VH; ++hf)
+        tma_load_3d(sV + hf * L::kHalf, &tm_v, bar.kv_full(), hf * 64, g, (int)(k0 + n0));
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t & 1;
+        if (!mbar_wait(bar.qd_empty(st), ((t >> 1) & 1) ^ 1, a.status)) break;
+        const int h = head_of(t);
+        const int row = (int)(q0 + qbase_of(t));
+        mbar_arrive_expect_tx(bar.qd_full(st), L::kQBytes + L::kOBytes);
+        for (int hf = 0; hf < L::KH; ++hf)
+          tma_load_3d(sQ + st * L::kQBytes + hf * L::kHalf, &tm_q, bar.qd_full(st), hf * 64, h, row);
+        for (int hf = 0; hf < L::VH; ++hf)
+          tma_load_3d(sO + st * L::kOBytes + hf * L::kHalf, &tm_do, bar.qd_full(st), hf * 64, h, row);
+        issued = t + 1;
+      }
+      mbar_wait(bar.kv_full(), 0, a.status);
+      for (int t = issued - 2 < 0 ? 0 : issued - 2; t < issued; ++t)
+        mbar_wait(bar.qd_full(t & 1), (t >> 1) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    // ================================ MMA issuer =========================================
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t id_s = idesc_bf16(kBN, kBM, 0, 0);   // S^T, dP^T: K-major A and B
+      constexpr uint32_t id_dv = idesc_bf16(kBN, DV, 0, 1);   // A from TMEM, B = dout MN-major
+      constexpr uint32_t id_dk = idesc_bf16(kBN, DK, 0, 1);   // A = dS^T K-major, B = Q MN-major
+      constexpr uint32_t id_dq = idesc_bf16(kBM, DK, 1, 1);   // A = dS MN-major, B = K MN-major
+      bool ok = mbar_wait(bar.kv_full(), 0, a.status);
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t & 1;
+        const uint32_t q_s = sQ + st * L::kQBytes, o_s = sO + st * L::kOBytes;
+        ok = mbar_wait(bar.qd_full(st), (t >> 1) & 1, a.status);
+        if (ok && t >= 1) ok = mbar_wait(bar.dv_done(), (t - 1) & 1, a.status);   // R0 free
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
+          mma_ss(tmem + kColR0, smem_desc(sK + off, 16, 1024, kLayoutSwizzle128B),
+                 smem_desc(q_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
+        }
+        if (t >= 1 && !(ok = mbar_wait(bar.dq_free(), (t - 1) & 1, a.status))) break;   // R1 free
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DV / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
+          mma_ss(tmem + kColR1, smem_desc(sV + off, 16, 1024, kLayoutSwizzle128B),
+                 smem_desc(o_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
+        }
+        mma_commit(bar.sdp_full());
+        if (!(ok = mbar_wait(bar.compute_done(), t & 1, a.status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk)
+          mma_ts(tmem + kColDV, tmem + kColR0 + kk * 8,
+                 smem_desc(o_s + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dv, (t > 0 || kk > 0));
+        mma_commit(bar.dv_done());
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk)
+          mma_ss(tmem + kColDK, smem_desc(sDS + (kk >> 2) * L::kHalf + (kk & 3) * 32, 16, 1024, kLayoutSwizzle128B),
+                 smem_desc(q_s + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dk, (t > 0 || kk > 0));
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ss(tmem + kColR1, smem_desc(sDS + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B),
+                 smem_desc(sK + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dq, kk > 0);
+        mma_commit(bar.dq_full());
+        mma_commit(bar.ds_free());
+        mma_commit(bar.qd_empty(st));
+      }
+      mma_commit(bar.drain());
+      mbar_wait(bar.drain(), 0, a.status);
+    }
+  } else if (warp < 6) {
+    // ================================ compute warps (thread = key row) ===================
+    const int lg = warp & 3;
+    const int r = lg * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    const long long j = n0 + r;                       // key index in the sequence
+    const bool key_ok = j < sk;
+    const float scale2 = a.scale * kLog2e;
+    const long long off = sk - sq;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int h = head_of(t);
+      const long long i0 = qbase_of(t);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.sdp_full(), t & 1, a.status))) { ok = false; break; }
+      if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar.ds_free(), (t - 1) & 1, a.status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* lt_row = a.lse_tot + (long long)h * a.total_q + q0;
+      const float* D_row = a.D + (long long)h * a.total_q + q0;
+#pragma unroll 1
+      for (int c = 0; c < kBM / 32; ++c) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tmem + lane_off + kColR0 + c * 32, sv);
+        tmem_ld32(tmem + lane_off + kColR1 + c * 32, dpv);
+        tmem_wait_ld();
+        uint32_t pk[16], dk_[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pp[2], dd[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const long long qi = i0 + c * 32 + e + u;
+            bool vis = key_ok && qi < sq;
+            const long long d = j - (qi + off);       // key offset from the query's diagonal
+            if (a.right < kUnbounded) vis = vis && d <= a.right;
+            if (a.left < kUnbounded) vis = vis && d >= -(long long)a.left;
+            float p = 0.f, ds = 0.f;
+            if (vis) {
+              const float lt = __ldg(lt_row + qi);
+              p = ex2(fmaf(__uint_as_float(sv[e + u]), scale2, -lt * kLog2e));
+              ds = p * (__uint_as_float(dpv[e + u]) - __ldg(D_row + qi));
+            }
+            pp[u] = p;
+            dd[u] = ds;
+          }
+          pk[e >> 1] = pack_bf16x2(pp[0], pp[1]);
+          dk_[e >> 1] = pack_bf16x2(dd[0], dd[1]);
+        }
+        // P^T chunk -> TMEM R0 (its S^T columns were already read)
+        tmem_st16(tmem + lane_off + kColR0 + c * 16, pk);
+        // dS^T chunk -> shared tile, row r, queries [32c, 32c + 32): 4 swizzled 16-byte chunks
+        const uint32_t half = sDS + (c >> 1) * L::kHalf + r * 128;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int ch = (c & 1) * 4 + v;
+          st_shared_v4(half + ((ch ^ (r & 7)) << 4), dk_[4 * v], dk_[4 * v + 1], dk_[4 * v + 2], dk_[4 * v + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.compute_done());
+    }
+    // ---- epilogue: dK = scale * acc, dV = acc, bf16, this thread's key row -----------------
+    const bool have = __all_sync(0xffffffffu, ok && T > 0 && mbar_wait(bar.ds_free(), (T - 1) & 1, a.status));
+    tc_fence_after();
+    __nv_bfloat16* dkp = static_cast<__nv_bfloat16*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
+    __nv_bfloat16* dvp = static_cast<__nv_bfloat16*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int ncol = pass == 0 ? DK : DV;
+      const uint32_t col = pass == 0 ? kColDK : kColDV;
+      const float mul = pass == 0 ? a.scale : 1.f;
+      uint4* dst = reinterpret_cast<uint4*>(pass == 0 ? dkp : dvp);
+      for (int c = 0; c < ncol / 32; ++c) {
+        uint32_t v[32];
+        if (T > 0) {
+          tmem_ld32(tmem + lane_off + col + c * 32, v);
+          tmem_wait_ld();
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = (T > 0 && have) ? __uint_as_float(v[2 * e]) * mul : 0.f;
+          const float x1 = (T > 0 && have) ? __uint_as_float(v[2 * e + 1]) * mul : 0.f;
+          pk[e] = pack_bf16x2(x0, x1);
+        }
+        if (key_ok) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dst[c * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+    }
+  } else {
+    // ================================ dQ warps (thread = query row) =======================
+    const int lg = warp & 3;
+    const int r = lg * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    for (int t = 0; t < T; ++t) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.dq_full(), t & 1, a.status))) break;
+      tc_fence_after();
+      uint32_t v[DK];
+#pragma unroll
+      for (int c = 0; c < DK / 32; ++c) {
+        uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]);
+        tmem_ld32(tmem + lane_off + kColR1 + c * 32, chunk);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.dq_free());
+      const long long qi = qbase_of(t) + r;
+      if (qi < sq) {
+        float* dst = a.dq_acc + ((q0 + qi) * a.hq + head_of(t)) * DK;
+#pragma unroll
+        for (int e = 0; e < DK; e += 4)
+          red_add_v4(dst + e, __uint_as_float(v[e]) * a.scale, __uint_as_float(v[e + 1]) * a.scale,
+                     __uint_as_float(v[e + 2]) * a.scale, __uint_as_float(v[e + 3]) * a.scale);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// dq = bf16(dq_acc), 8 elements per thread
+__global__ void dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 x = reinterpret_cast<const float4*>(acc)[2 * i];
+  const float4 y = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  uint4 o;
+  o.x = pack_bf16x2(x.x, x.y);
+  o.y = pack_bf16x2(x.z, x.w);
+  o.z = pack_bf16x2(y.x, y.y);
+  o.w = pack_bf16x2(y.z, y.w);
+  reinterpret_cast<uint4*>(dq)[i] = o;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, heads, d] bf16 as a 3-D tensor; boxes of 128 rows x 1 head x 64 columns, 128B swizzle.
+bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * heads};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK, int DV>
+cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
+  using L = BLayout<DK, DV>;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map(&tq, a.q, DK, a.hq, a.total_q) || !make_map(&tk, a.k, DK, a.hkv, a.total_k) ||
+      !make_map(&tv, a.v, DV, a.hkv, a.total_k) || !make_map(&to, a.dout, DV, a.hq, a.total_q))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * DK * sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  if ((e = launch_bwd_preprocess(a, 0, s)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(bwd_sm100_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) !=
+      cudaSuccess)
+    return e;
+  dim3 grid(a.hkv, a.batch, (a.max_sk + kBN - 1) / kBN);
+  bwd_sm100_kernel<DK, DV><<<grid, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const long long n8 = (long long)a.total_q * a.hq * DK / 8;
+  dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q),
+                                                                 n8);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bwd_sm100_supported(const BwdArgs& a, int dtype) {
+  if (dtype != 0 || a.dq_acc == nullptr) return false;
+  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
+  if (a.batch > 65535 || (a.max_sk + kBN - 1) / kBN > 65535 || a.hkv > 65535) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s) {
+  if (a.dk == 128 && a.dv == 128) return launch_typed<128, 128>(a, s);
+  if (a.dk == 128 && a.dv == 64) return launch_typed<128, 64>(a, s);
+  if (a.dk == 64 && a.dv == 64) return launch_typed<64, 64>(a, s);
+  if (a.dk == 64 && a.dv == 128) return launch_typed<64, 128>(a, s);
+  return cudaErrorInvalidValue;
+}
 
 }  // namespace attn_sink

@@ -90,6 +90,10 @@ BWD_CASES = [
     ("full_noncausal", [200], [170], 2, 2, 128, 128, False, -1, -1, "uniform", "bf16"),
     ("dk64_dv32", [150, 90], [160, 90], 2, 1, 64, 32, True, 40, 0, "normal", "bf16"),
     ("no_sink", [190], [190], 2, 2, 128, 64, True, -1, -1, None, "bf16"),
+    ("dk64_dv64_gqa", [300, 131], [300, 131], 4, 1, 64, 64, True, -1, -1, "normal", "bf16"),
+    ("dk64_dv128", [257], [300], 2, 2, 64, 128, True, -1, -1, "uniform", "bf16"),
+    ("gqa4_long_window", [700, 300], [700, 300], 8, 2, 128, 128, True, 200, 0, "normal", "bf16"),
+    ("neg_inf_sink_masked_rows", [5, 260], [2, 260], 4, 2, 128, 128, True, -1, -1, "neg_inf", "bf16"),
     ("fp32_gqa", [70, 33], [80, 33], 4, 2, 128, 64, True, -1, -1, "normal", "fp32"),
     ("fp32_window", [90], [90], 2, 2, 64, 64, False, 10, 5, "normal", "fp32"),
 ]
