@@ -282,6 +282,11 @@ def bench_fwd_bwd(args, world, peaks, peak_kind):
     import torch
     import softmax_attn_sink_b200 as sab
     p = W.config3()
+    if args.seqs < 4:  # a smaller case of the same kernels (for profiler captures)
+        t = 8192 * args.seqs
+        p.q, p.k, p.v, p.dout = p.q[:t], p.k[:t], p.v[:t], p.dout[:t]
+        p.cu_seqlens_q = p.cu_seqlens_q[:args.seqs + 1].copy()
+        p.cu_seqlens_k = p.cu_seqlens_q.copy()
     td = torch.bfloat16
     q, k, v, do = (torch.from_numpy(x).to(td).cuda() for x in (p.q, p.k, p.v, p.dout))
     cu = torch.from_numpy(p.cu_seqlens_q).cuda()
@@ -303,7 +308,7 @@ def bench_fwd_bwd(args, world, peaks, peak_kind):
     ba = bf / (statistics.mean(b_per) * 1e-3) / 1e12
     pk = peaks["bf16_tflops"]
     return {
-        "workload": "train4x8192_h16_d128_causal", "pairs": pairs, "steps": steps,
+        "workload": f"train{args.seqs}x8192_h16_d128_causal", "pairs": pairs, "steps": steps,
         "fwd": {"value": round(ff * world / (f_total / steps * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(f_total / steps, 4), "flops": ff,
                 "roofline": {"bound": "tensor", "achieved": round(fa, 2), "peak": pk,
@@ -428,6 +433,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["all", "fwd", "fwd_bwd", "decode"], default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqs", type=int, default=4, choices=[1, 2, 3, 4],
+                    help="sequences of the fwd_bwd leg (4 = the full training workload)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and args.workload == "all":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

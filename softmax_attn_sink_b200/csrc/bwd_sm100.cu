@@ -346,6 +346,376 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
   }
 }
 
+// ---- head dim 128: query tile in two 64-query halves, software-pipelined -----------------
+//
+// Same gradient as above.  Each 128-query tile is processed as two halves a/b so that the
+// tensor pipe works on one half while the compute warps work on the other:
+//   MMA order per tile t:  [wait compute_a] dV_a dK_a dQ^T_a  [wait compute_b]
+//                          S_a(t+1) dP_a(t+1)  dV_b dK_b dQ^T_b  S_b(t+1) dP_b(t+1)
+// dQ is produced transposed, dQ^T = K^T dS^T (M = head dim), so a dQ warp thread owns one
+// head-dim index and each warp-wide reduction covers 128 contiguous bytes of a dQ row.
+// TMEM: dK [0,128) dV [128,256) S_a [256,320) dP_a [320,384) S_b [384,448) dP_b [448,512);
+// P^T of a half is written over its S columns, dQ^T of a half over its dP columns.
+constexpr uint32_t kColSa = 256, kColDPa = 320, kColSb = 384, kColDPb = 448;
+
+template <int DV>
+struct PLayout {
+  static constexpr int DK = 128;
+  static constexpr int VH = DV / 64;
+  static constexpr int kHalf = 128 * 128;
+  static constexpr int kKBytes = 2 * kHalf, kVBytes = VH * kHalf;
+  static constexpr int kQBytes = 2 * kHalf, kOBytes = VH * kHalf;
+  static constexpr int kDSBytes = 2 * kHalf;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKBytes;
+  static constexpr int kOffQ = kOffV + kVBytes;
+  static constexpr int kOffO = kOffQ + 2 * kQBytes;
+  static constexpr int kOffDS = kOffO + 2 * kOBytes;
+  static constexpr int kOffLD = kOffDS + kDSBytes;         // lse_tot * log2e [128], D [128]
+  static constexpr int kOffBar = kOffLD + 1024;
+  static constexpr int kNumBars = 18;
+  static constexpr int kOffSlot = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffSlot + 16 + 1024;
+};
+
+struct PBars {
+  uint32_t base;
+  __device__ __forceinline__ uint32_t kv_full() const { return base; }
+  __device__ __forceinline__ uint32_t qd_full(int s) const { return base + 8u * (1 + s); }
+  __device__ __forceinline__ uint32_t qd_empty(int s) const { return base + 8u * (3 + s); }
+  __device__ __forceinline__ uint32_t sdp_full(int h) const { return base + 8u * (5 + h); }
+  __device__ __forceinline__ uint32_t compute_done(int h) const { return base + 8u * (7 + h); }
+  __device__ __forceinline__ uint32_t dv_done(int h) const { return base + 8u * (9 + h); }
+  __device__ __forceinline__ uint32_t dq_full(int h) const { return base + 8u * (11 + h); }
+  __device__ __forceinline__ uint32_t dq_free(int h) const { return base + 8u * (13 + h); }
+  __device__ __forceinline__ uint32_t ds_free(int h) const { return base + 8u * (15 + h); }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * 17; }
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_do) {
+  using L = PLayout<DV>;
+  constexpr int DK = 128;
+  extern __shared__ unsigned char smem_raw[];
+
+  const int g = blockIdx.x, b = blockIdx.y, nt = blockIdx.z;
+  const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
+  const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
+  const long long n0 = (long long)nt * kBN;
+  if (n0 >= sk) return;
+  const int group = a.hq / a.hkv;
+  const long long nkeys = (sk - n0 < kBN) ? sk - n0 : kBN;
+  long long qlo, qhi, qlo1, qhi1;
+  key_query_range(n0, sq, sk, a.left, a.right, qlo, qhi);
+  key_query_range(n0 + nkeys - 1, sq, sk, a.left, a.right, qlo1, qhi1);
+  qhi = qhi1;
+  const int n_m = qhi > qlo ? (int)((qhi - qlo + kBM - 1) / kBM) : 0;
+  const int T = n_m * group;
+
+  const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
+  const uint32_t sK = base_u32 + L::kOffK, sV = base_u32 + L::kOffV, sQ = base_u32 + L::kOffQ,
+                 sO = base_u32 + L::kOffO, sDS = base_u32 + L::kOffDS;
+  float* s_lt = reinterpret_cast<float*>(smem + L::kOffLD);
+  float* s_D = s_lt + 128;
+  const PBars bar{base_u32 + L::kOffBar};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar.kv_full(), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar.qd_full(s), 1);
+      mbar_init(bar.qd_empty(s), 1);
+      mbar_init(bar.sdp_full(s), 1);
+      mbar_init(bar.compute_done(s), 4);
+      mbar_init(bar.dv_done(s), 1);
+      mbar_init(bar.dq_full(s), 1);
+      mbar_init(bar.dq_free(s), 4);
+      mbar_init(bar.ds_free(s), 1);
+    }
+    mbar_init(bar.drain(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto head_of = [&](int t) { return g * group + t / n_m; };
+  auto qbase_of = [&](int t) { return qlo + (long long)(t % n_m) * kBM; };
+
+  if (warp == 0) {
+    // ================================ TMA producer ======================================
+    if (lane == 0 && T > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(bar.kv_full(), L::kKBytes + L::kVBytes);
+      for (int hf = 0; hf < 2; ++hf) tma_load_3d(sK + hf * L::kHalf, &tm_k, bar.kv_full(), hf * 64, g, (int)(k0 + n0));
+      for (int hf = 0; hf < L::VH; ++hf)
+        tma_load_3d(sV + hf * L::kHalf, &tm_v, bar.kv_full(), hf * 64, g, (int)(k0 + n0));
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t & 1;
+        if (!mbar_wait(bar.qd_empty(st), ((t >> 1) & 1) ^ 1, a.status)) break;
+        const int h = head_of(t);
+        const int row = (int)(q0 + qbase_of(t));
+        mbar_arrive_expect_tx(bar.qd_full(st), L::kQBytes + L::kOBytes);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_3d(sQ + st * L::kQBytes + hf * L::kHalf, &tm_q, bar.qd_full(st), hf * 64, h, row);
+        for (int hf = 0; hf < L::VH; ++hf)
+          tma_load_3d(sO + st * L::kOBytes + hf * L::kHalf, &tm_do, bar.qd_full(st), hf * 64, h, row);
+        issued = t + 1;
+      }
+      mbar_wait(bar.kv_full(), 0, a.status);
+      for (int t = issued - 2 < 0 ? 0 : issued - 2; t < issued; ++t)
+        mbar_wait(bar.qd_full(t & 1), (t >> 1) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    // ================================ MMA issuer =========================================
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t id_s = idesc_bf16(kBN, 64, 0, 0);    // S_h, dP_h: 128 keys x 64 queries
+      constexpr uint32_t id_dv = idesc_bf16(kBN, DV, 0, 1);   // P^T_h (TMEM) x dout_h (MN-major)
+      constexpr uint32_t id_dk = idesc_bf16(kBN, DK, 0, 1);   // dS^T_h (K-major) x Q_h (MN-major)
+      constexpr uint32_t id_dq = idesc_bf16(DK, 64, 1, 1);    // K^T (MN-major) x dS^T_h (MN-major)
+      // S_h(t) = K Q_h^T -> S columns; dP_h(t) = V dout_h^T -> dP columns
+      auto issue_sdp = [&](int t, int hh) -> bool {
+        const int st = t & 1;
+        const uint32_t q_s = sQ + st * L::kQBytes + hh * 8192, o_s = sO + st * L::kOBytes + hh * 8192;
+        const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
+        if (hh == 0 && !mbar_wait(bar.qd_full(st), (t >> 1) & 1, a.status)) return false;
+        if (t >= 1 && !mbar_wait(bar.dv_done(hh), (t - 1) & 1, a.status)) return false;   // P^T_h read
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
+          mma_ss(tmem + cS, smem_desc(sK + off, 16, 1024, kLayoutSwizzle128B),
+                 smem_desc(q_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
+        }
+        if (t >= 1 && !mbar_wait(bar.dq_free(hh), (t - 1) & 1, a.status)) return false;   // dQ^T_h read
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DV / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
+          mma_ss(tmem + cP, smem_desc(sV + off, 16, 1024, kLayoutSwizzle128B),
+                 smem_desc(o_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
+        }
+        mma_commit(bar.sdp_full(hh));
+        return true;
+      };
+      auto issue_grads = [&](int t, int hh) {
+        const int st = t & 1;
+        const uint32_t q_s = sQ + st * L::kQBytes, o_s = sO + st * L::kOBytes;
+        const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + kColDV, tmem + cS + kk * 8,
+                 smem_desc(o_s + (4 * hh + kk) * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dv,
+                 (t > 0 || hh > 0 || kk > 0));
+        mma_commit(bar.dv_done(hh));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + kColDK, smem_desc(sDS + hh * L::kHalf + kk * 32, 16, 1024, kLayoutSwizzle128B),
+                 smem_desc(q_s + (4 * hh + kk) * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dk,
+                 (t > 0 || hh > 0 || kk > 0));
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ss(tmem + cP, smem_desc(sK + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B),
+                 smem_desc(sDS + hh * L::kHalf + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dq, kk > 0);
+        mma_commit(bar.dq_full(hh));
+        mma_commit(bar.ds_free(hh));
+      };
+      bool ok = mbar_wait(bar.kv_full(), 0, a.status);
+      if (ok) ok = issue_sdp(0, 0) && issue_sdp(0, 1);
+      for (int t = 0; t < T && ok; ++t) {
+        if (!(ok = mbar_wait(bar.compute_done(0), t & 1, a.status))) break;
+        tc_fence_after();
+        issue_grads(t, 0);
+        if (!(ok = mbar_wait(bar.compute_done(1), t & 1, a.status))) break;
+        tc_fence_after();
+        if (t + 1 < T && !(ok = issue_sdp(t + 1, 0))) break;
+        issue_grads(t, 1);
+        mma_commit(bar.qd_empty(t & 1));
+        if (t + 1 < T && !(ok = issue_sdp(t + 1, 1))) break;
+      }
+      mma_commit(bar.drain());
+      mbar_wait(bar.drain(), 0, a.status);
+    }
+  } else if (warp < 6) {
+    // ================================ compute warps (thread = key row) ===================
+    const int lg = warp & 3;
+    const int r = lg * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    const long long j = n0 + r;
+    const bool key_ok = j < sk;
+    const float scale2 = a.scale * kLog2e;
+    const long long off = sk - sq;
+    bool ok = true;
+    // The two named barriers below are hardware waits with no time limit, so every compute
+    // warp passes both in every iteration: after a timed-out mbarrier wait a warp stops
+    // working (ok = false) but never leaves the loop.
+    for (int t = 0; t < T; ++t) {
+      const int h = head_of(t);
+      const long long i0 = qbase_of(t);
+      // stage lse_tot * log2e and D of this tile's 128 queries (all 128 compute threads)
+      named_bar_sync(1, 128);
+      {
+        const long long qi = i0 + r;
+        const bool qok = qi < sq;
+        s_lt[r] = qok ? a.lse_tot[(long long)h * a.total_q + q0 + qi] * kLog2e : 0.f;
+        s_D[r] = qok ? a.D[(long long)h * a.total_q + q0 + qi] : 0.f;
+      }
+      named_bar_sync(1, 128);
+#pragma unroll 1
+      for (int hh = 0; hh < 2 && ok; ++hh) {
+        const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.sdp_full(hh), t & 1, a.status))) { ok = false; break; }
+        if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar.ds_free(hh), (t - 1) & 1, a.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // every (key, query) pair of this half visible?  (then skip the per-element mask)
+        const long long qa = i0 + 64 * hh;
+        bool full = (nkeys == kBN) && (qa + 63 < sq);
+        if (a.right < kUnbounded) full = full && (n0 + kBN - 1 <= qa + off + a.right);
+        if (a.left < kUnbounded) full = full && (n0 >= qa + 63 + off - a.left);
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[32], dpv[32];
+          tmem_ld32(tmem + lane_off + cS + c * 32, sv);
+          tmem_ld32(tmem + lane_off + cP + c * 32, dpv);
+          tmem_wait_ld();
+          const int qc = 64 * hh + 32 * c;           // first query of the chunk within the tile
+          float lt[32], dd[32];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(s_lt + qc + e);
+            const float4 y = *reinterpret_cast<const float4*>(s_D + qc + e);
+            lt[e] = x.x; lt[e + 1] = x.y; lt[e + 2] = x.z; lt[e + 3] = x.w;
+            dd[e] = y.x; dd[e + 1] = y.y; dd[e + 2] = y.z; dd[e + 3] = y.w;
+          }
+          float p[32], ds[32];
+          if (full) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              p[e] = ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e]));
+              ds[e] = p[e] * (__uint_as_float(dpv[e]) - dd[e]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const long long qi = i0 + qc + e;
+              bool vis = key_ok && qi < sq;
+              const long long d = j - (qi + off);
+              if (a.right < kUnbounded) vis = vis && d <= a.right;
+              if (a.left < kUnbounded) vis = vis && d >= -(long long)a.left;
+              p[e] = vis ? ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e])) : 0.f;
+              ds[e] = p[e] * (__uint_as_float(dpv[e]) - dd[e]);
+            }
+          }
+          uint32_t pk[16], dk_[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+            dk_[e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
+          }
+          tmem_st16(tmem + lane_off + cS + c * 16, pk);
+          const uint32_t rowp = sDS + hh * L::kHalf + r * 128;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int ch = c * 4 + v;
+            st_shared_v4(rowp + ((ch ^ (r & 7)) << 4), dk_[4 * v], dk_[4 * v + 1], dk_[4 * v + 2], dk_[4 * v + 3]);
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar.compute_done(hh));
+      }
+    }
+    // ---- epilogue: dK = scale * acc, dV = acc -------------------------------------------
+    const bool have = __all_sync(0xffffffffu, ok && T > 0 && mbar_wait(bar.ds_free(1), (T - 1) & 1, a.status));
+    tc_fence_after();
+    __nv_bfloat16* dkp = static_cast<__nv_bfloat16*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
+    __nv_bfloat16* dvp = static_cast<__nv_bfloat16*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int ncol = pass == 0 ? DK : DV;
+      const uint32_t col = pass == 0 ? kColDK : kColDV;
+      const float mul = pass == 0 ? a.scale : 1.f;
+      uint4* dst = reinterpret_cast<uint4*>(pass == 0 ? dkp : dvp);
+      for (int c = 0; c < ncol / 32; ++c) {
+        uint32_t v[32];
+        if (T > 0) {
+          tmem_ld32(tmem + lane_off + col + c * 32, v);
+          tmem_wait_ld();
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = (T > 0 && have) ? __uint_as_float(v[2 * e]) * mul : 0.f;
+          const float x1 = (T > 0 && have) ? __uint_as_float(v[2 * e + 1]) * mul : 0.f;
+          pk[e] = pack_bf16x2(x0, x1);
+        }
+        if (key_ok) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dst[c * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+    }
+  } else {
+    // ================================ dQ warps (thread = head-dim index) ==================
+    const int lg = warp & 3;
+    const int d = lg * 32 + lane;                     // TMEM lane = head-dim index of dQ^T
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    bool ok = true;
+    for (int t = 0; t < T && ok; ++t) {
+      const int h = head_of(t);
+      const long long i0 = qbase_of(t);
+      for (int hh = 0; hh < 2; ++hh) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.dq_full(hh), t & 1, a.status))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_off + (hh ? kColDPb : kColDPa), *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + lane_off + (hh ? kColDPb : kColDPa) + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar.dq_free(hh));
+        const long long qa = i0 + 64 * hh;
+        float* dst = a.dq_acc + ((q0 + qa) * a.hq + h) * DK + d;
+        const long long rstride = (long long)a.hq * DK;
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (qa + e < sq) atomicAdd(dst + e * rstride, __uint_as_float(v[e]) * a.scale);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // dq = bf16(dq_acc), 8 elements per thread
 __global__ void dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -389,6 +759,28 @@ bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int DV>
+cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
+  using L = PLayout<DV>;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map(&tq, a.q, 128, a.hq, a.total_q) || !make_map(&tk, a.k, 128, a.hkv, a.total_k) ||
+      !make_map(&tv, a.v, DV, a.hkv, a.total_k) || !make_map(&to, a.dout, DV, a.hq, a.total_q))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * 128 * sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  if ((e = launch_bwd_preprocess(a, 0, s)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(bwd_sm100_d128_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                L::kSmem)) != cudaSuccess)
+    return e;
+  dim3 grid(a.hkv, a.batch, (a.max_sk + kBN - 1) / kBN);
+  bwd_sm100_d128_kernel<DV><<<grid, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const long long n8 = (long long)a.total_q * a.hq * 128 / 8;
+  dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q),
+                                                                 n8);
+  return cudaGetLastError();
+}
+
 template <int DK, int DV>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   using L = BLayout<DK, DV>;
@@ -421,8 +813,8 @@ bool bwd_sm100_supported(const BwdArgs& a, int dtype) {
 }
 
 cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s) {
-  if (a.dk == 128 && a.dv == 128) return launch_typed<128, 128>(a, s);
-  if (a.dk == 128 && a.dv == 64) return launch_typed<128, 64>(a, s);
+  if (a.dk == 128 && a.dv == 128) return launch_d128<128>(a, s);
+  if (a.dk == 128 && a.dv == 64) return launch_d128<64>(a, s);
   if (a.dk == 64 && a.dv == 64) return launch_typed<64, 64>(a, s);
   if (a.dk == 64 && a.dv == 128) return launch_typed<64, 128>(a, s);
   return cudaErrorInvalidValue;
