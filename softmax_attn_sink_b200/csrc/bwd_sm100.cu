@@ -357,6 +357,12 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
 // TMEM: dK [0,128) dV [128,256) S_a [256,320) dP_a [320,384) S_b [384,448) dP_b [448,512);
 // P^T of a half is written over its S columns, dQ^T of a half over its dP columns.
 constexpr uint32_t kColSa = 256, kColDPa = 320, kColSb = 384, kColDPb = 448;
+// 12 warps: warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 compute, warps 8-11 dQ.
+// Launched at 168 registers (384 x 168 = 64512); the first warpgroup (whose MMA issuer keeps
+// many descriptors live) drops to 120, compute and dQ take 192: 128 x 120 + 256 x 192 = 64512.
+constexpr int kThreadsP = 384;
+constexpr int kRegsLow = 120, kRegsHigh = 192;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreadsP * 168, "register split");
 
 template <int DV>
 struct PLayout {
@@ -397,7 +403,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
 }
 
 template <int DV>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsP, 1)
 bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_do) {
@@ -458,6 +464,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == 0) {
     // ================================ TMA producer ======================================
+    regs_dec<kRegsLow>();
     if (lane == 0 && T > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -486,6 +493,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
+    regs_dec<kRegsLow>();
     if (lane == 0 && T > 0) {
       constexpr uint32_t id_s = idesc_bf16(kBN, 64, 0, 0);    // S_h, dP_h: 128 keys x 64 queries
       constexpr uint32_t id_dv = idesc_bf16(kBN, DV, 0, 1);   // P^T_h (TMEM) x dout_h (MN-major)
@@ -554,8 +562,11 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       mma_commit(bar.drain());
       mbar_wait(bar.drain(), 0, a.status);
     }
-  } else if (warp < 6) {
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();   // warps 2-3: no role, but part of the first warpgroup
+  } else if (warp < 8) {
     // ================================ compute warps (thread = key row) ===================
+    regs_inc<kRegsHigh>();
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
@@ -564,6 +575,15 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     const float scale2 = a.scale * kLog2e;
     const long long off = sk - sq;
     bool ok = true;
+    // lse_tot * log2e and D of query r of tile t, loaded one tile ahead
+    float pf_lt = 0.f, pf_D = 0.f;
+    auto prefetch = [&](int t) {
+      const long long qi = qbase_of(t) + r;
+      const long long idx = (long long)head_of(t) * a.total_q + q0 + qi;
+      pf_lt = qi < sq ? a.lse_tot[idx] * kLog2e : 0.f;
+      pf_D = qi < sq ? a.D[idx] : 0.f;
+    };
+    if (T > 0) prefetch(0);
     // The two named barriers below are hardware waits with no time limit, so every compute
     // warp passes both in every iteration: after a timed-out mbarrier wait a warp stops
     // working (ok = false) but never leaves the loop.
@@ -572,13 +592,10 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       const long long i0 = qbase_of(t);
       // stage lse_tot * log2e and D of this tile's 128 queries (all 128 compute threads)
       named_bar_sync(1, 128);
-      {
-        const long long qi = i0 + r;
-        const bool qok = qi < sq;
-        s_lt[r] = qok ? a.lse_tot[(long long)h * a.total_q + q0 + qi] * kLog2e : 0.f;
-        s_D[r] = qok ? a.D[(long long)h * a.total_q + q0 + qi] : 0.f;
-      }
+      s_lt[r] = pf_lt;
+      s_D[r] = pf_D;
       named_bar_sync(1, 128);
+      if (t + 1 < T) prefetch(t + 1);   // in flight while this tile is computed
 #pragma unroll 1
       for (int hh = 0; hh < 2 && ok; ++hh) {
         const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
@@ -680,6 +697,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     }
   } else {
     // ================================ dQ warps (thread = head-dim index) ==================
+    regs_inc<kRegsHigh>();
     const int lg = warp & 3;
     const int d = lg * 32 + lane;                     // TMEM lane = head-dim index of dQ^T
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
@@ -773,7 +791,7 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
                                 L::kSmem)) != cudaSuccess)
     return e;
   dim3 grid(a.hkv, a.batch, (a.max_sk + kBN - 1) / kBN);
-  bwd_sm100_d128_kernel<DV><<<grid, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
+  bwd_sm100_d128_kernel<DV><<<grid, kThreadsP, L::kSmem, s>>>(a, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long n8 = (long long)a.total_q * a.hq * 128 / 8;
   dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q),
