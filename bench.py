@@ -326,16 +326,20 @@ def bench_decode(args, world, peaks, peak_kind):
     import torch
     import softmax_attn_sink_b200 as sab
     d = W.config5_meta()
+    nb = args.decode_batch
+    if nb < 64:  # a smaller case of the same kernels (for profiler captures)
+        d.q = d.q[:nb]
+        d.cu_seqlens_k = d.cu_seqlens_k[:nb + 1].copy()
     total_k = int(d.cu_seqlens_k[-1])
     k, v = W.decode_kv_on_device(total_k, 8, 128, 128, seed=4)
     q = torch.from_numpy(d.q).to(torch.bfloat16).cuda()
     cu = torch.from_numpy(d.cu_seqlens_k).cuda()
     sink = torch.from_numpy(d.sink).cuda()
     mk = int(np.diff(d.cu_seqlens_k).max())
-    out = torch.empty((64, 64, 128), dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty((64, 64), dtype=torch.float32, device="cuda")
-    splits = sab.decode_num_splits(64, mk, total_k, 64, 8, 128, 128)
-    ws = torch.empty(64 * 64 * splits * (128 + 2) * 4 + 4096, dtype=torch.uint8, device="cuda")
+    out = torch.empty((nb, 64, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((64, nb), dtype=torch.float32, device="cuda")
+    splits = sab.decode_num_splits(nb, mk, total_k, 64, 8, 128, 128)
+    ws = torch.empty(nb * 64 * splits * (128 + 2) * 4 + 4096, dtype=torch.uint8, device="cuda")
     flush = Flusher()
     steps = max(3, min(args.steps, 50))
     per, total = time_steps(
@@ -347,7 +351,7 @@ def bench_decode(args, world, peaks, peak_kind):
     gbs = algo / (statistics.mean(per) * 1e-3) / 1e9
     pk = peaks["hbm_gbs"]
     del k, v
-    return {"workload": "decode64_gqa64x8_d128_L8k-32k", "unit": "GB/s", "steps": steps,
+    return {"workload": f"decode{nb}_gqa64x8_d128_L8k-32k", "unit": "GB/s", "steps": steps,
             "value": round(algo * world / (total / steps * 1e-3) / 1e9, 1),
             "ms_per_step": round(total / steps, 4), "bytes_per_step": algo, "splits": splits,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk, "unit": "GB/s",
@@ -435,6 +439,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", type=int, default=4, choices=[1, 2, 3, 4],
                     help="sequences of the fwd_bwd leg (4 = the full training workload)")
+    ap.add_argument("--decode-batch", type=int, default=64,
+                    help="sequences of the decode leg (64 = the full decode workload)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and args.workload == "all":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -341,9 +341,17 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         for (int c = 0; c < kBN; ++c)
           if (c < klo || c >= khi) sr[c] = __float_as_uint(kNegInf);
       }
-      float mx = kNegInf;
+      // row max over 8 independent chains (a single chain would be 128 dependent steps)
+      float mxv[8];
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      for (int e = 0; e < 8; ++e) mxv[e] = __uint_as_float(sr[e]);
+#pragma unroll
+      for (int c = 8; c < kBN; ++c) mxv[c & 7] = fmaxf(mxv[c & 7], __uint_as_float(sr[c]));
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int e = 0; e < w; ++e) mxv[e] = fmaxf(mxv[e], mxv[e + w]);
+      const float mx = mxv[0];
       const float m_tile = mx * scale2;
       const bool need = m_tile > m + kRescaleThreshold;
       float alpha = 1.f;
@@ -352,22 +360,24 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         m = m_tile;
       }
       const bool any_rescale = __any_sync(0xffffffffu, need);
-      // P = 2^{S scale log2e - m} as bf16, over S columns already read, 64 keys at a time
-      float sum = 0.f;
+      // P = 2^{S scale log2e - m} as bf16, over S columns already read, 64 keys at a time.
+      // Masked scores are -inf and 2^-inf = +0, so they need no test; m = -inf only when
+      // every score is -inf (then neg_m = 0 keeps the argument -inf, not NaN).
       const float neg_m = (m == kNegInf) ? 0.f : -m;
+      float sv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float v0 = __uint_as_float(sr[hh * 64 + 2 * c]), v1 = __uint_as_float(sr[hh * 64 + 2 * c + 1]);
-          const float p0 = (v0 == kNegInf) ? 0.f : ex2(fmaf(v0, scale2, neg_m));
-          const float p1 = (v1 == kNegInf) ? 0.f : ex2(fmaf(v1, scale2, neg_m));
-          sum += p0 + p1;
+          const float p0 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c]), scale2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c + 1]), scale2, neg_m));
+          sv[c & 3] += p0 + p1;
           pk[c] = pack_bf16x2(p0, p1);
         }
         tmem_st32(tS + hh * 32, pk);
       }
+      const float sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
       l = l * alpha + sum;
 
       if (any_rescale && jj >= 1) {
