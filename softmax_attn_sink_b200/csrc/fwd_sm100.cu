@@ -42,8 +42,8 @@ constexpr int kBN = 128;       // keys per tile
 constexpr int kStages = 2;     // K / V ring depth
 constexpr int kThreads = 384;  // 3 warpgroups
 // Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup gives
-// back down to 40 and the two softmax warpgroups take 232: 128 x 40 + 256 x 232 = 64512.
-constexpr int kRegsLaunch = 168, kRegsProducer = 40, kRegsSoftmax = 232;
+// back down to 72 and the two softmax warpgroups take 216: 128 x 72 + 256 x 216 = 64512.
+constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsSoftmax = 216;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -236,6 +236,12 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       constexpr uint32_t idesc_pv = idesc_bf16(kBM, DV, 0, 1);
       bool ok = mbar_wait(bar.q_full(), 0, a.status);
       int k_waited = -1;  // last key tile whose K load we waited for
+      // Shared-memory descriptors, built once: an address offset is an addition to the start
+      // field (addresses stay below 2^18 bytes, so the 14-bit field never carries).
+      const uint64_t dQ0 = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t dQ1 = dQ0 + (uint64_t)(L::kQBytes >> 4);
+      const uint64_t dK0 = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t dV0 = smem_desc(sV, L::kHalfBytes, 1024, kLayoutSwizzle128B);
       const int jA0 = un[0].j0, jA1 = un[0].j1, jB0 = un[1].j0, jB1 = un[1].j1;
       auto j0_of = [&](int u) { return u ? jB0 : jA0; };
       // S_u(j) = Q_u K_j^T
@@ -249,12 +255,12 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         // S_u is overwritten while P_u (inside S_u) was read by the previous PV_u: MMAs issued
         // by one thread execute in issue order, so that read is done before this write.
         tc_fence_after();
-        const uint32_t qs = sQ + u * L::kQBytes;
+        const uint64_t dq = u ? dQ1 : dQ0, dk = dK0 + (uint64_t)(st * (L::kKBytes >> 4));
+        const uint32_t dS = tmem + col_S(u);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kHalfBytes + (ks & 3) * 32;
-          mma_ss(tmem + col_S(u), smem_desc(qs + off, 16, 1024, kLayoutSwizzle128B),
-                 smem_desc(sK + st * L::kKBytes + off, 16, 1024, kLayoutSwizzle128B), idesc_qk, ks > 0);
+          const uint32_t off16 = ((ks >> 2) * L::kHalfBytes + (ks & 3) * 32) >> 4;
+          mma_ss(dS, dq + off16, dk + off16, idesc_qk, ks > 0);
         }
         mma_commit(bar.s_full(u));
         return true;
@@ -264,11 +270,11 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         const int st = j % kStages, jj = j - j0_of(u);
         if (!mbar_wait(bar.p_full(u), jj & 1, a.status)) return false;
         tc_fence_after();
+        const uint64_t dv = dV0 + (uint64_t)(st * (L::kVBytes >> 4));
+        const uint32_t dO = tmem + col_O(u), aP = tmem + col_S(u);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + col_O(u), tmem + col_S(u) + kk * 8,
-                 smem_desc(sV + st * L::kVBytes + kk * 2048, L::kHalfBytes, 1024, kLayoutSwizzle128B),
-                 idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(dO, aP + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar.pv_done(u));
         return true;
       };
