@@ -359,9 +359,9 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
 constexpr uint32_t kColSa = 256, kColDPa = 320, kColSb = 384, kColDPb = 448;
 // 12 warps: warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 compute, warps 8-11 dQ.
 // Launched at 168 registers (384 x 168 = 64512); the first warpgroup (whose MMA issuer keeps
-// many descriptors live) drops to 120, compute and dQ take 192: 128 x 120 + 256 x 192 = 64512.
+// nine descriptors live) drops to 136, compute and dQ take 184: 128 x 136 + 256 x 184 = 64512.
 constexpr int kThreadsP = 384;
-constexpr int kRegsLow = 120, kRegsHigh = 192;
+constexpr int kRegsLow = 136, kRegsHigh = 184;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreadsP * 168, "register split");
 
 template <int DV>
@@ -500,49 +500,58 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       constexpr uint32_t id_dk = idesc_bf16(kBN, DK, 0, 1);   // dS^T_h (K-major) x Q_h (MN-major)
       constexpr uint32_t id_dq = idesc_bf16(DK, 64, 1, 1);    // K^T (MN-major) x dS^T_h (MN-major)
       // S_h(t) = K Q_h^T -> S columns; dP_h(t) = V dout_h^T -> dP columns
+      // Shared-memory descriptors, built once: an address offset is an addition to the start
+      // field (addresses stay below 2^18 bytes, so the 14-bit field never carries).  "k" =
+      // K-major view (LBO unused), "m" = MN-major view (LBO = the 16 KB between 64-column halves).
+      const uint64_t kK = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t mK = smem_desc(sK, L::kHalf, 1024, kLayoutSwizzle128B);
+      const uint64_t kV = smem_desc(sV, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t kQ = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t mQ = smem_desc(sQ, L::kHalf, 1024, kLayoutSwizzle128B);
+      const uint64_t kO = smem_desc(sO, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t mO = smem_desc(sO, L::kHalf, 1024, kLayoutSwizzle128B);
+      const uint64_t kDS = smem_desc(sDS, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t mDS = smem_desc(sDS, L::kHalf, 1024, kLayoutSwizzle128B);
       auto issue_sdp = [&](int t, int hh) -> bool {
         const int st = t & 1;
-        const uint32_t q_s = sQ + st * L::kQBytes + hh * 8192, o_s = sO + st * L::kOBytes + hh * 8192;
-        const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
+        const uint64_t qoff = (uint64_t)((st * L::kQBytes + hh * 8192) >> 4);
+        const uint64_t ooff = (uint64_t)((st * L::kOBytes + hh * 8192) >> 4);
+        const uint32_t cS = tmem + (hh ? kColSb : kColSa), cP = tmem + (hh ? kColDPb : kColDPa);
         if (hh == 0 && !mbar_wait(bar.qd_full(st), (t >> 1) & 1, a.status)) return false;
         if (t >= 1 && !mbar_wait(bar.dv_done(hh), (t - 1) & 1, a.status)) return false;   // P^T_h read
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
-          mma_ss(tmem + cS, smem_desc(sK + off, 16, 1024, kLayoutSwizzle128B),
-                 smem_desc(q_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
+          const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
+          mma_ss(cS, kK + off16, kQ + qoff + off16, id_s, ks > 0);
         }
         if (t >= 1 && !mbar_wait(bar.dq_free(hh), (t - 1) & 1, a.status)) return false;   // dQ^T_h read
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DV / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
-          mma_ss(tmem + cP, smem_desc(sV + off, 16, 1024, kLayoutSwizzle128B),
-                 smem_desc(o_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
+          const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
+          mma_ss(cP, kV + off16, kO + ooff + off16, id_s, ks > 0);
         }
         mma_commit(bar.sdp_full(hh));
         return true;
       };
       auto issue_grads = [&](int t, int hh) {
         const int st = t & 1;
-        const uint32_t q_s = sQ + st * L::kQBytes, o_s = sO + st * L::kOBytes;
-        const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
+        const uint64_t qoff = (uint64_t)((st * L::kQBytes) >> 4), ooff = (uint64_t)((st * L::kOBytes) >> 4);
+        const uint64_t dsoff = (uint64_t)((hh * L::kHalf) >> 4);
+        const uint32_t cS = tmem + (hh ? kColSb : kColSa), cP = tmem + (hh ? kColDPb : kColDPa);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kColDV, tmem + cS + kk * 8,
-                 smem_desc(o_s + (4 * hh + kk) * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dv,
+          mma_ts(tmem + kColDV, cS + kk * 8, mO + ooff + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_dv,
                  (t > 0 || hh > 0 || kk > 0));
         mma_commit(bar.dv_done(hh));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kColDK, smem_desc(sDS + hh * L::kHalf + kk * 32, 16, 1024, kLayoutSwizzle128B),
-                 smem_desc(q_s + (4 * hh + kk) * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dk,
-                 (t > 0 || hh > 0 || kk > 0));
+          mma_ss(tmem + kColDK, kDS + dsoff + (uint64_t)((kk * 32) >> 4),
+                 mQ + qoff + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_dk, (t > 0 || hh > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ss(tmem + cP, smem_desc(sK + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B),
-                 smem_desc(sDS + hh * L::kHalf + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dq, kk > 0);
+          mma_ss(cP, mK + (uint64_t)((kk * 2048) >> 4), mDS + dsoff + (uint64_t)((kk * 2048) >> 4), id_dq, kk > 0);
         mma_commit(bar.dq_full(hh));
         mma_commit(bar.ds_free(hh));
       };
