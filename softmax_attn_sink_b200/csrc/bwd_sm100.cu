@@ -724,12 +724,15 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar.dq_free(hh));
+        // dq_acc is head-major, [hq][total_q][128]: consecutive queries of a head are 512
+        // bytes apart, a compile-time stride that folds into each reduction's address.
         const long long qa = i0 + 64 * hh;
-        float* dst = a.dq_acc + ((q0 + qa) * a.hq + h) * DK + d;
-        const long long rstride = (long long)a.hq * DK;
+        const long long left = sq - qa;
+        const int nval = left < 64 ? (int)left : 64;
+        float* dst = a.dq_acc + ((long long)h * a.total_q + q0 + qa) * DK + d;
 #pragma unroll
         for (int e = 0; e < 64; ++e)
-          if (qa + e < sq) atomicAdd(dst + e * rstride, __uint_as_float(v[e]) * a.scale);
+          if (e < nval) atomicAdd(dst + e * DK, __uint_as_float(v[e]) * a.scale);
       }
     }
   }
@@ -749,6 +752,25 @@ __global__ void dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* 
   if (i >= n8) return;
   const float4 x = reinterpret_cast<const float4*>(acc)[2 * i];
   const float4 y = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  uint4 o;
+  o.x = pack_bf16x2(x.x, x.y);
+  o.y = pack_bf16x2(x.z, x.w);
+  o.z = pack_bf16x2(y.x, y.y);
+  o.w = pack_bf16x2(y.z, y.w);
+  reinterpret_cast<uint4*>(dq)[i] = o;
+}
+
+// dq[t][h][:] = bf16(dq_acc[h][t][:]) for the head-major accumulator, 8 elements per thread.
+__global__ void dq_convert_hmajor_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int total_q,
+                                         int hq, long long n8) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const int c = (int)(i & 15);                      // 8-element chunk of the 128 dims
+  const long long th = i >> 4;                      // t * hq + h (output order)
+  const long long t = th / hq, h = th % hq;
+  const float* src = acc + ((h * total_q + t) * 128 + c * 8);
+  const float4 x = reinterpret_cast<const float4*>(src)[0];
+  const float4 y = reinterpret_cast<const float4*>(src)[1];
   uint4 o;
   o.x = pack_bf16x2(x.x, x.y);
   o.y = pack_bf16x2(x.z, x.w);
@@ -803,8 +825,8 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   bwd_sm100_d128_kernel<DV><<<grid, kThreadsP, L::kSmem, s>>>(a, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long n8 = (long long)a.total_q * a.hq * 128 / 8;
-  dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q),
-                                                                 n8);
+  dq_convert_hmajor_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
+      a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q), a.total_q, a.hq, n8);
   return cudaGetLastError();
 }
 
