@@ -151,17 +151,29 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def _reduce_device():
+    import torch.distributed as dist
+    return "cpu" if dist.get_backend() == "gloo" else "cuda"
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's value (all ranks call this in the same order)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, total_ms_max: float, steps: int) -> float:
+    """Throughput of the whole job: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (total_ms_max / steps * 1e-3)
 
 
 # --- timing helpers ---------------------------------------------------------------------
@@ -247,7 +259,7 @@ def bench_fwd(args, world, peaks, peak_kind, sampler):
     flush = Flusher()
     per, total_ms = time_steps(step, args.steps, args.warmup, world, flush, sampler)
     ms = total_ms / args.steps
-    tflops = flops * world / (total_ms / args.steps * 1e-3) / 1e12
+    tflops = weak_scaling_value(flops, world, total_ms, args.steps) / 1e12
     kernel_ms = statistics.mean(per)
     achieved = flops / (kernel_ms * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],

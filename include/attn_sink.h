@@ -178,6 +178,16 @@ const char* attn_sink_status_string(int status);
  */
 int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits);
 
+/*
+ * Diagnostics, with no counterpart on the pages: launches a one-thread kernel whose bounded
+ * on-chip wait is made to run out (it waits for an mbarrier phase nothing completes), so the
+ * timeout path of the tensor-core kernels can be exercised without faulting or hanging the
+ * GPU.  Takes about 2 s of GPU time.  Afterwards attn_sink_get_device_status() returns
+ * ATTN_SINK_ERR_TIMEOUT (and clears the word); the context stays usable.  Returns the
+ * launch status.
+ */
+int attn_sink_selftest_wait_timeout(attn_sink_stream_t stream);
+
 /* Library version, e.g. 0x000100 for 0.1.0. */
 int attn_sink_version(void);
 

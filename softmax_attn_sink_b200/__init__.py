@@ -29,7 +29,7 @@ STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE
 _SYMBOLS = ("attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "attn_sink_fwd_workspace_size",
             "attn_sink_bwd_workspace_size", "attn_sink_decode_workspace_size",
             "attn_sink_decode_num_splits", "attn_sink_status_string",
-            "attn_sink_get_device_status", "attn_sink_version")
+            "attn_sink_get_device_status", "attn_sink_selftest_wait_timeout", "attn_sink_version")
 
 
 class AttnSinkParams(ctypes.Structure):
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.attn_sink_status_string.restype = ctypes.c_char_p
         L.attn_sink_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.attn_sink_get_device_status.restype = i32
+        L.attn_sink_selftest_wait_timeout.argtypes = [vp]
+        L.attn_sink_selftest_wait_timeout.restype = i32
         L.attn_sink_version.argtypes = []
         L.attn_sink_version.restype = i32
         _lib = L
@@ -263,6 +265,11 @@ def device_status(stream=None) -> Tuple[int, int]:
     return int(st), int(bits.value)
 
 
+def selftest_wait_timeout(stream=None) -> None:
+    """Launch the diagnostics kernel whose bounded wait runs out (about 2 s)."""
+    _check("attn_sink_selftest_wait_timeout", lib().attn_sink_selftest_wait_timeout(_stream(stream)))
+
+
 class SinkAttention:
     """Autograd wrapper: ``SinkAttention.apply(q, k, v, sink, cu_q, cu_k, max_q, max_k,
     scale, causal, window_left, window_right)`` -> out, with gradients for q, k, v and the
@@ -298,5 +305,5 @@ class SinkAttention:
 
 
 __all__ = ["attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "decode_num_splits",
-           "device_status", "SinkAttention", "AttnSinkError", "AttnSinkParams", "make_params",
+           "device_status", "selftest_wait_timeout", "SinkAttention", "AttnSinkError", "AttnSinkParams", "make_params",
            "lib", "LIB_PATH", "ATTN_SINK_BF16", "ATTN_SINK_FP32"]

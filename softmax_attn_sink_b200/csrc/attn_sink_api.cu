@@ -5,7 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
-#include "../../include/attn_sink.h"
+#include "attn_sink.h"
 #include "launch.h"
 
 using namespace attn_sink;
@@ -240,6 +240,12 @@ int attn_sink_decode(const attn_sink_params* p, const void* q, const void* k, co
   a.splits = splits; a.scale = p->softmax_scale; a.left = left; a.right = right;
   a.status = status_ptr();
   return from_cuda(launch_decode_split(a, s));
+}
+
+int attn_sink_selftest_wait_timeout(attn_sink_stream_t stream) {
+  unsigned* sp = status_ptr();
+  if (!sp) return ATTN_SINK_ERR_CUDA;
+  return from_cuda(launch_wait_timeout_selftest(sp, static_cast<cudaStream_t>(stream)));
 }
 
 int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits) {

@@ -20,7 +20,7 @@
 // previous call's leftovers are never read.
 #include <stdint.h>
 
-#include "../../include/attn_sink.h"
+#include "attn_sink.h"
 
 namespace {
 

@@ -80,6 +80,9 @@ bool bwd_sm100_supported(const BwdArgs& a, int dtype);
 cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s);
 
 cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
+
+// A one-thread kernel whose bounded mbarrier wait is made to run out (diagnostics).
+cudaError_t launch_wait_timeout_selftest(unsigned* status, cudaStream_t s);
 bool decode_split_supported(int dk, int dv, int dtype);
 
 }  // namespace attn_sink

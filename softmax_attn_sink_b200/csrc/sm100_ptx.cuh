@@ -52,16 +52,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Bounded: gives up after
-// kWaitLimitNs of global time, records kStatusTimeout in the status word and returns
-// false, so a kernel never spins forever on a barrier nobody will complete.
+// kWaitLimitNs of global time (or, as a second bound, kWaitLimitIters polls), records
+// kStatusTimeout in the status word and returns false, so a kernel never spins forever on
+// a barrier nobody will complete.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kWaitLimitIters = 1u << 28;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 255u) == 0 && (global_timer_ns() - t0 > kWaitLimitNs || it >= kWaitLimitIters)) {
       set_status(status, kStatusTimeout);
       return false;
     }
