@@ -66,6 +66,33 @@ def visible_pairs(cu_q, cu_k, hq, causal, window_left=-1, window_right=-1) -> in
     return total * int(hq)
 
 
+def source_digest(kernel_file: str) -> str:
+    """sha256[:16] of a kernel source and every header in csrc/ (what its build depends on)."""
+    import glob
+    import hashlib
+    csrc = os.path.join(ROOT, "softmax_attn_sink_b200", "csrc")
+    h = hashlib.sha256()
+    for path in [os.path.join(csrc, kernel_file)] + sorted(glob.glob(os.path.join(csrc, "*.cuh")) +
+                                                           glob.glob(os.path.join(csrc, "*.h"))):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def kernel_traffic(kernel_file: str):
+    """DRAM bytes per bench launch from profiles/traffic.txt, or None when the kernel's
+    sources have changed since that capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
+            for line in f:
+                parts = line.split()
+                if parts and not line.startswith("#") and parts[0] == kernel_file:
+                    return int(parts[2]) if parts[1] == source_digest(kernel_file) else None
+    except OSError:
+        pass
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -264,7 +291,8 @@ def bench_fwd(args, world, peaks, peak_kind, sampler):
     achieved = flops / (kernel_ms * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-            "traffic": None, "peak_source": f"bf16_tflops ({peak_kind}, burst: kernel timed alone)",
+            "traffic": kernel_traffic("fwd_sm100.cu"),
+            "peak_source": f"bf16_tflops ({peak_kind}, burst: kernel timed alone)",
             "kernel": "fwd (one launch per step)", "flops_per_launch": flops}
 
     # end to end through the public API with host buffers: H2D of the step's inputs from
@@ -329,7 +357,8 @@ def bench_fwd_bwd(args, world, peaks, peak_kind):
         "bwd": {"value": round(bf * world / (b_total / steps * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(b_total / steps, 4), "flops": bf,
                 "roofline": {"bound": "tensor", "achieved": round(ba, 2), "peak": pk,
-                             "unit": "TFLOP/s", "frac": round(ba / pk, 4), "traffic": None,
+                             "unit": "TFLOP/s", "frac": round(ba / pk, 4),
+                             "traffic": kernel_traffic("bwd_sm100.cu") if args.seqs == 4 else None,
                              "peak_source": f"bf16_tflops ({peak_kind}, burst)"}},
     }
 
@@ -367,7 +396,8 @@ def bench_decode(args, world, peaks, peak_kind):
             "value": round(algo * world / (total / steps * 1e-3) / 1e9, 1),
             "ms_per_step": round(total / steps, 4), "bytes_per_step": algo, "splits": splits,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk, "unit": "GB/s",
-                         "frac": round(gbs / pk, 4), "traffic": None,
+                         "frac": round(gbs / pk, 4),
+                         "traffic": kernel_traffic("decode_split.cu") if nb == 64 else None,
                          "peak_source": f"hbm_gbs ({peak_kind})",
                          "kernels": "split + merge (two launches per step)"}}
 
@@ -383,7 +413,7 @@ def cpu_cores():
 
 def cpu_baseline(budget_s=15.0):
     secs, flops, steps = 0.0, 0, 0
-    while secs < budget_s and steps < 400:
+    while secs < budget_s and steps < 5000:
         s, f = _oracle_step(steps)
         secs += s
         flops += f
