@@ -5,19 +5,25 @@
 //   S = scale * Q K^T,  m = max(sink, max S),
 //   out = sum e^{S-m} V / (sum e^{S-m} + e^{sink-m}),   lse = log sum e^{S}  (no sink).
 //
-// A CTA owns two 128-row query units, A and B, that read the same K/V tiles: two q heads
+// A work item is two 128-row query units, A and B, that read the same K/V tiles: two q heads
 // of one GQA group at the same row tile when the group size is even (identical key ranges),
 // otherwise two adjacent row tiles of one head.  Keys are streamed in 128-key tiles over the
 // union of the two units' visible ranges (bottom-right causal / sliding window, PyTorch
 // issue #108108 "Proposal"; slime wrapper docstring "window_size"); each unit only takes the
-// tiles that meet its own range.  Warp roles:
-//   warp 0      TMA producer: Q_A, Q_B once, then K and V tiles into a 2-stage ring.
+// tiles that meet its own range.  The kernel is persistent: one CTA per SM walks a
+// longest-first list of items (built in shared memory from cu_seqlens_q by every CTA), and
+// the K/V ring, the TMEM buffers and the mbarrier phases carry over from one item to the
+// next, so an item's Q load and first QK overlap the previous item's last tiles.  Warp roles:
+//   warp 0      TMA producer: Q_A, Q_B per item (once the previous item's last QK has read
+//               Q), then K and V tiles into a 2-stage ring.
 //   warp 1      TMEM allocation and the MMA issuer (one thread), in the order
 //                 PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1)
 //               so the tensor core works for one unit while the other unit's softmax runs.
 //               QK: S_U = Q_U K^T (A, B from shared memory); PV: O_U += P_U V (P from TMEM).
-//   warps 4-7   softmax of unit A, warps 8-11 softmax of unit B: thread t owns query row t
-//               (TMEM lane t).  The running max starts at the sink (log2 domain, the sink is
+//   warp 2      the scheduler: builds the item list, then decodes the CTA's items one by one
+//               into a 2-slot shared-memory ring that the other roles read (warp 3 idles).
+//   warps 4-7   softmax and epilogue of unit A, warps 8-11 of unit B: thread t owns query row
+//               t (TMEM lane t).  The running max starts at the sink (log2 domain, the sink is
 //               in post-scale units); the running sum counts keys only and e^{sink-m} joins
 //               the denominator in the epilogue, so the vanilla lse is m + log sum.  O is
 //               rescaled lazily, only when a row's max grows by more than 2^8 (exact: O and
@@ -41,6 +47,8 @@ constexpr int kBM = 128;       // query rows per unit
 constexpr int kBN = 128;       // keys per tile
 constexpr int kStages = 2;     // K / V ring depth
 constexpr int kThreads = 384;  // 3 warpgroups
+constexpr int kItemSlots = 2;  // scheduled items in flight
+constexpr int kItemReaders = 10;  // item slot readers: producer, MMA thread, 8 softmax warps
 // Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup gives
 // back down to 72 and the two softmax warpgroups take 216: 128 x 72 + 256 x 216 = 64512.
 constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsSoftmax = 216;
@@ -62,113 +70,262 @@ struct Layout {
   static constexpr int kOffK = kOffQ + 2 * kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKBytes;
   static constexpr int kOffBar = kOffV + kStages * kVBytes;
-  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int kNumBars = 1 + 4 * kStages + 6 + 1;
+  // q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
+  // pv_done[2], drain, item_full[I], item_empty[I]
+  static constexpr int kNumBars = 2 + 4 * kStages + 7 + 2 * kItemSlots;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-  static constexpr int kBytes = kOffTmemSlot + 16;
-  // + slack to align the base to 1 KB; at least 116 KB so that two CTAs never share an SM
-  // (each CTA holds all 512 TMEM columns)
-  static constexpr int kSmem = (kBytes + 1024) > 118784 ? (kBytes + 1024) : 118784;
+  static constexpr int kOffItems = (kOffTmemSlot + 16 + 127) / 128 * 128;  // ItemDesc[kItemSlots]
+  static constexpr int kOffTable = kOffItems + kItemSlots * 128;           // item list of a persistent launch
+  // bytes for a table of `table_ints` ints, + slack to align the base to 1 KB; at least 116 KB
+  // so that two CTAs never share an SM (each CTA holds all 512 TMEM columns)
+  static constexpr long long smem_bytes(long long table_ints) {
+    return (kOffTable + 4 * table_ints + 1024) > 118784 ? (kOffTable + 4 * table_ints + 1024) : 118784;
+  }
 };
 
 // mbarrier addresses, laid out back to back from `base`.
 struct Bars {
   uint32_t base;
   __device__ __forceinline__ uint32_t q_full() const { return base; }
-  __device__ __forceinline__ uint32_t k_full(int s) const { return base + 8u * (1 + s); }
-  __device__ __forceinline__ uint32_t k_empty(int s) const { return base + 8u * (1 + kStages + s); }
-  __device__ __forceinline__ uint32_t v_full(int s) const { return base + 8u * (1 + 2 * kStages + s); }
-  __device__ __forceinline__ uint32_t v_empty(int s) const { return base + 8u * (1 + 3 * kStages + s); }
-  __device__ __forceinline__ uint32_t s_full(int u) const { return base + 8u * (1 + 4 * kStages + u); }
-  __device__ __forceinline__ uint32_t p_full(int u) const { return base + 8u * (3 + 4 * kStages + u); }
-  __device__ __forceinline__ uint32_t pv_done(int u) const { return base + 8u * (5 + 4 * kStages + u); }
-  __device__ __forceinline__ uint32_t drain() const { return base + 8u * (7 + 4 * kStages); }
+  __device__ __forceinline__ uint32_t q_empty() const { return base + 8u; }
+  __device__ __forceinline__ uint32_t k_full(int s) const { return base + 8u * (2 + s); }
+  __device__ __forceinline__ uint32_t k_empty(int s) const { return base + 8u * (2 + kStages + s); }
+  __device__ __forceinline__ uint32_t v_full(int s) const { return base + 8u * (2 + 2 * kStages + s); }
+  __device__ __forceinline__ uint32_t v_empty(int s) const { return base + 8u * (2 + 3 * kStages + s); }
+  __device__ __forceinline__ uint32_t s_full(int u) const { return base + 8u * (2 + 4 * kStages + u); }
+  __device__ __forceinline__ uint32_t p_full(int u) const { return base + 8u * (4 + 4 * kStages + u); }
+  __device__ __forceinline__ uint32_t pv_done(int u) const { return base + 8u * (6 + 4 * kStages + u); }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * (8 + 4 * kStages); }
+  __device__ __forceinline__ uint32_t item_full(int s) const { return base + 8u * (9 + 4 * kStages + s); }
+  __device__ __forceinline__ uint32_t item_empty(int s) const {
+    return base + 8u * (9 + 4 * kStages + kItemSlots + s);
+  }
 };
 
-// One query unit of the CTA: q head, first row, rows, visible key range and the tiles of
-// the CTA's key loop that meet it, [j0, j1).
+// ---- work schedule -----------------------------------------------------------------------
+//
+// A work item is one CTA's worth of work: a sequence b, a unit pair x (a head pair of a GQA
+// group when the group size is even, otherwise a head) and a level z (the row tile, or the
+// pair of row tiles, that the two units take).  Items are numbered level by level from the
+// deepest level down, and within a level by sequence and then unit pair.  Under a causal mask
+// an item's cost grows with its level, so this order is longest-first.
+struct Sched {
+  int zmax;        // levels of the longest sequence (bounded by max_seqlen_q)
+  int width;       // unit pairs per (sequence, level)
+  int persistent;  // 1: the grid's CTAs walk the numbered list; 0: CTA i runs item i of the dense grid
+};
+
+// Levels of sequence b: its row tiles (two q heads per item) or row-tile pairs (one head per item).
+__device__ __forceinline__ int levels_of(const FwdArgs& a, const Sched& sc, bool even, int b) {
+  const int sq = a.cu_q[b + 1] - a.cu_q[b];
+  const int nt = sq > 0 ? (sq + kBM - 1) / kBM : 0;
+  const int nz = even ? nt : (nt + 1) / 2;
+  return nz < sc.zmax ? nz : sc.zmax;
+}
+
+// In-place inclusive suffix sum over v[0, n) by one warp: v[i] becomes sum_{k >= i} v[k].
+__device__ __forceinline__ void warp_suffix_sum(int* v, int n, int lane) {
+  const int C = (n + 31) / 32;
+  const int b0 = lane * C, b1 = (b0 + C < n) ? b0 + C : n;
+  int tot = 0;
+  for (int i = b0; i < b1; ++i) tot += v[i];
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += y;
+  }
+  int run = incl - tot;  // totals of the chunks above this lane's
+  for (int i = b1 - 1; i >= b0; --i) {
+    run += v[i];
+    v[i] = run;
+  }
+  __syncwarp();
+}
+
+// Item table of a persistent launch, built by one warp of every CTA (identical in all of them):
+//   cnt[z]   = sequences with more than z levels (the sequences present at level z),
+//   start[z] = number of the first item of level z,
+//   perm[j]  = the j-th sequence by descending level count (ties by index): the sequences
+//              present at level z are exactly perm[0, cnt[z]).
+__device__ void build_table(const FwdArgs& a, const Sched& sc, bool even, int* tbl, int lane) {
+  const int Z = sc.zmax, B = a.batch, W = sc.width;
+  int* cnt = tbl;
+  int* start = tbl + Z;
+  int* run = tbl + 2 * Z;
+  int* perm = tbl + 3 * Z;
+  for (int i = lane; i < Z; i += 32) cnt[i] = run[i] = 0;
+  __syncwarp();
+  for (int b = lane; b < B; b += 32) {
+    const int nz = levels_of(a, sc, even, b);
+    if (nz > 0) atomicAdd(&cnt[nz - 1], 1);  // histogram: cnt[n - 1] = sequences with n levels
+  }
+  __syncwarp();
+  warp_suffix_sum(cnt, Z, lane);             // cnt[z] = sequences with more than z levels
+  for (int i = lane; i < Z; i += 32) start[i] = cnt[i];
+  __syncwarp();
+  warp_suffix_sum(start, Z, lane);
+  for (int i = lane; i < Z; i += 32) start[i] = W * (start[i] - cnt[i]);
+  // stable counting sort of the sequences by descending level count
+  for (int c0 = 0; c0 < B; c0 += 32) {
+    const int b = c0 + lane;
+    const int nz = b < B ? levels_of(a, sc, even, b) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, nz);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (nz > 0) perm[(nz < Z ? cnt[nz] : 0) + run[nz - 1] + rank] = b;
+    __syncwarp();
+    if (nz > 0 && rank == 0) run[nz - 1] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// Item of round r for this CTA.  Persistent CTAs walk the list in a snake: round r takes items
+// [r G, (r + 1) G), forward on even rounds and backward on odd ones, which keeps the
+// longest-first order balanced across the CTAs.  In grid mode CTA i runs item i only.
+__device__ __forceinline__ long long item_of_round(const Sched& sc, int r) {
+  const long long G = gridDim.x, c = blockIdx.x;
+  if (!sc.persistent) return r == 0 ? c : -1;
+  return (long long)r * G + ((r & 1) ? G - 1 - c : c);
+}
+
+// Decodes item t into (b, x, z).  `lvl` is a per-thread cursor over the levels (items of one
+// CTA come in increasing order, so it only moves down).  Returns false past the last item, or
+// for a grid-mode item whose sequence has no such level.
+__device__ __forceinline__ bool decode_item(const FwdArgs& a, const Sched& sc, bool even, const int* tbl,
+                                            long long t, int& lvl, int& b, int& x, int& z) {
+  if (t < 0) return false;
+  const int W = sc.width;
+  if (sc.persistent) {
+    const int Z = sc.zmax;
+    const int* cnt = tbl;
+    const int* start = tbl + Z;
+    const int* perm = tbl + 3 * Z;
+    while (lvl >= 0 && t >= (long long)start[lvl] + (long long)W * cnt[lvl]) --lvl;
+    if (lvl < 0) return false;
+    const int r = (int)(t - start[lvl]);
+    const int j = r / W;
+    x = r - j * W;
+    b = perm[j];
+    z = lvl;
+    return true;
+  }
+  const long long per_level = (long long)a.batch * W;
+  const long long zr = t / per_level;
+  if (zr >= sc.zmax) return false;
+  const int rem = (int)(t - zr * per_level);
+  z = sc.zmax - 1 - (int)zr;
+  b = rem / W;
+  x = rem - b * W;
+  return z < levels_of(a, sc, even, b);
+}
+
+// One query unit of an item: q head, first row, rows, visible key range and the tiles of the
+// item's key loop that meet it, [j0, j1).  Rows and keys are below 2^31 (packed totals are int).
 struct Unit {
-  int h;
-  long long m0, nrows, lo, hi;
-  int j0, j1;
+  int h, m0, nrows, lo, hi, j0, j1;
   bool valid;
 };
 
+// Everything a role needs about an item.
+struct Item {
+  int g;                  // kv head
+  int q0, sq, k0, sk;     // sequence offsets and lengths
+  int lo;                 // first key of the item's key loop
+  int n_tiles;            // 128-key tiles in the loop (the union of the units' ranges)
+  Unit un[2];
+};
+
+__device__ __forceinline__ void setup_item(const FwdArgs& a, bool even, int group, int b, int x, int z,
+                                           Item& it) {
+  int hA, hB, mA, mB;
+  if (even) {
+    const int g_ = x / (group / 2), p_ = x % (group / 2);
+    hA = g_ * group + 2 * p_;
+    hB = hA + 1;
+    mA = mB = z;
+  } else {
+    hA = hB = x;
+    mA = 2 * z;
+    mB = 2 * z + 1;
+  }
+  it.q0 = a.cu_q[b];
+  it.sq = a.cu_q[b + 1] - it.q0;
+  it.k0 = a.cu_k[b];
+  it.sk = a.cu_k[b + 1] - it.k0;
+  it.g = hA / group;
+  const int hs[2] = {hA, hB}, ms[2] = {mA, mB};
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    Unit& y = it.un[u];
+    y.h = hs[u];
+    y.m0 = ms[u] * kBM;
+    y.valid = y.m0 < it.sq;
+    y.nrows = y.valid ? ((it.sq - y.m0 < kBM) ? it.sq - y.m0 : kBM) : 0;
+    y.lo = y.hi = 0;
+    if (y.valid) {
+      long long l1, h1, l2, h2;
+      row_key_range(y.m0, it.sq, it.sk, a.left, a.right, l1, h1);
+      row_key_range(y.m0 + y.nrows - 1, it.sq, it.sk, a.left, a.right, l2, h2);
+      y.lo = (int)l1;
+      y.hi = (int)(h2 < l1 ? l1 : h2);  // ranges move right with the row: the union is [lo(first), hi(last))
+    }
+  }
+  int lo = it.un[0].lo, hi = it.un[0].hi;
+  if (it.un[1].valid && it.un[1].hi > it.un[1].lo) {
+    if (hi <= lo) { lo = it.un[1].lo; hi = it.un[1].hi; }
+    else { lo = lo < it.un[1].lo ? lo : it.un[1].lo; hi = hi > it.un[1].hi ? hi : it.un[1].hi; }
+  }
+  it.lo = lo;
+  it.n_tiles = hi > lo ? (hi - lo + kBN - 1) / kBN : 0;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    Unit& y = it.un[u];
+    if (y.valid && y.hi > y.lo) {
+      y.j0 = (y.lo - lo) / kBN;
+      y.j1 = (y.hi - lo + kBN - 1) / kBN;
+    } else {
+      y.j0 = y.j1 = 0;
+    }
+  }
+}
+
+// An item as the scheduler warp hands it to the other roles (one 128-byte shared-memory slot).
+struct ItemDesc {
+  int kind;                  // 1: an item, 0: no more items
+  int q0, sq, k0, sk;        // sequence offsets and lengths
+  int lo, n_tiles, g;        // first key and 128-key tiles of the key loop, kv head
+  int h[2], m0[2], j0[2], j1[2], valid[2];  // units A and B
+  int pad[14];
+};
+static_assert(sizeof(ItemDesc) == 128, "item slot size");
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
-fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
+fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using L = Layout<DK, DV>;
   extern __shared__ unsigned char smem_raw[];
 
-  // ---- work: two units; heaviest (largest) row tiles launch first ------------------------
   const int group = a.hq / a.hkv;
-  const int b = blockIdx.y;
-  const int zr = (int)gridDim.z - 1 - (int)blockIdx.z;
-  int hA, hB, mA, mB;
-  if ((group & 1) == 0) {
-    const int g_ = blockIdx.x / (group / 2), p_ = blockIdx.x % (group / 2);
-    hA = g_ * group + 2 * p_;
-    hB = hA + 1;
-    mA = mB = zr;
-  } else {
-    hA = hB = blockIdx.x;
-    mA = 2 * zr;
-    mB = 2 * zr + 1;
+  const bool even = (group & 1) == 0;
+  if (!sc.persistent) {
+    // grid mode: a CTA whose item does not exist leaves before taking any resource
+    int lvl = 0, b, x, z;
+    if (!decode_item(a, sc, even, nullptr, blockIdx.x, lvl, b, x, z)) return;
   }
-  const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
-  const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
-  if ((long long)mA * kBM >= sq) return;  // unit B is never valid without unit A
-  const int g = hA / group;
-
-  Unit un[2];
-  {
-    const int hs[2] = {hA, hB}, ms[2] = {mA, mB};
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      Unit& x = un[u];
-      x.h = hs[u];
-      x.m0 = (long long)ms[u] * kBM;
-      x.valid = x.m0 < sq;
-      x.nrows = x.valid ? ((sq - x.m0 < kBM) ? sq - x.m0 : kBM) : 0;
-      x.lo = x.hi = 0;
-      if (x.valid) {
-        long long l1, h1, l2, h2;
-        row_key_range(x.m0, sq, sk, a.left, a.right, l1, h1);
-        row_key_range(x.m0 + x.nrows - 1, sq, sk, a.left, a.right, l2, h2);
-        x.lo = l1;
-        x.hi = h2;  // ranges move right with the row: the union is [lo(first), hi(last))
-        if (x.hi < x.lo) x.hi = x.lo;
-      }
-    }
-  }
-  long long lo = un[0].lo, hi = un[0].hi;
-  if (un[1].valid && un[1].hi > un[1].lo) {
-    if (hi <= lo) { lo = un[1].lo; hi = un[1].hi; }
-    else { lo = lo < un[1].lo ? lo : un[1].lo; hi = hi > un[1].hi ? hi : un[1].hi; }
-  }
-  const int n_tiles = hi > lo ? (int)((hi - lo + kBN - 1) / kBN) : 0;
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    Unit& x = un[u];
-    if (x.valid && x.hi > x.lo) {
-      x.j0 = (int)((x.lo - lo) / kBN);
-      x.j1 = (int)((x.hi - lo + kBN - 1) / kBN);
-    } else {
-      x.j0 = x.j1 = 0;
-    }
-  }
-
   const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
   const uint32_t sQ = base_u32 + L::kOffQ, sK = base_u32 + L::kOffK, sV = base_u32 + L::kOffV;
   const Bars bar{base_u32 + L::kOffBar};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffTmemSlot);
+  ItemDesc* items = reinterpret_cast<ItemDesc*>(smem + L::kOffItems);
+  int* tbl = reinterpret_cast<int*>(smem + L::kOffTable);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q_full(), 1);
+    mbar_init(bar.q_empty(), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar.k_full(s), 1);
       mbar_init(bar.k_empty(s), 1);
@@ -180,6 +337,10 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar.p_full(u), 4);   // one arrival per softmax warp of the unit
       mbar_init(bar.pv_done(u), 1);
     }
+    for (int s = 0; s < kItemSlots; ++s) {
+      mbar_init(bar.item_full(s), 1);
+      mbar_init(bar.item_empty(s), kItemReaders);
+    }
     mbar_init(bar.drain(), 1);
     fence_mbar_init();
   }
@@ -187,6 +348,7 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
+  if (warp == 2 && sc.persistent) build_table(a, sc, even, tbl, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -194,252 +356,340 @@ fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
   if (warp == 0) {
     // ================================ TMA producer ======================================
     regs_dec<kRegsProducer>();
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const int nq = un[1].valid ? 2 : 1;
-      mbar_arrive_expect_tx(bar.q_full(), nq * L::kQBytes);
-      for (int hf = 0; hf < L::KH; ++hf)
-        tma_load_3d(sQ + hf * L::kHalfBytes, &tm_q, bar.q_full(), hf * 64, un[0].h, (int)(q0 + un[0].m0));
-      if (nq == 2)
+      int kv = 0, qn = 0;
+      for (int r = 0;; ++r) {
+        const int slot = r % kItemSlots;
+        if (!mbar_wait(bar.item_full(slot), (r / kItemSlots) & 1, a.status)) break;
+        const ItemDesc& d = items[slot];
+        const int kind = d.kind, n = d.n_tiles, q0 = d.q0, k0 = d.k0, lo = d.lo, g = d.g;
+        const int hA = d.h[0], hB = d.h[1], mA = d.m0[0], mB = d.m0[1], nq = d.valid[1] ? 2 : 1;
+        mbar_arrive(bar.item_empty(slot));
+        if (kind == 0) break;
+        if (n == 0) continue;
+        // the previous item's last QK has read Q
+        if (!mbar_wait(bar.q_empty(), (qn & 1) ^ 1, a.status)) break;
+        mbar_arrive_expect_tx(bar.q_full(), nq * L::kQBytes);
         for (int hf = 0; hf < L::KH; ++hf)
-          tma_load_3d(sQ + L::kQBytes + hf * L::kHalfBytes, &tm_q, bar.q_full(), hf * 64, un[1].h,
-                      (int)(q0 + un[1].m0));
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % kStages;
-        const uint32_t par = ((j / kStages) & 1) ^ 1;
-        const int row = (int)(k0 + lo + (long long)j * kBN);
-        if (!mbar_wait(bar.k_empty(st), par, a.status)) break;
-        mbar_arrive_expect_tx(bar.k_full(st), L::kKBytes);
-        for (int hf = 0; hf < L::KH; ++hf)
-          tma_load_3d(sK + st * L::kKBytes + hf * L::kHalfBytes, &tm_k, bar.k_full(st), hf * 64, g, row);
-        issued = j + 1;
-        if (!mbar_wait(bar.v_empty(st), par, a.status)) break;
-        mbar_arrive_expect_tx(bar.v_full(st), L::kVBytes);
-        for (int hf = 0; hf < L::VH; ++hf)
-          tma_load_3d(sV + st * L::kVBytes + hf * L::kHalfBytes, &tm_v, bar.v_full(st), hf * 64, g, row);
+          tma_load_3d(sQ + hf * L::kHalfBytes, &tm_q, bar.q_full(), hf * 64, hA, q0 + mA);
+        if (nq == 2)
+          for (int hf = 0; hf < L::KH; ++hf)
+            tma_load_3d(sQ + L::kQBytes + hf * L::kHalfBytes, &tm_q, bar.q_full(), hf * 64, hB, q0 + mB);
+        ++qn;
+        bool ok = true;
+        for (int j = 0; j < n; ++j, ++kv) {
+          const int st = kv % kStages;
+          const uint32_t par = ((kv / kStages) & 1) ^ 1;
+          const int row = k0 + lo + j * kBN;
+          if (!(ok = mbar_wait(bar.k_empty(st), par, a.status))) break;
+          mbar_arrive_expect_tx(bar.k_full(st), L::kKBytes);
+          for (int hf = 0; hf < L::KH; ++hf)
+            tma_load_3d(sK + st * L::kKBytes + hf * L::kHalfBytes, &tm_k, bar.k_full(st), hf * 64, g, row);
+          if (!(ok = mbar_wait(bar.v_empty(st), par, a.status))) {
+            ++kv;  // K of this tile is in flight
+            break;
+          }
+          mbar_arrive_expect_tx(bar.v_full(st), L::kVBytes);
+          for (int hf = 0; hf < L::VH; ++hf)
+            tma_load_3d(sV + st * L::kVBytes + hf * L::kHalfBytes, &tm_v, bar.v_full(st), hf * 64, g, row);
+        }
+        if (!ok) break;
       }
       // make sure no copy is still landing in shared memory when the CTA exits
-      mbar_wait(bar.q_full(), 0, a.status);
-      for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j) {
-        mbar_wait(bar.k_full(j % kStages), (j / kStages) & 1, a.status);
-        mbar_wait(bar.v_full(j % kStages), (j / kStages) & 1, a.status);
+      if (qn > 0) mbar_wait(bar.q_full(), (qn - 1) & 1, a.status);
+      for (int p = kv - kStages < 0 ? 0 : kv - kStages; p < kv; ++p) {
+        mbar_wait(bar.k_full(p % kStages), (p / kStages) & 1, a.status);
+        mbar_wait(bar.v_full(p % kStages), (p / kStages) & 1, a.status);
       }
     }
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
     regs_dec<kRegsProducer>();
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(kBM, DV, 0, 1);
-      bool ok = mbar_wait(bar.q_full(), 0, a.status);
-      int k_waited = -1;  // last key tile whose K load we waited for
       // Shared-memory descriptors, built once: an address offset is an addition to the start
       // field (addresses stay below 2^18 bytes, so the 14-bit field never carries).
       const uint64_t dQ0 = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
       const uint64_t dQ1 = dQ0 + (uint64_t)(L::kQBytes >> 4);
       const uint64_t dK0 = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
       const uint64_t dV0 = smem_desc(sV, L::kHalfBytes, 1024, kLayoutSwizzle128B);
-      const int jA0 = un[0].j0, jA1 = un[0].j1, jB0 = un[1].j0, jB1 = un[1].j1;
-      auto j0_of = [&](int u) { return u ? jB0 : jA0; };
-      // S_u(j) = Q_u K_j^T
-      auto issue_qk = [&](int u, int j) -> bool {
-        const int st = j % kStages, jj = j - j0_of(u);
-        if (k_waited < j) {
-          if (!mbar_wait(bar.k_full(st), (j / kStages) & 1, a.status)) return false;
+      int kv = 0, qn = 0;
+      int pcA = 0, pcB = 0;  // P tiles taken so far per unit (p_full phases)
+      for (int r = 0;; ++r) {
+        const int slot = r % kItemSlots;
+        if (!mbar_wait(bar.item_full(slot), (r / kItemSlots) & 1, a.status)) break;
+        const ItemDesc& d = items[slot];
+        const int kind = d.kind, n = d.n_tiles;
+        const int jA0 = d.j0[0], jA1 = d.j1[0], jB0 = d.j0[1], jB1 = d.j1[1];
+        mbar_arrive(bar.item_empty(slot));
+        if (kind == 0) break;
+        if (n == 0) continue;
+        if (!mbar_wait(bar.q_full(), qn & 1, a.status)) break;
+        ++qn;
+        bool ok = true;
+        int k_waited = -1;  // last tile of this item whose K load was waited for
+        auto wait_k = [&](int j) -> bool {
+          if (k_waited >= j) return true;
+          const int p = kv + j;
+          if (!mbar_wait(bar.k_full(p % kStages), (p / kStages) & 1, a.status)) return false;
           k_waited = j;
-        }
-        (void)jj;
-        // S_u is overwritten while P_u (inside S_u) was read by the previous PV_u: MMAs issued
-        // by one thread execute in issue order, so that read is done before this write.
-        tc_fence_after();
-        const uint64_t dq = u ? dQ1 : dQ0, dk = dK0 + (uint64_t)(st * (L::kKBytes >> 4));
-        const uint32_t dS = tmem + col_S(u);
+          return true;
+        };
+        // S_u(j) = Q_u K_j^T.  S_u is overwritten while P_u (inside S_u) was read by the
+        // previous PV_u: MMAs issued by one thread execute in issue order, so that read is
+        // done before this write.
+        auto issue_qk = [&](int u, int j) -> bool {
+          if (!wait_k(j)) return false;
+          tc_fence_after();
+          const int st = (kv + j) % kStages;
+          const uint64_t dq = u ? dQ1 : dQ0, dk = dK0 + (uint64_t)(st * (L::kKBytes >> 4));
+          const uint32_t dS = tmem + col_S(u);
 #pragma unroll
-        for (int ks = 0; ks < DK / 16; ++ks) {
-          const uint32_t off16 = ((ks >> 2) * L::kHalfBytes + (ks & 3) * 32) >> 4;
-          mma_ss(dS, dq + off16, dk + off16, idesc_qk, ks > 0);
-        }
-        mma_commit(bar.s_full(u));
-        return true;
-      };
-      // O_u += P_u(j) V_j
-      auto issue_pv = [&](int u, int j) -> bool {
-        const int st = j % kStages, jj = j - j0_of(u);
-        if (!mbar_wait(bar.p_full(u), jj & 1, a.status)) return false;
-        tc_fence_after();
-        const uint64_t dv = dV0 + (uint64_t)(st * (L::kVBytes >> 4));
-        const uint32_t dO = tmem + col_O(u), aP = tmem + col_S(u);
+          for (int ks = 0; ks < DK / 16; ++ks) {
+            const uint32_t off16 = ((ks >> 2) * L::kHalfBytes + (ks & 3) * 32) >> 4;
+            mma_ss(dS, dq + off16, dk + off16, idesc_qk, ks > 0);
+          }
+          mma_commit(bar.s_full(u));
+          return true;
+        };
+        // O_u += P_u(j) V_j (the first tile of the unit overwrites O_u)
+        auto issue_pv = [&](int u, int j) -> bool {
+          const int ph = u ? pcB + (j - jB0) : pcA + (j - jA0);
+          if (!mbar_wait(bar.p_full(u), ph & 1, a.status)) return false;
+          tc_fence_after();
+          const int st = (kv + j) % kStages;
+          const bool first = j == (u ? jB0 : jA0);
+          const uint64_t dv = dV0 + (uint64_t)(st * (L::kVBytes >> 4));
+          const uint32_t dO = tmem + col_O(u), aP = tmem + col_S(u);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(dO, aP + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar.pv_done(u));
-        return true;
-      };
-      auto active = [&](int u, int j) { return u ? (j >= jB0 && j < jB1) : (j >= jA0 && j < jA1); };
-      for (int u = 0; u < 2 && ok; ++u)
-        if (active(u, 0)) ok = issue_qk(u, 0);
-      if (ok) mma_commit(bar.k_empty(0));
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        const int st = j % kStages;
-        if (!(ok = mbar_wait(bar.v_full(st), (j / kStages) & 1, a.status))) break;
-        for (int u = 0; u < 2 && ok; ++u) {
-          if (active(u, j)) ok = issue_pv(u, j);
-          if (ok && j + 1 < n_tiles && active(u, j + 1)) ok = issue_qk(u, j + 1);
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(dO, aP + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (!first || kk > 0) ? 1u : 0u);
+          mma_commit(bar.pv_done(u));
+          return true;
+        };
+        auto active = [&](int u, int j) { return u ? (j >= jB0 && j < jB1) : (j >= jA0 && j < jA1); };
+        for (int u = 0; u < 2 && ok; ++u)
+          if (active(u, 0)) ok = issue_qk(u, 0);
+        if (!ok) break;
+        if (n == 1) mma_commit(bar.q_empty());  // every QK of the item is issued
+        mma_commit(bar.k_empty(kv % kStages));
+        for (int j = 0; j < n && ok; ++j) {
+          const int p = kv + j, st = p % kStages;
+          if (!(ok = mbar_wait(bar.v_full(st), (p / kStages) & 1, a.status))) break;
+          for (int u = 0; u < 2 && ok; ++u) {
+            if (active(u, j)) ok = issue_pv(u, j);
+            if (ok && j + 1 < n && active(u, j + 1)) ok = issue_qk(u, j + 1);
+          }
+          if (!ok) break;
+          if (j + 2 == n) mma_commit(bar.q_empty());  // the last QKs are issued
+          mma_commit(bar.v_empty(st));
+          if (j + 1 < n) {
+            // a tile no unit needs still has to be consumed for the producer's accounting
+            if (!(ok = wait_k(j + 1))) break;
+            mma_commit(bar.k_empty((p + 1) % kStages));
+          }
         }
         if (!ok) break;
-        mma_commit(bar.v_empty(st));
-        if (j + 1 < n_tiles) {
-          // a tile no unit needs still has to be consumed for the producer's accounting
-          if (k_waited < j + 1) {
-            if (!(ok = mbar_wait(bar.k_full((j + 1) % kStages), ((j + 1) / kStages) & 1, a.status))) break;
-            k_waited = j + 1;
-          }
-          mma_commit(bar.k_empty((j + 1) % kStages));
-        }
+        kv += n;
+        pcA += jA1 - jA0;
+        pcB += jB1 - jB0;
       }
       // every MMA must be complete before the TMEM is freed
       mma_commit(bar.drain());
       mbar_wait(bar.drain(), 0, a.status);
     }
-  } else if (warp < 4) {
-    regs_dec<kRegsProducer>();   // warps 2-3: no role, but part of the first warpgroup
+  } else if (warp == 2) {
+    // ================================ scheduler ===========================================
+    regs_dec<kRegsProducer>();
+    if (lane == 0) {
+      int lvl = sc.zmax - 1;
+      for (int r = 0;; ++r) {
+        const int slot = r % kItemSlots;
+        if (!mbar_wait(bar.item_empty(slot), ((r / kItemSlots) & 1) ^ 1, a.status)) break;
+        int b, x, z;
+        const bool more = decode_item(a, sc, even, tbl, item_of_round(sc, r), lvl, b, x, z);
+        ItemDesc& d = items[slot];
+        d.kind = more ? 1 : 0;
+        if (more) {
+          Item it;
+          setup_item(a, even, group, b, x, z, it);
+          d.q0 = it.q0;
+          d.sq = it.sq;
+          d.k0 = it.k0;
+          d.sk = it.sk;
+          d.lo = it.lo;
+          d.n_tiles = it.n_tiles;
+          d.g = it.g;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            d.h[u] = it.un[u].h;
+            d.m0[u] = it.un[u].m0;
+            d.j0[u] = it.un[u].j0;
+            d.j1[u] = it.un[u].j1;
+            d.valid[u] = it.un[u].valid ? 1 : 0;
+          }
+        }
+        mbar_arrive(bar.item_full(slot));  // release: the slot's writes are visible to the readers
+        if (!more) break;
+      }
+    }
+  } else if (warp == 3) {
+    regs_dec<kRegsProducer>();   // no role, but part of the first warpgroup
   } else {
     // ================================ softmax warpgroups =================================
     regs_inc<kRegsSoftmax>();
     const int u = warp < 8 ? 0 : 1;
-    const Unit x = u ? un[1] : un[0];
     const int lg = warp & 3;                      // TMEM lane quarter this warp may access
     const int r = lg * 32 + lane;                 // row within the unit
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     const uint32_t tS = tmem + lane_off + col_S(u), tO = tmem + lane_off + col_O(u);
-    const long long i = x.m0 + r;
-    const bool row_ok = x.valid && i < sq;
-    // this row's visible keys relative to the CTA's first key: [rlo, rhi) (empty if no row)
-    int rlo = 0, rhi = 0;
-    if (row_ok) {
-      long long l_, h_;
-      row_key_range(i, sq, sk, a.left, a.right, l_, h_);
-      rlo = (int)(l_ - lo);
-      rhi = (int)(h_ - lo);
-    }
-    const float sink2 = a.sink ? a.sink[x.h] * kLog2e : kNegInf;
     const float scale2 = a.scale * kLog2e;
-    float m = sink2, l = 0.f;
-    bool ok = true;
-    const int nU = x.j1 - x.j0;
+    int sc_u = 0;  // S tiles of this unit taken so far (s_full / pv_done phases)
+    for (int it = 0;; ++it) {
+      const int slot = it % kItemSlots;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.item_full(slot), (it / kItemSlots) & 1, a.status))) break;
+      const ItemDesc& d = items[slot];
+      const int kind = d.kind, valid = d.valid[u], h = d.h[u], j0 = d.j0[u], j1 = d.j1[u];
+      const int q0 = d.q0, sq = d.sq, sk = d.sk, klo0 = d.lo, i = d.m0[u] + r;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.item_empty(slot));
+      if (kind == 0) break;
+      if (!valid) continue;
+      const bool row_ok = i < sq;
+      // this row's visible keys relative to the item's first key: [rlo, rhi) (empty if no row)
+      int rlo = 0, rhi = 0;
+      if (row_ok) {
+        long long l_, h_;
+        row_key_range(i, sq, sk, a.left, a.right, l_, h_);
+        rlo = (int)(l_ - klo0);
+        rhi = (int)(h_ - klo0);
+      }
+      float m = a.sink ? a.sink[h] * kLog2e : kNegInf, l = 0.f;
+      const int ph = sc_u - j0;                   // s_full / pv_done phase of tile j is ph + j
+      bool ok = true;
 
-    for (int jj = 0; jj < nU; ++jj) {
-      const int j = x.j0 + jj;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(u), jj & 1, a.status))) { ok = false; break; }
-      tc_fence_after();
-      const int klo = rlo - j * kBN, khi = rhi - j * kBN;   // visible columns [klo, khi)
-      const bool full = klo <= 0 && khi >= kBN;
-      // the whole S row in one read (one TMEM round trip on the critical path)
-      uint32_t sr[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-      tmem_wait_ld();
-      if (!full) {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c < klo || c >= khi) sr[c] = __float_as_uint(kNegInf);
-      }
-      // row max over 8 independent chains (a single chain would be 128 dependent steps)
-      float mxv[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mxv[e] = __uint_as_float(sr[e]);
-#pragma unroll
-      for (int c = 8; c < kBN; ++c) mxv[c & 7] = fmaxf(mxv[c & 7], __uint_as_float(sr[c]));
-#pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-        for (int e = 0; e < w; ++e) mxv[e] = fmaxf(mxv[e], mxv[e + w]);
-      const float mx = mxv[0];
-      const float m_tile = mx * scale2;
-      const bool need = m_tile > m + kRescaleThreshold;
-      float alpha = 1.f;
-      if (need) {
-        alpha = (m == kNegInf) ? 0.f : ex2(m - m_tile);
-        m = m_tile;
-      }
-      const bool any_rescale = __any_sync(0xffffffffu, need);
-      // P = 2^{S scale log2e - m} as bf16, over S columns already read, 64 keys at a time.
-      // Masked scores are -inf and 2^-inf = +0, so they need no test; m = -inf only when
-      // every score is -inf (then neg_m = 0 keeps the argument -inf, not NaN).
-      const float neg_m = (m == kNegInf) ? 0.f : -m;
-      float sv[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c]), scale2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c + 1]), scale2, neg_m));
-          sv[c & 3] += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + hh * 32, pk);
-      }
-      const float sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
-      l = l * alpha + sum;
-
-      if (any_rescale && jj >= 1) {
-        // O holds sum of the earlier P V: wait for the last of those MMAs, then scale rows
-        if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (jj - 1) & 1, a.status))) {
-          ok = false;
-          break;
-        }
+      for (int j = j0; j < j1; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(u), (ph + j) & 1, a.status))) { ok = false; break; }
         tc_fence_after();
+        const int klo = rlo - j * kBN, khi = rhi - j * kBN;   // visible columns [klo, khi)
+        const bool full = klo <= 0 && khi >= kBN;
+        // the whole S row in one read (one TMEM round trip on the critical path)
+        uint32_t sr[kBN];
 #pragma unroll
-        for (int c = 0; c < DV / 32; ++c) {
-          uint32_t o[32];
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c < klo || c >= khi) sr[c] = __float_as_uint(kNegInf);
+        }
+        // row max over 8 independent chains (a single chain would be 128 dependent steps)
+        float mxv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mxv[e] = __uint_as_float(sr[e]);
+#pragma unroll
+        for (int c = 8; c < kBN; ++c) mxv[c & 7] = fmaxf(mxv[c & 7], __uint_as_float(sr[c]));
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) mxv[e] = fmaxf(mxv[e], mxv[e + w]);
+        const float mx = mxv[0];
+        const float m_tile = mx * scale2;
+        const bool need = m_tile > m + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+          alpha = (m == kNegInf) ? 0.f : ex2(m - m_tile);
+          m = m_tile;
+        }
+        const bool any_rescale = __any_sync(0xffffffffu, need);
+        // P = 2^{S scale log2e - m} as bf16, over S columns already read, 64 keys at a time.
+        // Masked scores are -inf and 2^-inf = +0, so they need no test; m = -inf only when
+        // every score is -inf (then neg_m = 0 keeps the argument -inf, not NaN).
+        const float neg_m = (m == kNegInf) ? 0.f : -m;
+        float sv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c]), scale2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c + 1]), scale2, neg_m));
+            sv[c & 3] += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + hh * 32, pk);
+        }
+        const float sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+        l = l * alpha + sum;
+
+        if (any_rescale && j > j0) {
+          // O holds sum of the earlier P V: wait for the last of those MMAs, then scale rows
+          if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (ph + j - 1) & 1, a.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < DV / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar.p_full(u));
+      }
+      if (!ok) break;
+
+      // ---- epilogue: out = O / (l + 2^{sink2 - m}),  lse = (m + log2 l) ln 2 ---------------
+      // The next item's first PV_u overwrites O_u only after this unit's next P arrival,
+      // which these warps make after the reads below.
+      const bool have_o = j1 > j0;
+      if (have_o) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (ph + j1 - 1) & 1, a.status))) break;
+        tc_fence_after();
+      }
+      sc_u += j1 - j0;
+      const float sink2 = a.sink ? a.sink[h] * kLog2e : kNegInf;
+      const float e_sink = (sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m);
+      const float den = l + e_sink;
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const long long grow = (long long)q0 + i;   // packed row of this thread's query
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+      uint4* orow = reinterpret_cast<uint4*>(out + (grow * a.hq + h) * DV);
+#pragma unroll
+      for (int c = 0; c < DV / 32; ++c) {
+        uint32_t o[32];
+        if (have_o) {
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
+        } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + c * 32, o);
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        if (row_ok) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            orow[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      tmem_wait_st();
+      if (row_ok && a.lse)
+        a.lse[(long long)h * a.total_q + grow] = l > 0.f ? (m + __log2f(l)) * kLn2 : kNegInf;
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar.p_full(u));
     }
-
-    // ---- epilogue: out = O / (l + 2^{sink2 - m}),  lse = (m + log2 l) ln 2 -----------------
-    const bool have_o = __all_sync(0xffffffffu, ok && nU > 0 &&
-                                   mbar_wait(bar.pv_done(u), (nU - 1) & 1, a.status));
-    tc_fence_after();
-    const float e_sink = (sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m);
-    const float den = l + e_sink;
-    const float inv = (den > 0.f && have_o) ? 1.f / den : 0.f;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
-    uint4* orow = reinterpret_cast<uint4*>(out + ((q0 + i) * a.hq + x.h) * DV);
-#pragma unroll
-    for (int c = 0; c < DV / 32; ++c) {
-      uint32_t o[32];
-      if (nU > 0) {
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
-      }
-      uint32_t pk[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-      if (row_ok) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          orow[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-      }
-    }
-    if (row_ok && a.lse)
-      a.lse[(long long)x.h * a.total_q + q0 + i] = (l > 0.f && have_o) ? (m + __log2f(l)) * kLn2 : kNegInf;
   }
 
   tc_fence_before();
@@ -483,21 +733,62 @@ bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Multiprocessors and opt-in shared memory per block of the current device (cached per device).
+struct DeviceShape {
+  int sms = 0, smem_optin = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceShape g_shape[kMaxDevices];
+
+cudaError_t device_shape(DeviceShape& out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DeviceShape& d = g_shape[dev];
+  if (d.sms == 0) {
+    int sms = 0, optin = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+    d.smem_optin = optin;
+    d.sms = sms;
+  }
+  out = d;
+  return cudaSuccess;
+}
+
+// Levels of the longest sequence and unit pairs per level (see Sched).
+void schedule_shape(const FwdArgs& a, int& zmax, int& width) {
+  const int mtiles = (a.max_sq + kBM - 1) / kBM;
+  const int group = a.hq / a.hkv;
+  const bool even = group % 2 == 0;
+  zmax = even ? mtiles : (mtiles + 1) / 2;
+  width = even ? a.hq / 2 : a.hq;
+}
+
 template <int DK, int DV>
 cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   using L = Layout<DK, DV>;
+  int zmax, width;
+  schedule_shape(a, zmax, width);
+  if (zmax <= 0) return cudaSuccess;  // no query rows
+  DeviceShape dev;
+  cudaError_t e = device_shape(dev);
+  if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, a.q, DK, a.hq, a.total_q) || !make_map(&tk, a.k, DK, a.hkv, a.total_k) ||
       !make_map(&tv, a.v, DV, a.hkv, a.total_k))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       L::kSmem);
+  // Persistent launch (one CTA per SM walking the item list) when the item table fits in
+  // shared memory; otherwise one CTA per item of the dense (level, sequence, unit pair) grid.
+  const long long items_ub = (long long)zmax * a.batch * width;
+  const long long smem_p = L::smem_bytes(3LL * zmax + a.batch);
+  Sched sc{zmax, width, smem_p <= dev.smem_optin ? 1 : 0};
+  const long long smem = sc.persistent ? smem_p : L::smem_bytes(0);
+  const long long grid = sc.persistent ? (items_ub < dev.sms ? items_ub : dev.sms) : items_ub;
+  e = cudaFuncSetAttribute(fwd_sm100_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int mtiles = (a.max_sq + kBM - 1) / kBM;
-  const int group = a.hq / a.hkv;
-  // two units per CTA: head pairs of a GQA group (even group size) or row-tile pairs
-  dim3 grid = (group % 2 == 0) ? dim3(a.hq / 2, a.batch, mtiles) : dim3(a.hq, a.batch, (mtiles + 1) / 2);
-  fwd_sm100_kernel<DK, DV><<<grid, kThreads, L::kSmem, s>>>(a, tq, tk, tv);
+  fwd_sm100_kernel<DK, DV><<<(unsigned)grid, kThreads, (size_t)smem, s>>>(a, sc, tq, tk, tv);
   return cudaGetLastError();
 }
 
@@ -506,7 +797,9 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
 bool fwd_sm100_supported(const FwdArgs& a, int dtype) {
   if (dtype != 0 || a.cu_q == nullptr) return false;
   if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
-  if (a.batch > 65535 || (a.max_sq + kBM - 1) / kBM > 65535 || a.hq > 65535) return false;
+  int zmax, width;
+  schedule_shape(a, zmax, width);
+  if ((long long)zmax * a.batch * width > 0x7fffffffLL) return false;  // item numbers are 32-bit
   return encode_fn() != nullptr;
 }
 

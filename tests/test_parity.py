@@ -28,6 +28,10 @@ def _oracle_fwd(p):
                    p.causal, p.window_left, p.window_right)
 
 
+_LENS_A = [int(n) for n in np.random.default_rng(11).integers(0, 700, size=40)] + [0, 1]
+_LENS_B = [int(n) for n in np.random.default_rng(12).integers(1, 900, size=30)]
+_LENS_C = [int(n) for n in np.random.default_rng(13).integers(0, 5, size=9000)]
+
 FWD_CASES = [
     # name, lens_q, lens_k, hq, hkv, dk, dv, causal, wl, wr, sink, dtype
     ("full_d128", [300, 300], [300, 300], 4, 4, 128, 128, False, -1, -1, "normal", "bf16"),
@@ -49,6 +53,16 @@ FWD_CASES = [
     ("fp32_causal_gqa", [70, 1, 130], [90, 5, 130], 4, 2, 128, 64, True, -1, -1, "normal", "fp32"),
     ("fp32_window", [100], [120], 2, 2, 64, 32, True, 20, 0, "normal", "fp32"),
     ("fp32_full_d64", [65, 33], [65, 200], 2, 1, 64, 64, False, -1, -1, "uniform", "fp32"),
+    # More work items than SMs, so the persistent forward's CTAs each take several items of
+    # mixed cost (zero-length and one-row sequences included): row-tile pairs of one head
+    # (odd group), head pairs (even group), and keys longer than queries with a window.
+    ("persistent_odd_group", _LENS_A, _LENS_A, 6, 2, 128, 128, True, -1, -1, "normal", "bf16"),
+    ("persistent_even_group", _LENS_B, _LENS_B, 8, 2, 128, 128, True, -1, -1, "normal", "bf16"),
+    ("persistent_window_sk_gt_sq", _LENS_A, [n + 37 for n in _LENS_A], 4, 4, 128, 64, True, 200, 0,
+     "uniform", "bf16"),
+    # 9000 sequences: the item table would not fit in shared memory, so the forward runs one
+    # CTA per item of the dense grid instead.
+    ("grid_mode_many_sequences", _LENS_C, _LENS_C, 2, 1, 128, 128, True, -1, -1, "normal", "bf16"),
 ]
 
 
@@ -60,6 +74,14 @@ def test_fwd_matches_oracle(case):
     ro, rl = _oracle_fwd(p)
     check_out(to_np(out), ro, dtype)
     check_lse(to_np(lse), rl, dtype)
+
+
+def test_fwd_is_deterministic():
+    """Two runs of the same forward give the same bits (no atomics, fixed item order)."""
+    p = W.random_problem(7, _LENS_B, _LENS_B, 8, 2, 128, 128, True)
+    o1, l1 = run_fwd(p)
+    o2, l2 = run_fwd(p)
+    assert np.array_equal(to_np(o1), to_np(o2)) and np.array_equal(to_np(l1), to_np(l2))
 
 
 def test_fwd_softmax_n_and_vanilla_identity():
