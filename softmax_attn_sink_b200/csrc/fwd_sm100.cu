@@ -587,17 +587,17 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           for (int c = 0; c < kBN; ++c)
             if (c < klo || c >= khi) sr[c] = __float_as_uint(kNegInf);
         }
-        // row max over 8 independent chains (a single chain would be 128 dependent steps)
+        // row max over 8 independent chains of three-input maxima (a single chain would be
+        // 128 dependent steps)
         float mxv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mxv[e] = __uint_as_float(sr[e]);
+        for (int e = 0; e < 8; ++e) mxv[e] = fmaxf(__uint_as_float(sr[e]), __uint_as_float(sr[8 + e]));
 #pragma unroll
-        for (int c = 8; c < kBN; ++c) mxv[c & 7] = fmaxf(mxv[c & 7], __uint_as_float(sr[c]));
+        for (int c = 16; c < kBN; c += 16)
 #pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-          for (int e = 0; e < w; ++e) mxv[e] = fmaxf(mxv[e], mxv[e + w]);
-        const float mx = mxv[0];
+          for (int e = 0; e < 8; ++e)
+            mxv[e] = fmax3(mxv[e], __uint_as_float(sr[c + e]), __uint_as_float(sr[c + 8 + e]));
+        const float mx = fmax3(fmax3(mxv[0], mxv[1], mxv[2]), fmax3(mxv[3], mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7]));
         const float m_tile = mx * scale2;
         const bool need = m_tile > m + kRescaleThreshold;
         float alpha = 1.f;
@@ -610,20 +610,23 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         // Masked scores are -inf and 2^-inf = +0, so they need no test; m = -inf only when
         // every score is -inf (then neg_m = 0 keeps the argument -inf, not NaN).
         const float neg_m = (m == kNegInf) ? 0.f : -m;
-        float sv[4] = {0.f, 0.f, 0.f, 0.f};
+        // two columns per packed multiply-add and per packed sum update
+        const float2 sc2 = make_float2(scale2, scale2), nm2 = make_float2(neg_m, neg_m);
+        float2 sv[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c]), scale2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[hh * 64 + 2 * c + 1]), scale2, neg_m));
-            sv[c & 3] += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
+            const float2 x = ffma2(make_float2(__uint_as_float(sr[hh * 64 + 2 * c]), __uint_as_float(sr[hh * 64 + 2 * c + 1])),
+                                   sc2, nm2);
+            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+            sv[c & 1] = fadd2(sv[c & 1], pp);
+            pk[c] = pack_bf16x2(pp.x, pp.y);
           }
           tmem_st32(tS + hh * 32, pk);
         }
-        const float sum = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+        const float sum = (sv[0].x + sv[0].y) + (sv[1].x + sv[1].y);
         l = l * alpha + sum;
 
         if (any_rescale && j > j0) {
