@@ -67,13 +67,22 @@ def visible_pairs(cu_q, cu_k, hq, causal, window_left=-1, window_right=-1) -> in
 
 
 def source_digest(kernel_file: str) -> str:
-    """sha256[:16] of a kernel source and every header in csrc/ (what its build depends on)."""
-    import glob
+    """sha256[:16] over a kernel source and the project headers it includes, directly or
+    through other headers (what its build depends on), in a fixed order."""
     import hashlib
-    csrc = os.path.join(ROOT, "softmax_attn_sink_b200", "csrc")
+    import re
+    dirs = [os.path.join(ROOT, "softmax_attn_sink_b200", "csrc"), os.path.join(ROOT, "include")]
+    seen, todo = [], [kernel_file]
+    while todo:
+        name = todo.pop()
+        path = next((os.path.join(d, name) for d in dirs if os.path.exists(os.path.join(d, name))), None)
+        if path is None or path in seen:
+            continue
+        seen.append(path)
+        with open(path, encoding="utf-8") as f:
+            todo += re.findall(r'^\s*#\s*include\s+"([^"]+)"', f.read(), flags=re.M)
     h = hashlib.sha256()
-    for path in [os.path.join(csrc, kernel_file)] + sorted(glob.glob(os.path.join(csrc, "*.cuh")) +
-                                                           glob.glob(os.path.join(csrc, "*.h"))):
+    for path in [seen[0]] + sorted(seen[1:]):
         with open(path, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
