@@ -400,15 +400,40 @@ def bench_decode(args, world, peaks, peak_kind):
     algo = kv_bytes + io_bytes
     gbs = algo / (statistics.mean(per) * 1e-3) / 1e9
     pk = peaks["hbm_gbs"]
+    res = {"workload": f"decode{nb}_gqa64x8_d128_L8k-32k", "unit": "GB/s", "steps": steps,
+           "value": round(algo * world / (total / steps * 1e-3) / 1e9, 1),
+           "ms_per_step": round(total / steps, 4), "bytes_per_step": algo, "splits": splits,
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk, "unit": "GB/s",
+                        "frac": round(gbs / pk, 4),
+                        "traffic": kernel_traffic("decode_split.cu") if nb == 64 else None,
+                        "peak_source": f"hbm_gbs ({peak_kind})",
+                        "kernels": "split + merge (two launches per step)"}}
+
+    # the same keys and values in a paged cache: 64-key blocks in a seeded random order
+    bs = 64
+    lens = np.diff(d.cu_seqlens_k)
+    table, n_blocks = W.paged_layout(40, lens, bs)
+    kc = W.to_paged(k, d.cu_seqlens_k, table, bs, n_blocks)
+    vc = W.to_paged(v, d.cu_seqlens_k, table, bs, n_blocks)
     del k, v
-    return {"workload": f"decode{nb}_gqa64x8_d128_L8k-32k", "unit": "GB/s", "steps": steps,
-            "value": round(algo * world / (total / steps * 1e-3) / 1e9, 1),
-            "ms_per_step": round(total / steps, 4), "bytes_per_step": algo, "splits": splits,
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk, "unit": "GB/s",
-                         "frac": round(gbs / pk, 4),
-                         "traffic": kernel_traffic("decode_split.cu") if nb == 64 else None,
-                         "peak_source": f"hbm_gbs ({peak_kind})",
-                         "kernels": "split + merge (two launches per step)"}}
+    tab = torch.from_numpy(table).cuda()
+    used = torch.from_numpy(lens.astype(np.int32)).cuda()
+    per_p, total_p = time_steps(
+        lambda: sab.attn_sink_decode_paged(q, kc, vc, tab, used, mk, sink, d.softmax_scale, True, (-1, -1),
+                                           0, out=out, lse=lse, workspace=ws),
+        steps, args.warmup, world, flush)
+    table_bytes = int(sum(-(-int(n) // bs) for n in lens)) * 4 + used.numel() * 4
+    algo_p = kv_bytes + io_bytes - cu.numel() * 4 + table_bytes
+    gbs_p = algo_p / (statistics.mean(per_p) * 1e-3) / 1e9
+    res["paged"] = {"workload": f"decode{nb}_gqa64x8_d128_L8k-32k_paged{bs}", "unit": "GB/s",
+                    "value": round(algo_p * world / (total_p / steps * 1e-3) / 1e9, 1),
+                    "ms_per_step": round(total_p / steps, 4), "bytes_per_step": algo_p,
+                    "block_size": bs, "num_blocks": n_blocks,
+                    "roofline": {"bound": "hbm", "achieved": round(gbs_p, 1), "peak": pk, "unit": "GB/s",
+                                 "frac": round(gbs_p / pk, 4), "traffic": None,
+                                 "peak_source": f"hbm_gbs ({peak_kind})"}}
+    del kc, vc
+    return res
 
 
 # --- the oracle on the host -------------------------------------------------------------

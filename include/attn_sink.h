@@ -70,7 +70,10 @@ typedef enum {
   ATTN_SINK_ERR_UNSUPPORTED = 2,   /* head dims / dtype outside the supported set     */
   ATTN_SINK_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required      */
   ATTN_SINK_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed            */
-  ATTN_SINK_ERR_TIMEOUT = 5        /* device status: a bounded on-chip wait ran out   */
+  ATTN_SINK_ERR_TIMEOUT = 5,       /* device status: a bounded on-chip wait ran out   */
+  ATTN_SINK_ERR_BAD_INDEX = 6      /* device status: a paged block id, a key count or a
+                                      sequence length fell outside what the call's
+                                      tables and sizes allow; those keys were skipped  */
 } attn_sink_status;
 
 /* Problem description shared by the three entry points (plain struct, by pointer). */
@@ -137,6 +140,35 @@ int attn_sink_decode(const attn_sink_params* params, const void* q, const void* 
                      attn_sink_stream_t stream);
 
 /*
+ * Paged decode: attn_sink_decode with K/V in a block cache (CANN doc, "Paged Attention
+ * Parameter Group", and the PA_BBND layout of k / v in its parameter table).
+ *   k_cache [num_blocks, block_size, Hkv, dk], v_cache [num_blocks, block_size, Hkv, dv]
+ *     (dtype; contiguous).  Key t of sequence b is row t % block_size of block
+ *     block_table[b * max_blocks_per_seq + t / block_size].
+ *   block_table int32 [batch, max_blocks_per_seq]: block ids in [0, num_blocks).  Only the
+ *     first ceil(seqused_k[b] / block_size) entries of row b are read; blocks may be shared
+ *     between sequences and appear in any order.
+ *   seqused_k int32 [batch]: keys of each sequence, 0 <= seqused_k[b] <=
+ *     max_blocks_per_seq * block_size, and <= params->max_seqlen_k.
+ *   16 <= block_size <= 1024 and block_size % 16 == 0 (the CANN doc's range).
+ * params: total_q == batch, max_seqlen_q == 1 as for attn_sink_decode; total_k must equal
+ * num_blocks * block_size; max_seqlen_k bounds every seqused_k[b] (it sizes the chunks).
+ * The query of sequence b sits at key position seqused_k[b] - 1 (bottom-right), so causal
+ * decode sees all of its keys and a window keeps the last window_left + 1 of them.
+ * Writes out [batch, Hq, dv] and, when not NULL, lse [Hq, batch]; the workspace is the one
+ * attn_sink_decode_workspace_size() gives for the same params and num_splits.  bf16 only
+ * (ATTN_SINK_ERR_UNSUPPORTED otherwise).  Table contents are the caller's contract: a
+ * block id outside [0, num_blocks) or a seqused_k beyond its table row is not read (those
+ * keys count as zero vectors) and sets the device status that
+ * attn_sink_get_device_status() reports as ATTN_SINK_ERR_BAD_INDEX.
+ */
+int attn_sink_decode_paged(const attn_sink_params* params, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* block_table, const int32_t* seqused_k,
+                           int num_blocks, int block_size, int max_blocks_per_seq, const float* sink,
+                           int num_splits, void* out, float* lse, void* workspace,
+                           size_t workspace_bytes, attn_sink_stream_t stream);
+
+/*
  * Decode that allocates nothing and takes no workspace.  None of the pages this library
  * follows has a counterpart: it exists for callers that cannot allocate device memory
  * (a plugin or custom-op host that passes only the call's tensors and offers no
@@ -173,7 +205,8 @@ const char* attn_sink_status_string(int status);
 
 /*
  * Synchronises `stream`, then reads and clears the calling device's status word.
- * Returns ATTN_SINK_OK, ATTN_SINK_ERR_TIMEOUT (a bounded wait ran out) or
+ * Returns ATTN_SINK_OK, ATTN_SINK_ERR_TIMEOUT (a bounded wait ran out; bit 0),
+ * ATTN_SINK_ERR_BAD_INDEX (an index or length outside its table was skipped; bit 1) or
  * ATTN_SINK_ERR_CUDA.  *bits (if not NULL) receives the raw word.
  */
 int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits);

@@ -33,8 +33,11 @@ Sources, by page and section:
 * Decode split + LSE merge -- CANN doc, the ``softmax_lse`` note (partial results of
   ring attention are combined through max / sum / log); the sink enters once, after
   the partials are combined.
+* Paged K/V -- CANN doc, "Paged Attention Parameter Group" (block_table (B,
+  max_num_blocks_per_seq) int32, block_size in [16, 1024] and a multiple of 16, seqused_kv)
+  and the PA_BBND layout of k / v, (num_blocks, block_size, KV_N, D).
 
-Readings where the pages are silent (also listed in the design doc): a row with no visible
+Readings where the pages are silent: a row with no visible
 key has lse = -inf; with sink = -inf as well its output is 0; the window is measured
 from the bottom-right diagonal and causal clamps right to min(right, 0).
 """
@@ -191,6 +194,35 @@ def decode(q, k, v, cu_seqlens_k, sink, softmax_scale: float, causal: bool = Tru
     b = q.shape[0]
     cu_q = np.arange(b + 1, dtype=np.int64)
     return fwd(q, k, v, cu_q, cu_seqlens_k, sink, softmax_scale, causal, window_left, window_right)
+
+
+def gather_paged(cache, block_table, seqused_k, block_size: int):
+    """Keys (or values) of each sequence read through its block-table row: key t of
+    sequence b is row t % block_size of block block_table[b, t // block_size] of a cache
+    [num_blocks, block_size, H, d] (CANN flash_attn doc, "Paged Attention Parameter Group";
+    the PA_BBND layout (num_blocks, block_size, KV_N, D) of its parameter table).
+    Returns the packed rows [sum seqused_k, H, d] and their cu_seqlens."""
+    cache = np.asarray(cache)
+    table = np.asarray(block_table)
+    used = [int(n) for n in np.asarray(seqused_k)]
+    rows = []
+    for b, n in enumerate(used):
+        t = np.arange(n)
+        rows.append(cache[table[b, t // block_size], t % block_size])
+    cu = np.zeros(len(used) + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(used)
+    packed = np.concatenate(rows, axis=0) if rows else cache[:0, 0]
+    return packed, cu
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seqused_k, block_size: int, sink,
+                 softmax_scale: float, causal: bool = True, window_left: int = -1,
+                 window_right: int = -1):
+    """Decode over a paged K/V cache: the plain decode of the keys and values each
+    sequence's block-table row names.  Returns out [B, Hq, dv], lse [Hq, B]."""
+    k, cu = gather_paged(k_cache, block_table, seqused_k, block_size)
+    v, _ = gather_paged(v_cache, block_table, seqused_k, block_size)
+    return decode(q, k, v, cu, sink, softmax_scale, causal, window_left, window_right)
 
 
 # --- split-KV partials and the LSE merge --------------------------------------------

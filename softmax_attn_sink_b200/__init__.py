@@ -66,7 +66,8 @@ def lib() -> ctypes.CDLL:
         L.attn_sink_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.attn_sink_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.attn_sink_decode.argtypes = [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]
-        for f in (L.attn_sink_fwd, L.attn_sink_bwd, L.attn_sink_decode):
+        L.attn_sink_decode_paged.argtypes = [P, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, sz, vp]
+        for f in (L.attn_sink_fwd, L.attn_sink_bwd, L.attn_sink_decode, L.attn_sink_decode_paged):
             f.restype = i32
         for f in (L.attn_sink_fwd_workspace_size, L.attn_sink_bwd_workspace_size):
             f.argtypes, f.restype = [P], sz
@@ -249,6 +250,53 @@ def attn_sink_decode(q, k, v, cu_seqlens_k, max_seqlen_k: int, sink=None,
     return out, lse
 
 
+def attn_sink_decode_paged(q, k_cache, v_cache, block_table, seqused_k, max_seqlen_k: int, sink=None,
+                           softmax_scale: Optional[float] = None, causal: bool = True,
+                           window_size: Sequence[int] = (-1, -1), num_splits: int = 0, out=None,
+                           lse=None, return_lse=True, workspace=None, stream=None):
+    """Split-KV decode over a paged K/V cache: q [B, Hq, dk], k_cache [num_blocks,
+    block_size, Hkv, dk], v_cache [num_blocks, block_size, Hkv, dv], block_table int32
+    [B, max_blocks_per_seq], seqused_k int32 [B].  Returns (out, lse)."""
+    torch = _torch()
+    _require(q, "q", ndim=3)
+    _require(k_cache, "k_cache", q.dtype, 4)
+    _require(v_cache, "v_cache", q.dtype, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(seqused_k, "seqused_k", torch.int32, 1)
+    if sink is not None:
+        _require(sink, "sink", torch.float32, 1)
+        if sink.shape[0] != q.shape[1]:
+            raise ValueError("sink must have one value per q head")
+    num_blocks, block_size = k_cache.shape[0], k_cache.shape[1]
+    if tuple(v_cache.shape[:3]) != (num_blocks, block_size, k_cache.shape[2]):
+        raise ValueError("k_cache and v_cache must share [num_blocks, block_size, Hkv]")
+    if block_table.shape[0] != q.shape[0] or seqused_k.shape[0] != q.shape[0]:
+        raise ValueError("block_table and seqused_k need one row / entry per sequence")
+    scale = 1.0 / math.sqrt(q.shape[-1]) if softmax_scale is None else float(softmax_scale)
+    wl, wr = window_size
+    p = make_params(batch=q.shape[0], total_q=q.shape[0], total_k=num_blocks * block_size,
+                    max_seqlen_q=1, max_seqlen_k=max_seqlen_k, num_heads_q=q.shape[1],
+                    num_heads_kv=k_cache.shape[2], head_dim_qk=q.shape[2], head_dim_v=v_cache.shape[3],
+                    softmax_scale=scale, causal=causal, window_left=wl, window_right=wr,
+                    dtype=_dtype_code(q))
+    if out is None:
+        out = torch.empty((q.shape[0], q.shape[1], v_cache.shape[3]), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    ws_bytes = lib().attn_sink_decode_workspace_size(ctypes.byref(p), int(num_splits))
+    if ws_bytes == ctypes.c_size_t(-1).value:
+        raise AttnSinkError("attn_sink_decode_workspace_size", 1)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_sink_decode_paged(ctypes.byref(p), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                      block_table.data_ptr(), seqused_k.data_ptr(), int(num_blocks),
+                                      int(block_size), int(block_table.shape[1]), _ptr(sink),
+                                      int(num_splits), out.data_ptr(), _ptr(lse), workspace.data_ptr(),
+                                      workspace.numel(), _stream(stream))
+    _check("attn_sink_decode_paged", st)
+    return out, lse
+
+
 def decode_num_splits(batch, max_seqlen_k, total_k, num_heads_q, num_heads_kv, head_dim_qk,
                       head_dim_v, dtype=ATTN_SINK_BF16) -> int:
     p = make_params(batch=batch, total_q=batch, total_k=total_k, max_seqlen_q=1,
@@ -304,6 +352,6 @@ class SinkAttention:
         return cls._fn.apply(*args)
 
 
-__all__ = ["attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "decode_num_splits",
+__all__ = ["attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "attn_sink_decode_paged", "decode_num_splits",
            "device_status", "selftest_wait_timeout", "SinkAttention", "AttnSinkError", "AttnSinkParams", "make_params",
            "lib", "LIB_PATH", "ATTN_SINK_BF16", "ATTN_SINK_FP32"]

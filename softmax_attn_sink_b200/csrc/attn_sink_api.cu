@@ -12,7 +12,8 @@ using namespace attn_sink;
 
 namespace {
 
-// Bits set by kernels whose bounded waits ran out (kStatusTimeout).
+// Bits set by kernels: a bounded wait ran out (kStatusTimeout), an index or length outside
+// its table was skipped (kStatusBadIndex).
 __device__ unsigned int g_status_word;
 
 constexpr int kMaxDevices = 64;
@@ -102,6 +103,24 @@ size_t decode_ws(const attn_sink_params* p, int splits) {
   return align_up(rows * p->head_dim_v * 4, 256) + align_up(rows * 2 * 4, 256);
 }
 
+// Split + merge launch shared by the packed and paged decode entry points: workspace check,
+// partial-buffer layout and the remaining DecodeArgs fields.
+int launch_decode(const attn_sink_params* p, DecodeArgs& a, int num_splits, void* workspace,
+                  size_t workspace_bytes, int left, int right, cudaStream_t s) {
+  const int splits = num_splits == 0 ? decode_auto_splits(p) : num_splits;
+  const size_t need = decode_ws(p, splits);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
+  const size_t rows = (size_t)p->batch * p->num_heads_q * splits;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  a.part_o = reinterpret_cast<float*>(ws);
+  a.part_ml = reinterpret_cast<float*>(ws + align_up(rows * p->head_dim_v * 4, 256));
+  a.batch = p->batch; a.total_k = p->total_k; a.max_sk = p->max_seqlen_k;
+  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
+  a.splits = splits; a.scale = p->softmax_scale; a.left = left; a.right = right;
+  a.status = status_ptr();
+  return from_cuda(launch_decode_split(a, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -116,6 +135,7 @@ const char* attn_sink_status_string(int status) {
     case ATTN_SINK_ERR_WORKSPACE: return "workspace missing or too small";
     case ATTN_SINK_ERR_CUDA: return "CUDA error";
     case ATTN_SINK_ERR_TIMEOUT: return "a bounded on-chip wait timed out";
+    case ATTN_SINK_ERR_BAD_INDEX: return "an index or length outside its table was skipped on the device";
     default: return "unknown status";
   }
 }
@@ -226,20 +246,35 @@ int attn_sink_decode(const attn_sink_params* p, const void* q, const void* k, co
     a.status = status_ptr();
     return from_cuda(launch_fwd_simt(a, 1, s));
   }
-  const int splits = num_splits == 0 ? decode_auto_splits(p) : num_splits;
-  const size_t need = decode_ws(p, splits);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
-  const size_t rows = (size_t)p->batch * p->num_heads_q * splits;
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
   DecodeArgs a{};
   a.q = q; a.k = k; a.v = v; a.cu_k = cu_seqlens_k; a.sink = sink; a.out = out; a.lse = lse;
-  a.part_o = reinterpret_cast<float*>(ws);
-  a.part_ml = reinterpret_cast<float*>(ws + align_up(rows * p->head_dim_v * 4, 256));
-  a.batch = p->batch; a.total_k = p->total_k; a.max_sk = p->max_seqlen_k;
-  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
-  a.splits = splits; a.scale = p->softmax_scale; a.left = left; a.right = right;
-  a.status = status_ptr();
-  return from_cuda(launch_decode_split(a, s));
+  return launch_decode(p, a, num_splits, workspace, workspace_bytes, left, right, s);
+}
+
+int attn_sink_decode_paged(const attn_sink_params* p, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* block_table, const int32_t* seqused_k,
+                           int num_blocks, int block_size, int max_blocks_per_seq, const float* sink,
+                           int num_splits, void* out, float* lse, void* workspace,
+                           size_t workspace_bytes, attn_sink_stream_t stream) {
+  int st = validate_params(p, true);
+  if (st != ATTN_SINK_OK) return st;
+  if (p->dtype != ATTN_SINK_BF16) return ATTN_SINK_ERR_UNSUPPORTED;
+  if (num_splits < 0) return ATTN_SINK_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !block_table || !seqused_k || !out) return ATTN_SINK_ERR_INVALID_ARG;
+  if (block_size < 16 || block_size > 1024 || block_size % 16 != 0) return ATTN_SINK_ERR_INVALID_ARG;
+  if (num_blocks <= 0 || max_blocks_per_seq <= 0) return ATTN_SINK_ERR_INVALID_ARG;
+  if ((long long)num_blocks * block_size != p->total_k) return ATTN_SINK_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k_cache, v_cache, (const void*)out})
+    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
+  if ((lse && !aligned16(lse)) || (sink && !aligned16(sink))) return ATTN_SINK_ERR_INVALID_ARG;
+  int left, right;
+  effective_window(p, left, right);
+  DecodeArgs a{};
+  a.q = q; a.k = k_cache; a.v = v_cache; a.cu_k = nullptr; a.sink = sink; a.out = out; a.lse = lse;
+  a.block_table = block_table; a.seqused_k = seqused_k;
+  a.block_size = block_size; a.max_blocks = max_blocks_per_seq; a.num_blocks = num_blocks;
+  return launch_decode(p, a, num_splits, workspace, workspace_bytes, left, right,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int attn_sink_selftest_wait_timeout(attn_sink_stream_t stream) {
@@ -258,7 +293,8 @@ int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits) {
   if (cudaMemsetAsync(sp, 0, sizeof(unsigned), s) != cudaSuccess) return ATTN_SINK_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_SINK_ERR_CUDA;
   if (bits) *bits = host;
-  return host ? ATTN_SINK_ERR_TIMEOUT : ATTN_SINK_OK;
+  if (host & kStatusTimeout) return ATTN_SINK_ERR_TIMEOUT;
+  return host ? ATTN_SINK_ERR_BAD_INDEX : ATTN_SINK_OK;
 }
 
 }  // extern "C"

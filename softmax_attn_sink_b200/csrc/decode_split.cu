@@ -1,4 +1,7 @@
-// Split-KV decode for bf16: one query per sequence, GQA heads of a kv head together.
+// Split-KV decode for bf16: one query per sequence, GQA heads of a kv head together.  K/V
+// are either packed ([total_k, hkv, d] with cu_seqlens_k) or paged ([num_blocks, block_size,
+// hkv, d] with a block table and per-sequence key counts; CANN flash_attn doc, "Paged
+// Attention Parameter Group" and the PA_BBND layout of k in its parameter table).
 //
 // Work unit: (sequence b, kv head g, block of up to 16 q heads of g's group, key chunk c).
 // The visible keys of a decode query form one contiguous range [vlo, vhi) (bottom-right
@@ -79,16 +82,35 @@ __device__ __forceinline__ int swz(int row, int c) {
   return c ^ (row & M);
 }
 
-// Visible key range of the single decode query of sequence b.
+// Visible key range of the single decode query of sequence b.  Packed K/V: the sequence's
+// keys start at row k0 = cu_k[b].  Paged K/V: k0 = 0 and the key count is seqused_k[b],
+// clamped (with the status bit set) to what the sequence's block-table row can address.
 __device__ __forceinline__ void decode_range(const DecodeArgs& a, int b, long long& k0,
                                              long long& vlo, long long& vhi) {
-  k0 = a.cu_k[b];
-  const long long sk = a.cu_k[b + 1] - k0;
+  long long sk;
+  if (a.block_table) {
+    k0 = 0;
+    sk = a.seqused_k[b];
+    const long long cap = (long long)a.max_blocks * a.block_size;
+    if (sk < 0 || sk > cap) {
+      set_status(a.status, kStatusBadIndex);
+      sk = sk < 0 ? 0 : cap;
+    }
+  } else {
+    k0 = a.cu_k[b];
+    sk = a.cu_k[b + 1] - k0;
+  }
   row_key_range(0, 1, sk, a.left, a.right, vlo, vhi);
 }
 
-template <int DK, int DV>
-__global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const DecodeArgs a, int chunk) {
+// K/V addressing of the split kernel: packed rows, or a block table read from shared memory
+// (the chunk's block ids staged once per CTA) or, when they do not fit, from global memory.
+enum KvMode { kPacked = 0, kPagedSmemTable = 1, kPagedGlobalTable = 2 };
+
+template <int DK, int DV, int MODE>
+__global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const DecodeArgs a, int chunk,
+                                                                       int extra_off) {
+  constexpr bool PAGED = MODE != kPacked;
   constexpr int KCH = DK / 8, VCH = DV / 8;        // 16-byte chunks per row
   constexpr int KSTEPS = DK / 16, VTILES = DV / 8;
   constexpr int STAGE_BYTES = kStageKeys * (DK + DV) * 2;
@@ -113,22 +135,78 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
   const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* vp = static_cast<const __nv_bfloat16*>(a.v);
   const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q);
+  // Paged K/V: the cache row of every key of a stage is computed once, by one thread per key,
+  // into s_row (kStages stage slots of 64 rows, -1 = no key or a block id outside the cache)
+  // one iteration before the stage's copies are issued; the copies then read it like the
+  // packed path reads k0 + t.  With the shared-memory table, the chunk's block ids
+  // [first block, last block] are staged once per CTA in s_blk.
+  const unsigned bs = PAGED ? (unsigned)a.block_size : 1u;
+  const bool bs_pow2 = (bs & (bs - 1)) == 0;
+  const int bs_log2 = __ffs((int)bs) - 1;
+  const long long blk_first = PAGED ? c_lo / bs : 0;
+  long long* s_row = reinterpret_cast<long long*>(smem + extra_off);
+  int* s_blk = reinterpret_cast<int*>(smem + extra_off + kStages * kStageKeys * 8);
+  const int* trow = PAGED ? a.block_table + (long long)b * a.max_blocks : nullptr;
+  if constexpr (MODE == kPagedSmemTable) {
+    const int n_blk = (int)((c_hi - 1) / bs - blk_first + 1);
+    for (int i = tid; i < n_blk; i += kWarps * 32) s_blk[i] = trow[blk_first + i];
+    __syncthreads();
+  }
+  auto compute_rows = [&](int st) {
+    if (tid < kStageKeys) {
+      const long long t = c_lo + (long long)st * kStageKeys + tid;
+      long long row = -1;
+      if (t < c_hi) {
+        const unsigned tu = (unsigned)t;   // keys are below 2^31
+        const unsigned q = bs_pow2 ? tu >> bs_log2 : tu / bs;
+        const int blk = (MODE == kPagedSmemTable) ? s_blk[q - (unsigned)blk_first] : trow[q];
+        if ((unsigned)blk < (unsigned)a.num_blocks)
+          row = (long long)blk * bs + (bs_pow2 ? (tu & (bs - 1)) : tu % bs);
+        else
+          set_status(a.status, kStatusBadIndex);
+      }
+      s_row[(st % kStages) * kStageKeys + tid] = row;
+    }
+  };
+  if constexpr (PAGED) {
+#pragma unroll
+    for (int st = 0; st < kStages; ++st) compute_rows(st);
+    __syncthreads();
+  }
 
   auto issue_stage = [&](int st) {
     unsigned char* base = smem + (st % kStages) * STAGE_BYTES;
     const uint32_t k_s = smem_u32(base), v_s = smem_u32(base + kStageKeys * DK * 2);
     const long long t0 = c_lo + (long long)st * kStageKeys;
-    for (int idx = tid; idx < kStageKeys * KCH; idx += kWarps * 32) {
-      const int r = idx / KCH, ch = idx % KCH;
-      const bool ok = t0 + r < c_hi;
-      const __nv_bfloat16* src = ok ? kp + ((k0 + t0 + r) * a.hkv + g) * DK + ch * 8 : kp;
-      cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, src, ok);
-    }
-    for (int idx = tid; idx < kStageKeys * VCH; idx += kWarps * 32) {
-      const int r = idx / VCH, ch = idx % VCH;
-      const bool ok = t0 + r < c_hi;
-      const __nv_bfloat16* src = ok ? vp + ((k0 + t0 + r) * a.hkv + g) * DV + ch * 8 : vp;
-      cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, src, ok);
+    if constexpr (!PAGED) {
+      for (int idx = tid; idx < kStageKeys * KCH; idx += kWarps * 32) {
+        const int r = idx / KCH, ch = idx % KCH;
+        const bool ok = t0 + r < c_hi;
+        const __nv_bfloat16* src = ok ? kp + ((k0 + t0 + r) * a.hkv + g) * DK + ch * 8 : kp;
+        cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, src, ok);
+      }
+      for (int idx = tid; idx < kStageKeys * VCH; idx += kWarps * 32) {
+        const int r = idx / VCH, ch = idx % VCH;
+        const bool ok = t0 + r < c_hi;
+        const __nv_bfloat16* src = ok ? vp + ((k0 + t0 + r) * a.hkv + g) * DV + ch * 8 : vp;
+        cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, src, ok);
+      }
+    } else {
+      const long long* rows = s_row + (st % kStages) * kStageKeys;
+      for (int idx = tid; idx < kStageKeys * KCH; idx += kWarps * 32) {
+        const int r = idx / KCH, ch = idx % KCH;
+        const long long row = rows[r];
+        const bool ok = row >= 0;
+        const __nv_bfloat16* src = ok ? kp + (row * a.hkv + g) * DK + ch * 8 : kp;
+        cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, src, ok);
+      }
+      for (int idx = tid; idx < kStageKeys * VCH; idx += kWarps * 32) {
+        const int r = idx / VCH, ch = idx % VCH;
+        const long long row = rows[r];
+        const bool ok = row >= 0;
+        const __nv_bfloat16* src = ok ? vp + (row * a.hkv + g) * DV + ch * 8 : vp;
+        cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, src, ok);
+      }
     }
   };
 
@@ -167,6 +245,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
     __syncthreads();
     if (st + kStages - 1 < nstages) issue_stage(st + kStages - 1);
     cp_async_commit();
+    // the slot of stage st (issued two iterations ago) now takes stage st + kStages's rows;
+    // the barrier at the top of the next iteration orders these writes before their reads
+    if constexpr (PAGED)
+      if (st + kStages < nstages) compute_rows(st + kStages);
 
     const unsigned char* base = smem + (st % kStages) * STAGE_BYTES;
     const uint32_t k_s = smem_u32(base), v_s = smem_u32(base + kStageKeys * DK * 2);
@@ -302,7 +384,11 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, i
   const int b = (int)(row / a.hq), h = (int)(row % a.hq);
   long long k0, vlo, vhi;
   decode_range(a, b, k0, vlo, vhi);
-  const int n = vhi > vlo ? (int)((vhi - vlo + chunk - 1) / chunk) : 0;
+  int n = vhi > vlo ? (int)((vhi - vlo + chunk - 1) / chunk) : 0;
+  if (n > a.splits) {  // more keys than max_seqlen_k announced: only a.splits chunks exist
+    set_status(a.status, kStatusBadIndex);
+    n = a.splits;
+  }
   const float* ml = a.part_ml + row * a.splits * 2;
   float M = kNegInf;
   for (int c = lane; c < n; c += 32) M = fmaxf(M, ml[2 * c]);
@@ -333,6 +419,17 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, i
     a.lse[(long long)h * a.batch + b] = (M == kNegInf || lM <= 0.f) ? kNegInf : (M + __log2f(lM)) * kLn2;
 }
 
+template <int DK, int DV, int MODE>
+cudaError_t launch_split(const DecodeArgs& a, int chunk, int smem, int extra_off, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<DK, DV, MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int group = a.hq / a.hkv;
+  dim3 grid(a.splits, a.hkv * ((group + 15) / 16), a.batch);
+  decode_split_kernel<DK, DV, MODE><<<grid, kWarps * 32, smem, s>>>(a, chunk, extra_off);
+  return cudaGetLastError();
+}
+
 template <int DK, int DV>
 cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
   const int group = a.hq / a.hkv;
@@ -343,12 +440,21 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
   constexpr int PIPE = kStages * STAGE_BYTES;
   constexpr int COMBINE = kWarps * 16 * (DV + 2) * 4;
   constexpr int SMEM = PIPE > COMBINE ? PIPE : COMBINE;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<DK, DV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  (void)hblocks;
+  const int ch = chunk > 0 ? chunk : 1;
+  cudaError_t e;
+  if (!a.block_table) {
+    e = launch_split<DK, DV, kPacked>(a, ch, SMEM, 0, s);
+  } else {
+    // a chunk spans at most ch / block_size + 2 blocks; stage their ids in shared memory
+    // when that keeps two CTAs per SM (113 KB each), else read the table from global memory
+    const long long rows = kStages * kStageKeys * 8;
+    const long long ids = (long long)ch / a.block_size + 2;
+    const long long smem_t = (long long)SMEM + rows + 4 * ((ids + 31) / 32 * 32);
+    e = smem_t <= 113 * 1024 ? launch_split<DK, DV, kPagedSmemTable>(a, ch, (int)smem_t, SMEM, s)
+                             : launch_split<DK, DV, kPagedGlobalTable>(a, ch, SMEM + (int)rows, SMEM, s);
+  }
   if (e != cudaSuccess) return e;
-  dim3 grid(a.splits, a.hkv * hblocks, a.batch);
-  decode_split_kernel<DK, DV><<<grid, kWarps * 32, SMEM, s>>>(a, chunk > 0 ? chunk : 1);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long rows = (long long)a.batch * a.hq;
   decode_merge_kernel<DV><<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(a, chunk > 0 ? chunk : 1);
   return cudaGetLastError();

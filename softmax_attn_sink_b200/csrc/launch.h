@@ -13,6 +13,7 @@ constexpr int kUnbounded = 1 << 30;
 
 // Bits of the per-device status word.
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusBadIndex = 2u;  // a paged block id or key count outside its table
 
 struct FwdArgs {
   const void* q;
@@ -66,6 +67,12 @@ struct DecodeArgs {
   float scale;
   int left, right;
   unsigned* status;
+  // Paged K/V (block_table != nullptr): k/v are caches [num_blocks, block_size, hkv, d];
+  // key t of sequence b is row t % block_size of block block_table[b * max_blocks +
+  // t / block_size]; sequence b has seqused_k[b] keys and cu_k is unused.
+  const int32_t* block_table;
+  const int32_t* seqused_k;
+  int block_size, max_blocks, num_blocks;
 };
 
 // dtype: 0 = bf16, 1 = fp32.  Each returns cudaSuccess or the launch error.

@@ -114,3 +114,22 @@ def test_python_binding_requires_cuda_tensors():
     cu = torch.tensor([0, 4], dtype=torch.int32)
     with pytest.raises(ValueError):
         sab.attn_sink_fwd(q, q, q, cu, cu, 4, 4)
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(block_size=40), 1), (dict(block_size=8), 1), (dict(block_size=2048), 1),
+    (dict(num_blocks=3), 1), (dict(max_blocks=0), 1), (dict(table=None), 1),
+    (dict(dtype=sab.ATTN_SINK_FP32), 2), (dict(total_q=5), 1),
+])
+def test_paged_decode_rejects_bad_arguments_on_host(change, status):
+    """The paged decode validates its table shape and block size before any launch (fake,
+    aligned, non-null device addresses: nothing is dereferenced)."""
+    a = dict(block_size=16, num_blocks=4, max_blocks=2, table=256, dtype=sab.ATTN_SINK_BF16, total_q=2)
+    a.update(change)
+    p = _params(batch=2, total_q=a["total_q"], total_k=64, max_seqlen_q=1, max_seqlen_k=32,
+                dtype=a["dtype"])
+    fake = 4096
+    st = sab.lib().attn_sink_decode_paged(ctypes.byref(p), fake, fake, fake, a["table"], fake,
+                                          a["num_blocks"], a["block_size"], a["max_blocks"], None, 0,
+                                          fake, None, fake, 1 << 20, None)
+    assert st == status

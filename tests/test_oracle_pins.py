@@ -285,7 +285,7 @@ def test_p9_gradients_match_finite_differences():
         assert rel <= 1e-6, (name, rel)
 
 
-# --- P10: the page-1 form of the backward -----------------------------------------------
+# --- P10: the backward in the form of the slime docstring -----------------------------------
 
 def test_p10_learnable_offset_backward_form():
     p = W.random_problem(10, [9], [9], hq=2, hkv=1, dk=5, dv=4, dtype="fp32", with_dout=True,
@@ -386,7 +386,7 @@ def test_p12_sink_in_every_split_is_wrong():
 def test_decode_equals_fwd_with_one_query_per_sequence():
     d = W.random_decode(17, [5, 9], hq=2, hkv=1, dk=4, dv=4)
     out, lse = ref.decode(d.q, d.k, d.v, d.cu_seqlens_k, d.sink, d.softmax_scale)
-    # the page-5 decode example: the one query sees every cached key
+    # the decode example of PyTorch issue #108108 ("Benefits"): the one query sees every cached key
     for b, (k0, k1) in enumerate([(0, 5), (5, 14)]):
         for h in range(2):
             S = d.softmax_scale * (d.k[k0:k1, 0].astype(np.float64) @ d.q[b, h].astype(np.float64))
@@ -424,3 +424,69 @@ def test_bf16_rounding_matches_torch():
     ours = W.bf16_round(x)
     theirs = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
     np.testing.assert_array_equal(ours, theirs)
+
+
+# --- P13: paged K/V (CANN flash_attn doc, "Paged Attention Parameter Group", PA_BBND) ----
+
+def test_p13_paged_gather_literal():
+    """Key t of a sequence is row t % block_size of block table[t // block_size]: a cache
+    whose row r of block p holds (p, r), read through the table [2, 0] for 20 keys with
+    block_size 16, gives (2, 0) ... (2, 15), then (0, 0) ... (0, 3)."""
+    bs, nb = 16, 3
+    cache = np.zeros((nb, bs, 1, 2))
+    for p_ in range(nb):
+        for r in range(bs):
+            cache[p_, r, 0] = (p_, r)
+    packed, cu = ref.gather_paged(cache, np.array([[2, 0, 1]], np.int32), np.array([20], np.int32), bs)
+    expected = [(2, r) for r in range(16)] + [(0, r) for r in range(4)]
+    assert cu.tolist() == [0, 20]
+    assert packed[:, 0].tolist() == [list(map(float, e)) for e in expected]
+
+
+def _scatter_to_cache(x, cu, table, bs, nb):
+    """Write packed rows into a block cache, one key at a time, through the table."""
+    cache = np.zeros((nb, bs) + x.shape[1:])
+    for b in range(len(cu) - 1):
+        for t in range(int(cu[b + 1] - cu[b])):
+            cache[table[b][t // bs], t % bs] = x[cu[b] + t]
+    return cache
+
+
+@pytest.mark.parametrize("bs", [16, 48, 64])
+def test_p13_paged_decode_equals_packed_decode(bs):
+    """A cache filled through a random block table (physical blocks shuffled, tail blocks
+    partly used, a zero-length sequence) decodes exactly like the packed keys."""
+    rng = np.random.default_rng(130 + bs)
+    lens = [37, 0, 130, 16, 95]
+    p = W.random_problem(131 + bs, [1] * len(lens), lens, 4, 2, 16, 8, True, sink="normal")
+    per = [-(-n // bs) for n in lens]
+    max_blocks = max(per) + 1
+    nb = sum(per) + 3
+    perm = rng.permutation(nb)
+    table = np.full((len(lens), max_blocks), nb - 1, np.int32)   # unused entries: any valid id
+    i = 0
+    for b, n in enumerate(per):
+        table[b, :n] = perm[i:i + n]
+        i += n
+    kc = _scatter_to_cache(p.k, p.cu_seqlens_k, table, bs, nb)
+    vc = _scatter_to_cache(p.v, p.cu_seqlens_k, table, bs, nb)
+    used = np.array(lens, np.int32)
+    o1, l1 = ref.decode_paged(p.q, kc, vc, table, used, bs, p.sink, p.softmax_scale, True)
+    o2, l2 = ref.decode(p.q, p.k, p.v, p.cu_seqlens_k, p.sink, p.softmax_scale, True)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_p13_shared_prefix_block():
+    """Two sequences whose tables name the same first block see the same first keys:
+    with identical queries and one shared full block, their outputs agree."""
+    bs = 16
+    rng = np.random.default_rng(7)
+    kc = W.bf16_round(rng.standard_normal((3, bs, 1, 8), dtype=np.float32))
+    vc = W.bf16_round(rng.standard_normal((3, bs, 1, 8), dtype=np.float32))
+    q = np.repeat(W.bf16_round(rng.standard_normal((1, 2, 8), dtype=np.float32)), 2, axis=0)
+    table = np.array([[1, 2], [1, 0]], np.int32)
+    o, l = ref.decode_paged(q, kc, vc, table, np.array([16, 16], np.int32), bs, None, 0.3, True)
+    assert np.array_equal(o[0], o[1]) and np.array_equal(l[:, 0], l[:, 1])
+    # and the result is attention over block 1 alone
+    o_ref, _ = ref.decode(q[:1], kc[1], vc[1], np.array([0, 16]), None, 0.3, True)
+    assert np.allclose(o[0], o_ref[0], rtol=0, atol=1e-15)

@@ -257,6 +257,50 @@ def decode_kv_on_device(total_k: int, hkv: int, dk: int, dv: int, seed: int = 4,
     return out[0], out[1]
 
 
+def paged_layout(seed: int, lens_k: Sequence[int], block_size: int, spare_blocks: int = 3,
+                 spare_columns: int = 1):
+    """A block table for sequences of lens_k keys: each sequence gets ceil(len / block_size)
+    physical blocks, drawn as a seeded random permutation of all num_blocks ids (so no
+    sequence's blocks are adjacent or in order); `spare_blocks` ids stay unused and every
+    row has `spare_columns` extra entries (set to a valid, unused id).
+    Returns (block_table int32 [B, max_blocks], num_blocks)."""
+    rng = np.random.default_rng(seed)
+    per = [-(-int(n) // block_size) for n in lens_k]
+    num_blocks = sum(per) + spare_blocks
+    perm = rng.permutation(num_blocks).astype(np.int32)
+    table = np.full((len(per), max(per + [0]) + spare_columns), perm[-1], dtype=np.int32)
+    i = 0
+    for b, n in enumerate(per):
+        table[b, :n] = perm[i:i + n]
+        i += n
+    return table, num_blocks
+
+
+def paged_rows(cu_seqlens_k, block_table, block_size: int):
+    """For every packed key row (sequence b, key t): its (block, row-in-block) in the cache."""
+    cu = np.asarray(cu_seqlens_k, dtype=np.int64)
+    blk, off = [], []
+    for b in range(len(cu) - 1):
+        t = np.arange(int(cu[b + 1] - cu[b]))
+        blk.append(np.asarray(block_table)[b, t // block_size])
+        off.append(t % block_size)
+    return np.concatenate(blk).astype(np.int64), np.concatenate(off).astype(np.int64)
+
+
+def to_paged(x, cu_seqlens_k, block_table, block_size: int, num_blocks: int):
+    """Packed rows x [total, H, d] (numpy or torch) laid out as a block cache
+    [num_blocks, block_size, H, d]; unused cache rows are zero."""
+    blk, off = paged_rows(cu_seqlens_k, block_table, block_size)
+    if isinstance(x, np.ndarray):
+        cache = np.zeros((num_blocks, block_size) + x.shape[1:], dtype=x.dtype)
+        cache[blk, off] = x
+        return cache
+    import torch
+    cache = torch.zeros((num_blocks, block_size) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
+    cache[torch.from_numpy(blk).to(x.device), torch.from_numpy(off).to(x.device)] = x
+    return cache
+
+
 def random_decode(seed: int, lens_k: Sequence[int], hq: int, hkv: int, dk: int, dv: int,
                   causal: bool = True, window_left: int = -1, window_right: int = -1,
                   sink="normal", dtype: str = "bf16") -> DecodeProblem:
