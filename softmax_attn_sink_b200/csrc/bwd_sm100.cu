@@ -34,6 +34,37 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s);
 
 namespace {
 
+// Work order of the key-tile CTAs (1-D grid).  The (sequence, kv head) groups are taken in
+// bands of a.band_groups; inside a band the CTAs go key tile by key tile (tile 0, which sees
+// the most queries under a causal mask, first), cycling through the band's groups.  So the
+// CTAs resident at any time reduce into the dq_acc rows and read the Q / dO tiles of a few
+// groups only, a working set the launcher sizes to stay in L2: fp32 reductions into
+// L2-resident lines run about 1.7x faster than into lines that spill to DRAM.
+__device__ __forceinline__ void bwd_tile_of(const BwdArgs& a, int ntiles, int& g, int& b, int& nt) {
+  const long long id = blockIdx.x;
+  const int G = a.batch * a.hkv, S = a.band_groups;
+  const long long per_band = (long long)S * ntiles;
+  const int band = (int)(id / per_band);
+  const int first = band * S, members = (G - first < S) ? G - first : S;
+  const long long rem = id - (long long)band * per_band;
+  nt = (int)(rem / members);
+  const int grp = first + (int)(rem - (long long)nt * members);
+  b = grp / a.hkv;
+  g = grp - b * a.hkv;
+}
+
+// Groups per band: as many (sequence, kv head) groups as fit, with their dq_acc rows and
+// Q / dO tiles, in about half of the 126 MB L2.
+inline int bwd_band_groups(const BwdArgs& a) {
+  const long long per_group = (long long)(a.max_sq > 0 ? a.max_sq : 1) * (a.hq / a.hkv) *
+                              ((long long)a.dk * 4 + (long long)(a.dk + a.dv) * 2);
+  long long s = (64LL << 20) / (per_group > 0 ? per_group : 1);
+  const long long G = (long long)a.batch * a.hkv;
+  if (s < 1) s = 1;
+  if (s > G) s = G;
+  return (int)s;
+}
+
 using namespace sm100;
 
 constexpr int kBN = 128;  // keys per CTA
@@ -81,8 +112,9 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
   using L = BLayout<DK, DV>;
   extern __shared__ unsigned char smem_raw[];
 
-  // ---- work unit: key tile nt of (sequence b, kv head g); tile 0 (most queries) first --
-  const int g = blockIdx.x, b = blockIdx.y, nt = blockIdx.z;
+  // ---- work unit: key tile nt of (sequence b, kv head g) ---------------------------------
+  int g, b, nt;
+  bwd_tile_of(a, (a.max_sk + kBN - 1) / kBN, g, b, nt);
   const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
   const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
   const long long n0 = (long long)nt * kBN;
@@ -411,7 +443,8 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
   constexpr int DK = 128;
   extern __shared__ unsigned char smem_raw[];
 
-  const int g = blockIdx.x, b = blockIdx.y, nt = blockIdx.z;
+  int g, b, nt;
+  bwd_tile_of(a, (a.max_sk + kBN - 1) / kBN, g, b, nt);
   const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
   const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
   const long long n0 = (long long)nt * kBN;
@@ -821,8 +854,10 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   if ((e = cudaFuncSetAttribute(bwd_sm100_d128_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 L::kSmem)) != cudaSuccess)
     return e;
-  dim3 grid(a.hkv, a.batch, (a.max_sk + kBN - 1) / kBN);
-  bwd_sm100_d128_kernel<DV><<<grid, kThreadsP, L::kSmem, s>>>(a, tq, tk, tv, to);
+  BwdArgs ab = a;
+  ab.band_groups = bwd_band_groups(a);
+  const long long ctas = (long long)a.hkv * a.batch * ((a.max_sk + kBN - 1) / kBN);
+  bwd_sm100_d128_kernel<DV><<<(unsigned)ctas, kThreadsP, L::kSmem, s>>>(ab, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long n8 = (long long)a.total_q * a.hq * 128 / 8;
   dq_convert_hmajor_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
@@ -843,8 +878,10 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   if ((e = cudaFuncSetAttribute(bwd_sm100_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) !=
       cudaSuccess)
     return e;
-  dim3 grid(a.hkv, a.batch, (a.max_sk + kBN - 1) / kBN);
-  bwd_sm100_kernel<DK, DV><<<grid, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
+  BwdArgs ab = a;
+  ab.band_groups = bwd_band_groups(a);
+  const long long ctas = (long long)a.hkv * a.batch * ((a.max_sk + kBN - 1) / kBN);
+  bwd_sm100_kernel<DK, DV><<<(unsigned)ctas, kThreads, L::kSmem, s>>>(ab, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long n8 = (long long)a.total_q * a.hq * DK / 8;
   dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q),
@@ -857,7 +894,7 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
 bool bwd_sm100_supported(const BwdArgs& a, int dtype) {
   if (dtype != 0 || a.dq_acc == nullptr) return false;
   if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
-  if (a.batch > 65535 || (a.max_sk + kBN - 1) / kBN > 65535 || a.hkv > 65535) return false;
+  if ((long long)a.batch * a.hkv * ((a.max_sk + kBN - 1) / kBN) > 0x7fffffffLL) return false;  // 1-D grid
   return encode_fn() != nullptr;
 }
 

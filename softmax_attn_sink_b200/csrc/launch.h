@@ -51,6 +51,7 @@ struct BwdArgs {
   float scale;
   int left, right;
   unsigned* status;
+  int band_groups;       // tensor-core path: (sequence, kv head) groups whose key tiles run together
 };
 
 struct DecodeArgs {
