@@ -327,6 +327,34 @@ def bench_fwd(args, world, peaks, peak_kind, sampler):
             "pairs": pairs, "flops": flops, "p": p}
 
 
+def bench_fwd_fp16(args, world, peaks, peak_kind):
+    """The headline forward with fp16 inputs (the same draws rounded to fp16)."""
+    import torch
+    import softmax_attn_sink_b200 as sab
+    p = W.config2("fp16")
+    td = torch.float16
+    q, k, v = (torch.from_numpy(x).to(td).cuda() for x in (p.q, p.k, p.v))
+    cu = torch.from_numpy(p.cu_seqlens_q).cuda()
+    sink = torch.from_numpy(p.sink).cuda()
+    pairs = visible_pairs(p.cu_seqlens_q, p.cu_seqlens_k, p.num_heads_q, True)
+    flops = 2 * (128 + 128) * pairs
+    out = torch.empty((p.q.shape[0], 32, 128), dtype=td, device="cuda")
+    lse = torch.empty((32, p.q.shape[0]), dtype=torch.float32, device="cuda")
+    flush = Flusher()
+    steps = max(3, min(args.steps, 50))
+    per, total = time_steps(lambda: sab.attn_sink_fwd(q, k, v, cu, cu, p.max_seqlen_q, p.max_seqlen_k, sink,
+                                                      p.softmax_scale, True, out=out, lse=lse),
+                            steps, args.warmup, world, flush)
+    achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
+    pk = peaks["bf16_tflops"]   # dense fp16 and bf16 tensor rates are equal (nominal ratio 1)
+    return {"workload": p.name, "unit": "TFLOP/s", "steps": steps,
+            "value": round(weak_scaling_value(flops, world, total, steps) / 1e12, 2),
+            "ms_per_step": round(total / steps, 4), "flops": flops,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk, "unit": "TFLOP/s",
+                         "frac": round(achieved / pk, 4), "traffic": None,
+                         "peak_source": f"bf16_tflops x 1 (nominal fp16 / bf16 dense ratio; {peak_kind}, burst)"}}
+
+
 def bench_fwd_bwd(args, world, peaks, peak_kind):
     import torch
     import softmax_attn_sink_b200 as sab
@@ -511,7 +539,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all", "fwd", "fwd_bwd", "decode"], default="all")
+    ap.add_argument("--workload", choices=["all", "fwd", "fwd_fp16", "fwd_bwd", "decode"], default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", type=int, default=4, choices=[1, 2, 3, 4],
                     help="sequences of the fwd_bwd leg (4 = the full training workload)")
@@ -547,6 +575,8 @@ def main():
             })
             if sampler is not None:
                 line["clocks"] = sampler.summary()
+        if args.workload in ("all", "fwd_fp16"):
+            extra["fwd_fp16"] = bench_fwd_fp16(args, world, peaks, peak_kind)
         if args.workload in ("all", "fwd_bwd"):
             extra["fwd_bwd"] = bench_fwd_bwd(args, world, peaks, peak_kind)
         if args.workload in ("all", "decode"):
@@ -557,7 +587,7 @@ def main():
             key = args.workload
             e = extra[key]
             v = e["fwd"]["value"] if key == "fwd_bwd" else e["value"]
-            line.update({"value": v, "unit": "TFLOP/s" if key == "fwd_bwd" else "GB/s",
+            line.update({"value": v, "unit": e.get("unit", "TFLOP/s"),
                          "ms_per_step": e["fwd"]["ms_per_step"] if key == "fwd_bwd" else e["ms_per_step"],
                          "config": {"workload": e["workload"]}})
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -36,8 +36,10 @@
  *     A row that sees no key outputs 0 (issue #108108) and has lse = -inf.
  *   - lse is the vanilla log-sum-exp of the visible scaled scores, natural log,
  *     WITHOUT the sink (CANN doc, softmax_lse formula).
- *   - dtype: ATTN_SINK_BF16 (bf16 q/k/v/out/dout/dq/dk/dv, fp32 accumulation, outputs
- *     rounded once to nearest-even) or ATTN_SINK_FP32 (fp32 everywhere, no tensor cores).
+ *   - dtype: ATTN_SINK_BF16 or ATTN_SINK_FP16 (16-bit q/k/v/out/dout/dq/dk/dv, fp32
+ *     accumulation, P and dS rounded to the same 16-bit type for the tensor cores, outputs
+ *     rounded once to nearest-even; the CANN doc lists both BFLOAT16 and FLOAT16 for
+ *     q / k / v) or ATTN_SINK_FP32 (fp32 everywhere, no tensor cores).
  *   - Supported head dims: head_dim_qk in {64, 128}; head_dim_v in {32, 64, 128}.
  *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace).  The
  *     library never allocates, frees or synchronises; every pointer except `params`
@@ -62,7 +64,7 @@
 extern "C" {
 #endif
 
-typedef enum { ATTN_SINK_BF16 = 0, ATTN_SINK_FP32 = 1 } attn_sink_dtype;
+typedef enum { ATTN_SINK_BF16 = 0, ATTN_SINK_FP32 = 1, ATTN_SINK_FP16 = 2 } attn_sink_dtype;
 
 typedef enum {
   ATTN_SINK_OK = 0,
@@ -156,8 +158,8 @@ int attn_sink_decode(const attn_sink_params* params, const void* q, const void* 
  * The query of sequence b sits at key position seqused_k[b] - 1 (bottom-right), so causal
  * decode sees all of its keys and a window keeps the last window_left + 1 of them.
  * Writes out [batch, Hq, dv] and, when not NULL, lse [Hq, batch]; the workspace is the one
- * attn_sink_decode_workspace_size() gives for the same params and num_splits.  bf16 only
- * (ATTN_SINK_ERR_UNSUPPORTED otherwise).  Table contents are the caller's contract: a
+ * attn_sink_decode_workspace_size() gives for the same params and num_splits.  bf16 or fp16
+ * (ATTN_SINK_ERR_UNSUPPORTED for fp32).  Table contents are the caller's contract: a
  * block id outside [0, num_blocks) or a seqused_k beyond its table row is not read (those
  * keys count as zero vectors) and sets the device status that
  * attn_sink_get_device_status() reports as ATTN_SINK_ERR_BAD_INDEX.

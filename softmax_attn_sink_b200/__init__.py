@@ -22,14 +22,15 @@ from typing import Optional, Sequence, Tuple
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn_sink.so")
 
-ATTN_SINK_BF16, ATTN_SINK_FP32 = 0, 1
+ATTN_SINK_BF16, ATTN_SINK_FP32, ATTN_SINK_FP16 = 0, 1, 2
 STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE", 4: "ERR_CUDA",
-          5: "ERR_TIMEOUT"}
+          5: "ERR_TIMEOUT", 6: "ERR_BAD_INDEX"}
 
 _SYMBOLS = ("attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "attn_sink_fwd_workspace_size",
             "attn_sink_bwd_workspace_size", "attn_sink_decode_workspace_size",
             "attn_sink_decode_num_splits", "attn_sink_status_string",
-            "attn_sink_get_device_status", "attn_sink_selftest_wait_timeout", "attn_sink_version")
+            "attn_sink_get_device_status", "attn_sink_selftest_wait_timeout", "attn_sink_version",
+            "attn_sink_decode_paged", "attn_sink_decode_noalloc")
 
 
 class AttnSinkParams(ctypes.Structure):
@@ -125,7 +126,9 @@ def _dtype_code(t) -> int:
         return ATTN_SINK_BF16
     if t.dtype == torch.float32:
         return ATTN_SINK_FP32
-    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+    if t.dtype == torch.float16:
+        return ATTN_SINK_FP16
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16, float16 or float32")
 
 
 def _require(t, name, dtype=None, ndim=None):
@@ -354,4 +357,4 @@ class SinkAttention:
 
 __all__ = ["attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "attn_sink_decode_paged", "decode_num_splits",
            "device_status", "selftest_wait_timeout", "SinkAttention", "AttnSinkError", "AttnSinkParams", "make_params",
-           "lib", "LIB_PATH", "ATTN_SINK_BF16", "ATTN_SINK_FP32"]
+           "lib", "LIB_PATH", "ATTN_SINK_BF16", "ATTN_SINK_FP32", "ATTN_SINK_FP16"]

@@ -40,7 +40,8 @@ bool dims_supported(int dk, int dv) {
 
 int validate_params(const attn_sink_params* p, bool decode) {
   if (!p) return ATTN_SINK_ERR_INVALID_ARG;
-  if (p->dtype != ATTN_SINK_BF16 && p->dtype != ATTN_SINK_FP32) return ATTN_SINK_ERR_UNSUPPORTED;
+  if (p->dtype != ATTN_SINK_BF16 && p->dtype != ATTN_SINK_FP32 && p->dtype != ATTN_SINK_FP16)
+    return ATTN_SINK_ERR_UNSUPPORTED;
   if (p->batch <= 0 || p->total_q <= 0 || p->total_k <= 0) return ATTN_SINK_ERR_INVALID_ARG;
   if (p->num_heads_q <= 0 || p->num_heads_kv <= 0) return ATTN_SINK_ERR_INVALID_ARG;
   if (p->num_heads_q % p->num_heads_kv != 0) return ATTN_SINK_ERR_INVALID_ARG;
@@ -72,7 +73,7 @@ BwdLayout bwd_layout(const attn_sink_params* p) {
   l.lse_tot = align_up(l.D + rows * 4, 256);
   l.dq_acc = align_up(l.lse_tot + rows * 4, 256);
   size_t end = l.dq_acc;
-  if (p->dtype == ATTN_SINK_BF16) end += (size_t)p->total_q * p->num_heads_q * p->head_dim_qk * 4;
+  if (p->dtype != ATTN_SINK_FP32) end += (size_t)p->total_q * p->num_heads_q * p->head_dim_qk * 4;
   l.total = align_up(end, 256);
   return l;
 }
@@ -98,7 +99,7 @@ int decode_auto_splits(const attn_sink_params* p) {
 }
 
 size_t decode_ws(const attn_sink_params* p, int splits) {
-  if (p->dtype != ATTN_SINK_BF16) return 0;
+  if (p->dtype == ATTN_SINK_FP32) return 0;
   const size_t rows = (size_t)p->batch * p->num_heads_q * splits;
   return align_up(rows * p->head_dim_v * 4, 256) + align_up(rows * 2 * 4, 256);
 }
@@ -118,7 +119,7 @@ int launch_decode(const attn_sink_params* p, DecodeArgs& a, int num_splits, void
   a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
   a.splits = splits; a.scale = p->softmax_scale; a.left = left; a.right = right;
   a.status = status_ptr();
-  return from_cuda(launch_decode_split(a, s));
+  return from_cuda(launch_decode_split(a, p->dtype, s));
 }
 
 }  // namespace
@@ -182,8 +183,8 @@ int attn_sink_fwd(const attn_sink_params* p, const void* q, const void* k, const
   effective_window(p, a.left, a.right);
   a.status = status_ptr();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int dt = p->dtype == ATTN_SINK_FP32 ? 1 : 0;
-  if (dt == 0 && fwd_sm100_supported(a, dt)) return from_cuda(launch_fwd_sm100(a, s));
+  const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
+  if (fwd_sm100_supported(a, dt)) return from_cuda(launch_fwd_sm100(a, dt, s));
   return from_cuda(launch_fwd_simt(a, dt, s));
 }
 
@@ -208,7 +209,7 @@ int attn_sink_bwd(const attn_sink_params* p, const void* q, const void* k, const
   a.grad_q = dq; a.grad_k = dk; a.grad_v = dv; a.dsink = dsink;
   a.D = reinterpret_cast<float*>(ws + lay.D);
   a.lse_tot = reinterpret_cast<float*>(ws + lay.lse_tot);
-  a.dq_acc = p->dtype == ATTN_SINK_BF16 ? reinterpret_cast<float*>(ws + lay.dq_acc) : nullptr;
+  a.dq_acc = p->dtype != ATTN_SINK_FP32 ? reinterpret_cast<float*>(ws + lay.dq_acc) : nullptr;
   a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
   a.max_sq = p->max_seqlen_q; a.max_sk = p->max_seqlen_k;
   a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
@@ -216,8 +217,8 @@ int attn_sink_bwd(const attn_sink_params* p, const void* q, const void* k, const
   effective_window(p, a.left, a.right);
   a.status = status_ptr();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int dt = p->dtype == ATTN_SINK_FP32 ? 1 : 0;
-  if (dt == 0 && bwd_sm100_supported(a, dt)) return from_cuda(launch_bwd_sm100(a, s));
+  const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
+  if (bwd_sm100_supported(a, dt)) return from_cuda(launch_bwd_sm100(a, dt, s));
   return from_cuda(launch_bwd_simt(a, dt, s));
 }
 
@@ -258,7 +259,7 @@ int attn_sink_decode_paged(const attn_sink_params* p, const void* q, const void*
                            size_t workspace_bytes, attn_sink_stream_t stream) {
   int st = validate_params(p, true);
   if (st != ATTN_SINK_OK) return st;
-  if (p->dtype != ATTN_SINK_BF16) return ATTN_SINK_ERR_UNSUPPORTED;
+  if (p->dtype == ATTN_SINK_FP32) return ATTN_SINK_ERR_UNSUPPORTED;
   if (num_splits < 0) return ATTN_SINK_ERR_INVALID_ARG;
   if (!q || !k_cache || !v_cache || !block_table || !seqused_k || !out) return ATTN_SINK_ERR_INVALID_ARG;
   if (block_size < 16 || block_size > 1024 || block_size % 16 != 0) return ATTN_SINK_ERR_INVALID_ARG;

@@ -302,6 +302,8 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s) {
   dim3 grid((a.total_q + 63) / 64, a.hq);
   if (dtype == 1)
     bwd_preprocess_kernel<float><<<grid, 256, 0, s>>>(a);
+  else if (dtype == 2)
+    bwd_preprocess_kernel<__half><<<grid, 256, 0, s>>>(a);
   else
     bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();
@@ -310,7 +312,8 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s) {
 cudaError_t launch_bwd_simt(const BwdArgs& a, int dtype, cudaStream_t s) {
   cudaError_t e = launch_bwd_preprocess(a, dtype, s);
   if (e != cudaSuccess) return e;
-  return dtype == 1 ? dispatch_dims<float>(a, s) : dispatch_dims<__nv_bfloat16>(a, s);
+  if (dtype == 1) return dispatch_dims<float>(a, s);
+  return dtype == 2 ? dispatch_dims<__half>(a, s) : dispatch_dims<__nv_bfloat16>(a, s);
 }
 
 }  // namespace attn_sink

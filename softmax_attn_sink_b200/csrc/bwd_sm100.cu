@@ -105,7 +105,7 @@ struct BBars {
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * 11; }
 };
 
-template <int DK, int DV>
+template <typename Elem, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do) {
@@ -195,10 +195,10 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
     if (lane == 0 && T > 0) {
-      constexpr uint32_t id_s = idesc_bf16(kBN, kBM, 0, 0);   // S^T, dP^T: K-major A and B
-      constexpr uint32_t id_dv = idesc_bf16(kBN, DV, 0, 1);   // A from TMEM, B = dout MN-major
-      constexpr uint32_t id_dk = idesc_bf16(kBN, DK, 0, 1);   // A = dS^T K-major, B = Q MN-major
-      constexpr uint32_t id_dq = idesc_bf16(kBM, DK, 1, 1);   // A = dS MN-major, B = K MN-major
+      constexpr uint32_t id_s = idesc_of<Elem>(kBN, kBM, 0, 0);   // S^T, dP^T: K-major A and B
+      constexpr uint32_t id_dv = idesc_of<Elem>(kBN, DV, 0, 1);   // A from TMEM, B = dout MN-major
+      constexpr uint32_t id_dk = idesc_of<Elem>(kBN, DK, 0, 1);   // A = dS^T K-major, B = Q MN-major
+      constexpr uint32_t id_dq = idesc_of<Elem>(kBM, DK, 1, 1);   // A = dS MN-major, B = K MN-major
       bool ok = mbar_wait(bar.kv_full(), 0, a.status);
       for (int t = 0; t < T && ok; ++t) {
         const int st = t & 1;
@@ -291,8 +291,8 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
             pp[u] = p;
             dd[u] = ds;
           }
-          pk[e >> 1] = pack_bf16x2(pp[0], pp[1]);
-          dk_[e >> 1] = pack_bf16x2(dd[0], dd[1]);
+          pk[e >> 1] = pack2<Elem>(pp[0], pp[1]);
+          dk_[e >> 1] = pack2<Elem>(dd[0], dd[1]);
         }
         // P^T chunk -> TMEM R0 (its S^T columns were already read)
         tmem_st16(tmem + lane_off + kColR0 + c * 16, pk);
@@ -313,8 +313,8 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
     // ---- epilogue: dK = scale * acc, dV = acc, bf16, this thread's key row -----------------
     const bool have = __all_sync(0xffffffffu, ok && T > 0 && mbar_wait(bar.ds_free(), (T - 1) & 1, a.status));
     tc_fence_after();
-    __nv_bfloat16* dkp = static_cast<__nv_bfloat16*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
-    __nv_bfloat16* dvp = static_cast<__nv_bfloat16*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
+    Elem* dkp = static_cast<Elem*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
+    Elem* dvp = static_cast<Elem*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       const int ncol = pass == 0 ? DK : DV;
@@ -332,7 +332,7 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
         for (int e = 0; e < 16; ++e) {
           const float x0 = (T > 0 && have) ? __uint_as_float(v[2 * e]) * mul : 0.f;
           const float x1 = (T > 0 && have) ? __uint_as_float(v[2 * e + 1]) * mul : 0.f;
-          pk[e] = pack_bf16x2(x0, x1);
+          pk[e] = pack2<Elem>(x0, x1);
         }
         if (key_ok) {
 #pragma unroll
@@ -434,7 +434,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <int DV>
+template <typename Elem, int DV>
 __global__ void __launch_bounds__(kThreadsP, 1)
 bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -528,10 +528,10 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     // ================================ MMA issuer =========================================
     regs_dec<kRegsLow>();
     if (lane == 0 && T > 0) {
-      constexpr uint32_t id_s = idesc_bf16(kBN, 64, 0, 0);    // S_h, dP_h: 128 keys x 64 queries
-      constexpr uint32_t id_dv = idesc_bf16(kBN, DV, 0, 1);   // P^T_h (TMEM) x dout_h (MN-major)
-      constexpr uint32_t id_dk = idesc_bf16(kBN, DK, 0, 1);   // dS^T_h (K-major) x Q_h (MN-major)
-      constexpr uint32_t id_dq = idesc_bf16(DK, 64, 1, 1);    // K^T (MN-major) x dS^T_h (MN-major)
+      constexpr uint32_t id_s = idesc_of<Elem>(kBN, 64, 0, 0);    // S_h, dP_h: 128 keys x 64 queries
+      constexpr uint32_t id_dv = idesc_of<Elem>(kBN, DV, 0, 1);   // P^T_h (TMEM) x dout_h (MN-major)
+      constexpr uint32_t id_dk = idesc_of<Elem>(kBN, DK, 0, 1);   // dS^T_h (K-major) x Q_h (MN-major)
+      constexpr uint32_t id_dq = idesc_of<Elem>(DK, 64, 1, 1);    // K^T (MN-major) x dS^T_h (MN-major)
       // S_h(t) = K Q_h^T -> S columns; dP_h(t) = V dout_h^T -> dP columns
       // Shared-memory descriptors, built once: an address offset is an addition to the start
       // field (addresses stay below 2^18 bytes, so the 14-bit field never carries).  "k" =
@@ -689,8 +689,8 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
           uint32_t pk[16], dk_[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
-            dk_[e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
+            pk[e] = pack2<Elem>(p[2 * e], p[2 * e + 1]);
+            dk_[e] = pack2<Elem>(ds[2 * e], ds[2 * e + 1]);
           }
           tmem_st16(tmem + lane_off + cS + c * 16, pk);
           const uint32_t rowp = sDS + hh * L::kHalf + r * 128;
@@ -710,8 +710,8 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     // ---- epilogue: dK = scale * acc, dV = acc -------------------------------------------
     const bool have = __all_sync(0xffffffffu, ok && T > 0 && mbar_wait(bar.ds_free(1), (T - 1) & 1, a.status));
     tc_fence_after();
-    __nv_bfloat16* dkp = static_cast<__nv_bfloat16*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
-    __nv_bfloat16* dvp = static_cast<__nv_bfloat16*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
+    Elem* dkp = static_cast<Elem*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
+    Elem* dvp = static_cast<Elem*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       const int ncol = pass == 0 ? DK : DV;
@@ -729,7 +729,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         for (int e = 0; e < 16; ++e) {
           const float x0 = (T > 0 && have) ? __uint_as_float(v[2 * e]) * mul : 0.f;
           const float x1 = (T > 0 && have) ? __uint_as_float(v[2 * e + 1]) * mul : 0.f;
-          pk[e] = pack_bf16x2(x0, x1);
+          pk[e] = pack2<Elem>(x0, x1);
         }
         if (key_ok) {
 #pragma unroll
@@ -780,21 +780,23 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 }
 
 // dq = bf16(dq_acc), 8 elements per thread
-__global__ void dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8) {
+template <typename T>
+__global__ void dq_convert_kernel(const float* __restrict__ acc, T* __restrict__ dq, long long n8) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const float4 x = reinterpret_cast<const float4*>(acc)[2 * i];
   const float4 y = reinterpret_cast<const float4*>(acc)[2 * i + 1];
   uint4 o;
-  o.x = pack_bf16x2(x.x, x.y);
-  o.y = pack_bf16x2(x.z, x.w);
-  o.z = pack_bf16x2(y.x, y.y);
-  o.w = pack_bf16x2(y.z, y.w);
+  o.x = pack2<T>(x.x, x.y);
+  o.y = pack2<T>(x.z, x.w);
+  o.z = pack2<T>(y.x, y.y);
+  o.w = pack2<T>(y.z, y.w);
   reinterpret_cast<uint4*>(dq)[i] = o;
 }
 
 // dq[t][h][:] = bf16(dq_acc[h][t][:]) for the head-major accumulator, 8 elements per thread.
-__global__ void dq_convert_hmajor_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int total_q,
+template <typename T>
+__global__ void dq_convert_hmajor_kernel(const float* __restrict__ acc, T* __restrict__ dq, int total_q,
                                          int hq, long long n8) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
@@ -805,10 +807,10 @@ __global__ void dq_convert_hmajor_kernel(const float* __restrict__ acc, __nv_bfl
   const float4 x = reinterpret_cast<const float4*>(src)[0];
   const float4 y = reinterpret_cast<const float4*>(src)[1];
   uint4 o;
-  o.x = pack_bf16x2(x.x, x.y);
-  o.y = pack_bf16x2(x.z, x.w);
-  o.z = pack_bf16x2(y.x, y.y);
-  o.w = pack_bf16x2(y.z, y.w);
+  o.x = pack2<T>(x.x, x.y);
+  o.y = pack2<T>(x.z, x.w);
+  o.z = pack2<T>(y.x, y.y);
+  o.w = pack2<T>(y.z, y.w);
   reinterpret_cast<uint4*>(dq)[i] = o;
 }
 
@@ -828,82 +830,96 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, heads, d] bf16 as a 3-D tensor; boxes of 128 rows x 1 head x 64 columns, 128B swizzle.
-bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows) {
+// [rows, heads, d] of 16-bit elements as a 3-D tensor; boxes of 128 rows x 1 head x 64
+// columns, 128B swizzle.
+bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows, CUtensorMapDataType dt) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * heads};
   const cuuint32_t box[3] = {64, 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DV>
+template <typename T> constexpr CUtensorMapDataType tma_dtype();
+template <> constexpr CUtensorMapDataType tma_dtype<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
+template <> constexpr CUtensorMapDataType tma_dtype<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
+template <typename T> constexpr int dtype_code();
+template <> constexpr int dtype_code<__nv_bfloat16>() { return 0; }
+template <> constexpr int dtype_code<__half>() { return 2; }
+
+template <typename T, int DV>
 cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   using L = PLayout<DV>;
+  constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, a.q, 128, a.hq, a.total_q) || !make_map(&tk, a.k, 128, a.hkv, a.total_k) ||
-      !make_map(&tv, a.v, DV, a.hkv, a.total_k) || !make_map(&to, a.dout, DV, a.hq, a.total_q))
+  if (!make_map(&tq, a.q, 128, a.hq, a.total_q, dt) || !make_map(&tk, a.k, 128, a.hkv, a.total_k, dt) ||
+      !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * 128 * sizeof(float), s);
   if (e != cudaSuccess) return e;
-  if ((e = launch_bwd_preprocess(a, 0, s)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(bwd_sm100_d128_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(bwd_sm100_d128_kernel<T, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 L::kSmem)) != cudaSuccess)
     return e;
   BwdArgs ab = a;
   ab.band_groups = bwd_band_groups(a);
   const long long ctas = (long long)a.hkv * a.batch * ((a.max_sk + kBN - 1) / kBN);
-  bwd_sm100_d128_kernel<DV><<<(unsigned)ctas, kThreadsP, L::kSmem, s>>>(ab, tq, tk, tv, to);
+  bwd_sm100_d128_kernel<T, DV><<<(unsigned)ctas, kThreadsP, L::kSmem, s>>>(ab, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long n8 = (long long)a.total_q * a.hq * 128 / 8;
-  dq_convert_hmajor_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
-      a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q), a.total_q, a.hq, n8);
+  dq_convert_hmajor_kernel<T><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
+      a.dq_acc, static_cast<T*>(a.grad_q), a.total_q, a.hq, n8);
   return cudaGetLastError();
 }
 
-template <int DK, int DV>
+template <typename T, int DK, int DV>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   using L = BLayout<DK, DV>;
+  constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, a.q, DK, a.hq, a.total_q) || !make_map(&tk, a.k, DK, a.hkv, a.total_k) ||
-      !make_map(&tv, a.v, DV, a.hkv, a.total_k) || !make_map(&to, a.dout, DV, a.hq, a.total_q))
+  if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
+      !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * DK * sizeof(float), s);
   if (e != cudaSuccess) return e;
-  if ((e = launch_bwd_preprocess(a, 0, s)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(bwd_sm100_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) !=
-      cudaSuccess)
+  if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(bwd_sm100_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                L::kSmem)) != cudaSuccess)
     return e;
   BwdArgs ab = a;
   ab.band_groups = bwd_band_groups(a);
   const long long ctas = (long long)a.hkv * a.batch * ((a.max_sk + kBN - 1) / kBN);
-  bwd_sm100_kernel<DK, DV><<<(unsigned)ctas, kThreads, L::kSmem, s>>>(ab, tq, tk, tv, to);
+  bwd_sm100_kernel<T, DK, DV><<<(unsigned)ctas, kThreads, L::kSmem, s>>>(ab, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long n8 = (long long)a.total_q * a.hq * DK / 8;
-  dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.grad_q),
-                                                                 n8);
+  dq_convert_kernel<T><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<T*>(a.grad_q), n8);
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dims(const BwdArgs& a, cudaStream_t s) {
+  if (a.dk == 128 && a.dv == 128) return launch_d128<T, 128>(a, s);
+  if (a.dk == 128 && a.dv == 64) return launch_d128<T, 64>(a, s);
+  if (a.dk == 64 && a.dv == 64) return launch_typed<T, 64, 64>(a, s);
+  if (a.dk == 64 && a.dv == 128) return launch_typed<T, 64, 128>(a, s);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 bool bwd_sm100_supported(const BwdArgs& a, int dtype) {
-  if (dtype != 0 || a.dq_acc == nullptr) return false;
+  if ((dtype != 0 && dtype != 2) || a.dq_acc == nullptr) return false;
   if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
   if ((long long)a.batch * a.hkv * ((a.max_sk + kBN - 1) / kBN) > 0x7fffffffLL) return false;  // 1-D grid
   return encode_fn() != nullptr;
 }
 
-cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s) {
-  if (a.dk == 128 && a.dv == 128) return launch_d128<128>(a, s);
-  if (a.dk == 128 && a.dv == 64) return launch_d128<64>(a, s);
-  if (a.dk == 64 && a.dv == 64) return launch_typed<64, 64>(a, s);
-  if (a.dk == 64 && a.dv == 128) return launch_typed<64, 128>(a, s);
-  return cudaErrorInvalidValue;
+cudaError_t launch_bwd_sm100(const BwdArgs& a, int dtype, cudaStream_t s) {
+  return dtype == 2 ? launch_dims<__half>(a, s) : launch_dims<__nv_bfloat16>(a, s);
 }
 
 }  // namespace attn_sink

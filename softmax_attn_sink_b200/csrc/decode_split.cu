@@ -1,4 +1,4 @@
-// Split-KV decode for bf16: one query per sequence, GQA heads of a kv head together.  K/V
+// Split-KV decode for bf16 and fp16: one query per sequence, GQA heads of a kv head together.  K/V
 // are either packed ([total_k, hkv, d] with cu_seqlens_k) or paged ([num_blocks, block_size,
 // hkv, d] with a block table and per-sequence key counts; CANN flash_attn doc, "Paged
 // Attention Parameter Group" and the PA_BBND layout of k in its parameter table).
@@ -18,9 +18,11 @@
 // Each key is read from HBM once per 16 q heads; K/V go HBM -> shared memory through a
 // 3-stage cp.async pipeline (16-byte copies, XOR-swizzled rows so ldmatrix is
 // conflict-free).  The two contractions per 16 keys (S = Q K^T over the head dim and
-// O += P V over the keys) use m16n8k16 bf16 MMAs with fp32 accumulation; the query
+// O += P V over the keys) use m16n8k16 MMAs (bf16 or f16 inputs) with fp32 accumulation; the query
 // heads form the M dimension.  Scores are kept in the log2 domain (scale * log2 e folded
 // into one multiply) and exponentiated with ex2.approx.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace attn_sink {
@@ -61,18 +63,21 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, u
                : "r"(addr));
 }
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
+// D += A B for one m16n8k16 tile with fp32 accumulation; A and B both bf16 or both f16.
+template <typename T>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (std::is_same<T, __half>::value)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // physical 16-byte chunk of logical chunk c in a row of NCH chunks
@@ -107,7 +112,7 @@ __device__ __forceinline__ void decode_range(const DecodeArgs& a, int b, long lo
 // (the chunk's block ids staged once per CTA) or, when they do not fit, from global memory.
 enum KvMode { kPacked = 0, kPagedSmemTable = 1, kPagedGlobalTable = 2 };
 
-template <int DK, int DV, int MODE>
+template <typename T, int DK, int DV, int MODE>
 __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const DecodeArgs a, int chunk,
                                                                        int extra_off) {
   constexpr bool PAGED = MODE != kPacked;
@@ -132,9 +137,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h_base = g * group + hb * 16;
   const int nh = (group - hb * 16) < 16 ? (group - hb * 16) : 16;
-  const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* vp = static_cast<const __nv_bfloat16*>(a.v);
-  const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q);
+  const T* kp = static_cast<const T*>(a.k);
+  const T* vp = static_cast<const T*>(a.v);
+  const T* qp = static_cast<const T*>(a.q);
   // Paged K/V: the cache row of every key of a stage is computed once, by one thread per key,
   // into s_row (kStages stage slots of 64 rows, -1 = no key or a block id outside the cache)
   // one iteration before the stage's copies are issued; the copies then read it like the
@@ -182,13 +187,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
       for (int idx = tid; idx < kStageKeys * KCH; idx += kWarps * 32) {
         const int r = idx / KCH, ch = idx % KCH;
         const bool ok = t0 + r < c_hi;
-        const __nv_bfloat16* src = ok ? kp + ((k0 + t0 + r) * a.hkv + g) * DK + ch * 8 : kp;
+        const T* src = ok ? kp + ((k0 + t0 + r) * a.hkv + g) * DK + ch * 8 : kp;
         cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, src, ok);
       }
       for (int idx = tid; idx < kStageKeys * VCH; idx += kWarps * 32) {
         const int r = idx / VCH, ch = idx % VCH;
         const bool ok = t0 + r < c_hi;
-        const __nv_bfloat16* src = ok ? vp + ((k0 + t0 + r) * a.hkv + g) * DV + ch * 8 : vp;
+        const T* src = ok ? vp + ((k0 + t0 + r) * a.hkv + g) * DV + ch * 8 : vp;
         cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, src, ok);
       }
     } else {
@@ -197,14 +202,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
         const int r = idx / KCH, ch = idx % KCH;
         const long long row = rows[r];
         const bool ok = row >= 0;
-        const __nv_bfloat16* src = ok ? kp + (row * a.hkv + g) * DK + ch * 8 : kp;
+        const T* src = ok ? kp + (row * a.hkv + g) * DK + ch * 8 : kp;
         cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, src, ok);
       }
       for (int idx = tid; idx < kStageKeys * VCH; idx += kWarps * 32) {
         const int r = idx / VCH, ch = idx % VCH;
         const long long row = rows[r];
         const bool ok = row >= 0;
-        const __nv_bfloat16* src = ok ? vp + (row * a.hkv + g) * DV + ch * 8 : vp;
+        const T* src = ok ? vp + (row * a.hkv + g) * DV + ch * 8 : vp;
         cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, src, ok);
       }
     }
@@ -265,8 +270,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
       const int ch = ks * 2 + (mi & 1);
       uint32_t b0, b1, b2, b3;
       ldmatrix_x4(k_s + (row * KCH + swz<KCH>(row, ch)) * 16, b0, b1, b2, b3);
-      mma_bf16(s[0], qa[ks], b0, b1);
-      mma_bf16(s[1], qa[ks], b2, b3);
+      mma16816<T>(s[0], qa[ks], b0, b1);
+      mma16816<T>(s[1], qa[ks], b2, b3);
     }
     // mask keys past the chunk end, online softmax in the log2 domain
     const int kc = (lane & 3) * 2;
@@ -308,10 +313,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
       o_acc[nt][3] *= alpha[1];
     }
     uint32_t pa[4];
-    pa[0] = pack_bf16(p[0][0], p[0][1]);
-    pa[1] = pack_bf16(p[0][2], p[0][3]);
-    pa[2] = pack_bf16(p[1][0], p[1][1]);
-    pa[3] = pack_bf16(p[1][2], p[1][3]);
+    pa[0] = pack2<T>(p[0][0], p[0][1]);
+    pa[1] = pack2<T>(p[0][2], p[0][3]);
+    pa[2] = pack2<T>(p[1][0], p[1][1]);
+    pa[3] = pack2<T>(p[1][2], p[1][3]);
     // O += P V
 #pragma unroll
     for (int ntp = 0; ntp < VTILES / 2; ++ntp) {
@@ -320,8 +325,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
       const int ch = ntp * 2 + (mi >> 1);
       uint32_t b0, b1, b2, b3;
       ldmatrix_x4_trans(v_s + (row * VCH + swz<VCH>(row, ch)) * 16, b0, b1, b2, b3);
-      mma_bf16(o_acc[2 * ntp], pa, b0, b1);
-      mma_bf16(o_acc[2 * ntp + 1], pa, b2, b3);
+      mma16816<T>(o_acc[2 * ntp], pa, b0, b1);
+      mma16816<T>(o_acc[2 * ntp + 1], pa, b2, b3);
     }
   }
   cp_async_wait<0>();
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const Deco
 }
 
 // One warp per (sequence, q head): merge the chunks of that row, apply the sink once.
-template <int DV>
+template <typename T, int DV>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, int chunk) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * 4 + warp;   // b * hq + h
@@ -412,25 +417,25 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, i
   }
   const float den = lm + ((sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m));
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+  T* out = static_cast<T*>(a.out);
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) out[row * DV + lane + 32 * j] = __float2bfloat16_rn(o[j] * inv);
+  for (int j = 0; j < VPL; ++j) out[row * DV + lane + 32 * j] = from_float<T>(o[j] * inv);
   if (a.lse && lane == 0)
     a.lse[(long long)h * a.batch + b] = (M == kNegInf || lM <= 0.f) ? kNegInf : (M + __log2f(lM)) * kLn2;
 }
 
-template <int DK, int DV, int MODE>
+template <typename T, int DK, int DV, int MODE>
 cudaError_t launch_split(const DecodeArgs& a, int chunk, int smem, int extra_off, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<DK, DV, MODE>,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<T, DK, DV, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int group = a.hq / a.hkv;
   dim3 grid(a.splits, a.hkv * ((group + 15) / 16), a.batch);
-  decode_split_kernel<DK, DV, MODE><<<grid, kWarps * 32, smem, s>>>(a, chunk, extra_off);
+  decode_split_kernel<T, DK, DV, MODE><<<grid, kWarps * 32, smem, s>>>(a, chunk, extra_off);
   return cudaGetLastError();
 }
 
-template <int DK, int DV>
+template <typename T, int DK, int DV>
 cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
   const int group = a.hq / a.hkv;
   const int hblocks = (group + 15) / 16;
@@ -444,31 +449,33 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
   const int ch = chunk > 0 ? chunk : 1;
   cudaError_t e;
   if (!a.block_table) {
-    e = launch_split<DK, DV, kPacked>(a, ch, SMEM, 0, s);
+    e = launch_split<T, DK, DV, kPacked>(a, ch, SMEM, 0, s);
   } else {
     // a chunk spans at most ch / block_size + 2 blocks; stage their ids in shared memory
     // when that keeps two CTAs per SM (113 KB each), else read the table from global memory
     const long long rows = kStages * kStageKeys * 8;
     const long long ids = (long long)ch / a.block_size + 2;
     const long long smem_t = (long long)SMEM + rows + 4 * ((ids + 31) / 32 * 32);
-    e = smem_t <= 113 * 1024 ? launch_split<DK, DV, kPagedSmemTable>(a, ch, (int)smem_t, SMEM, s)
-                             : launch_split<DK, DV, kPagedGlobalTable>(a, ch, SMEM + (int)rows, SMEM, s);
+    e = smem_t <= 113 * 1024 ? launch_split<T, DK, DV, kPagedSmemTable>(a, ch, (int)smem_t, SMEM, s)
+                             : launch_split<T, DK, DV, kPagedGlobalTable>(a, ch, SMEM + (int)rows, SMEM, s);
   }
   if (e != cudaSuccess) return e;
   const long long rows = (long long)a.batch * a.hq;
-  decode_merge_kernel<DV><<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(a, chunk > 0 ? chunk : 1);
+  decode_merge_kernel<T, DV><<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(a, chunk > 0 ? chunk : 1);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool decode_split_supported(int dk, int dv, int dtype) {
-  return dtype == 0 && (dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128);
+  return (dtype == 0 || dtype == 2) && (dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128);
 }
 
-cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s) {
+namespace {
+template <typename T>
+cudaError_t launch_dims(const DecodeArgs& a, cudaStream_t s) {
 #define ATTN_SINK_DEC_CASE(DK_, DV_) \
-  if (a.dk == DK_ && a.dv == DV_) return launch_typed<DK_, DV_>(a, s);
+  if (a.dk == DK_ && a.dv == DV_) return launch_typed<T, DK_, DV_>(a, s);
   ATTN_SINK_DEC_CASE(64, 32)
   ATTN_SINK_DEC_CASE(64, 64)
   ATTN_SINK_DEC_CASE(64, 128)
@@ -477,6 +484,11 @@ cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s) {
   ATTN_SINK_DEC_CASE(128, 128)
 #undef ATTN_SINK_DEC_CASE
   return cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t launch_decode_split(const DecodeArgs& a, int dtype, cudaStream_t s) {
+  return dtype == 2 ? launch_dims<__half>(a, s) : launch_dims<__nv_bfloat16>(a, s);
 }
 
 }  // namespace attn_sink

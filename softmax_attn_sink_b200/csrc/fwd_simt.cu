@@ -150,7 +150,8 @@ cudaError_t dispatch_dims(const FwdArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_fwd_simt(const FwdArgs& a, int dtype, cudaStream_t s) {
-  return dtype == 1 ? dispatch_dims<float>(a, s) : dispatch_dims<__nv_bfloat16>(a, s);
+  if (dtype == 1) return dispatch_dims<float>(a, s);
+  return dtype == 2 ? dispatch_dims<__half>(a, s) : dispatch_dims<__nv_bfloat16>(a, s);
 }
 
 }  // namespace attn_sink

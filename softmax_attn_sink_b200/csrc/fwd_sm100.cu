@@ -299,7 +299,7 @@ struct ItemDesc {
 };
 static_assert(sizeof(ItemDesc) == 128, "item slot size");
 
-template <int DK, int DV>
+template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -409,8 +409,8 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
     // ================================ MMA issuer =========================================
     regs_dec<kRegsProducer>();
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(kBM, DV, 0, 1);
+      constexpr uint32_t idesc_qk = idesc_of<T>(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_of<T>(kBM, DV, 0, 1);
       // Shared-memory descriptors, built once: an address offset is an addition to the start
       // field (addresses stay below 2^18 bytes, so the 14-bit field never carries).
       const uint64_t dQ0 = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
@@ -622,7 +622,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
                                    sc2, nm2);
             const float2 pp = make_float2(ex2(x.x), ex2(x.y));
             sv[c & 1] = fadd2(sv[c & 1], pp);
-            pk[c] = pack_bf16x2(pp.x, pp.y);
+            pk[c] = pack2<T>(pp.x, pp.y);
           }
           tmem_st32(tS + hh * 32, pk);
         }
@@ -667,7 +667,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       const float den = l + e_sink;
       const float inv = den > 0.f ? 1.f / den : 0.f;
       const long long grow = (long long)q0 + i;   // packed row of this thread's query
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+      T* out = static_cast<T*>(a.out);
       uint4* orow = reinterpret_cast<uint4*>(out + (grow * a.hq + h) * DV);
 #pragma unroll
       for (int c = 0; c < DV / 32; ++c) {
@@ -682,7 +682,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          pk[e] = pack2<T>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         if (row_ok) {
 #pragma unroll
           for (int v = 0; v < 4; ++v)
@@ -722,16 +722,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, heads, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 128 rows x 1 head x
-// 64 columns (128 bytes), 128-byte swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows) {
+// [rows, heads, d] of 16-bit elements viewed as a 3-D tensor (d innermost); boxes of 128 rows x
+// 1 head x 64 columns (128 bytes), 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows, CUtensorMapDataType dt) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * heads};
   const cuuint32_t box[3] = {64, 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -769,7 +769,11 @@ void schedule_shape(const FwdArgs& a, int& zmax, int& width) {
   width = even ? a.hq / 2 : a.hq;
 }
 
-template <int DK, int DV>
+template <typename T> constexpr CUtensorMapDataType tma_dtype();
+template <> constexpr CUtensorMapDataType tma_dtype<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
+template <> constexpr CUtensorMapDataType tma_dtype<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
+
+template <typename T, int DK, int DV>
 cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   using L = Layout<DK, DV>;
   int zmax, width;
@@ -779,8 +783,9 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   cudaError_t e = device_shape(dev);
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, a.q, DK, a.hq, a.total_q) || !make_map(&tk, a.k, DK, a.hkv, a.total_k) ||
-      !make_map(&tv, a.v, DV, a.hkv, a.total_k))
+  constexpr CUtensorMapDataType dt = tma_dtype<T>();
+  if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
+      !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt))
     return cudaErrorInvalidValue;
   // Persistent launch (one CTA per SM walking the item list) when the item table fits in
   // shared memory; otherwise one CTA per item of the dense (level, sequence, unit pair) grid.
@@ -789,16 +794,16 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   Sched sc{zmax, width, smem_p <= dev.smem_optin ? 1 : 0};
   const long long smem = sc.persistent ? smem_p : L::smem_bytes(0);
   const long long grid = sc.persistent ? (items_ub < dev.sms ? items_ub : dev.sms) : items_ub;
-  e = cudaFuncSetAttribute(fwd_sm100_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(fwd_sm100_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  fwd_sm100_kernel<DK, DV><<<(unsigned)grid, kThreads, (size_t)smem, s>>>(a, sc, tq, tk, tv);
+  fwd_sm100_kernel<T, DK, DV><<<(unsigned)grid, kThreads, (size_t)smem, s>>>(a, sc, tq, tk, tv);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool fwd_sm100_supported(const FwdArgs& a, int dtype) {
-  if (dtype != 0 || a.cu_q == nullptr) return false;
+  if ((dtype != 0 && dtype != 2) || a.cu_q == nullptr) return false;
   if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
   int zmax, width;
   schedule_shape(a, zmax, width);
@@ -806,12 +811,19 @@ bool fwd_sm100_supported(const FwdArgs& a, int dtype) {
   return encode_fn() != nullptr;
 }
 
-cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s) {
-  if (a.dk == 128 && a.dv == 128) return launch_typed<128, 128>(a, s);
-  if (a.dk == 128 && a.dv == 64) return launch_typed<128, 64>(a, s);
-  if (a.dk == 64 && a.dv == 64) return launch_typed<64, 64>(a, s);
-  if (a.dk == 64 && a.dv == 128) return launch_typed<64, 128>(a, s);
+namespace {
+template <typename T>
+cudaError_t launch_dims(const FwdArgs& a, cudaStream_t s) {
+  if (a.dk == 128 && a.dv == 128) return launch_typed<T, 128, 128>(a, s);
+  if (a.dk == 128 && a.dv == 64) return launch_typed<T, 128, 64>(a, s);
+  if (a.dk == 64 && a.dv == 64) return launch_typed<T, 64, 64>(a, s);
+  if (a.dk == 64 && a.dv == 128) return launch_typed<T, 64, 128>(a, s);
   return cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const FwdArgs& a, int dtype, cudaStream_t s) {
+  return dtype == 2 ? launch_dims<__half>(a, s) : launch_dims<__nv_bfloat16>(a, s);
 }
 
 }  // namespace attn_sink

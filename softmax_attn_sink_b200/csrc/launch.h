@@ -76,18 +76,18 @@ struct DecodeArgs {
   int block_size, max_blocks, num_blocks;
 };
 
-// dtype: 0 = bf16, 1 = fp32.  Each returns cudaSuccess or the launch error.
+// dtype: 0 = bf16, 1 = fp32, 2 = fp16.  Each returns cudaSuccess or the launch error.
 cudaError_t launch_fwd_simt(const FwdArgs& a, int dtype, cudaStream_t s);
 bool fwd_sm100_supported(const FwdArgs& a, int dtype);
-cudaError_t launch_fwd_sm100(const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_fwd_sm100(const FwdArgs& a, int dtype, cudaStream_t s);
 
 // D, lse_tot and dsink (dsink cleared first); shared by both backward paths.
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_bwd_simt(const BwdArgs& a, int dtype, cudaStream_t s);
 bool bwd_sm100_supported(const BwdArgs& a, int dtype);
-cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
 
-cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_split(const DecodeArgs& a, int dtype, cudaStream_t s);
 
 // A one-thread kernel whose bounded mbarrier wait is made to run out (diagnostics).
 cudaError_t launch_wait_timeout_selftest(unsigned* status, cudaStream_t s);

@@ -214,12 +214,25 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
 // a_mn / b_mn: 1 = the operand is MN-major (its M or N index is the contiguous one).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+// Instruction descriptor of a kind::f16 MMA with fp32 accumulation: A and B both bf16
+// (fmt 1) or both f16 (fmt 0).
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, int a_mn, int b_mn, uint32_t fmt) {
   return (1u << 4)                       // D format: f32
-         | (1u << 7)                     // A format: bf16
-         | (1u << 10)                    // B format: bf16
+         | (fmt << 7)                    // A format
+         | (fmt << 10)                   // B format (same type as A)
          | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return idesc_f16kind(M, N, a_mn, b_mn, 1u);
+}
+// A/B format code of an element type in the descriptor above.
+template <typename T> struct TcFmt;
+template <> struct TcFmt<__nv_bfloat16> { static constexpr uint32_t value = 1u; };
+template <> struct TcFmt<__half> { static constexpr uint32_t value = 0u; };
+template <typename T>
+__host__ __device__ constexpr uint32_t idesc_of(int M, int N, int a_mn, int b_mn) {
+  return idesc_f16kind(M, N, a_mn, b_mn, TcFmt<T>::value);
 }
 
 __device__ __forceinline__ float ex2(float x) {

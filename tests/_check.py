@@ -3,6 +3,9 @@
 Tolerances (stated for this operation): bf16 inputs with fp32 accumulation
   |out - ref| <= 1e-2 + 1e-2 |ref|,  |lse - ref| <= 2e-3,
   dq / dk / dv / dsink relative L2 error <= 2e-2;
+fp16 inputs: out 2.5e-3 + 2.5e-3 |ref|, lse 1e-3, gradients 5e-3: the tensor cores see P
+  and dS rounded to fp16 (unit roundoff 2^-11 = 4.9e-4) and the outputs are rounded once
+  more, so about five unit roundoffs per output with room for fp32 accumulation order;
 fp32 inputs: the same checks with 1e-4 in place of each bf16 bound.
 A row with no visible key must have lse = -inf on both sides.
 """
@@ -10,6 +13,7 @@ import numpy as np
 
 TOL = {
     "bf16": {"out_abs": 1e-2, "out_rel": 1e-2, "lse": 2e-3, "grad": 2e-2},
+    "fp16": {"out_abs": 2.5e-3, "out_rel": 2.5e-3, "lse": 1e-3, "grad": 5e-3},
     "fp32": {"out_abs": 1e-4, "out_rel": 1e-4, "lse": 1e-4, "grad": 1e-4},
 }
 

@@ -7,7 +7,7 @@ import softmax_attn_sink_b200 as sab
 
 
 def tdtype(p):
-    return torch.bfloat16 if p.dtype == "bf16" else torch.float32
+    return {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}[p.dtype]
 
 
 def dev(x, dtype=None):
@@ -45,7 +45,7 @@ def run_bwd(p):
 
 
 def run_decode(d, num_splits=0, k_dev=None, v_dev=None):
-    td = torch.bfloat16 if d.dtype == "bf16" else torch.float32
+    td = tdtype(d)
     q = dev(d.q, td)
     k = k_dev if k_dev is not None else dev(d.k, td)
     v = v_dev if v_dev is not None else dev(d.v, td)

@@ -490,3 +490,10 @@ def test_p13_shared_prefix_block():
     # and the result is attention over block 1 alone
     o_ref, _ = ref.decode(q[:1], kc[1], vc[1], np.array([0, 16]), None, 0.3, True)
     assert np.allclose(o[0], o_ref[0], rtol=0, atol=1e-15)
+
+
+def test_fp16_rounding_matches_torch():
+    """The fp16 inputs are the values torch's float16 conversion gives (nearest, ties to even)."""
+    x = np.random.default_rng(3).standard_normal(10000).astype(np.float32) * 100
+    x[:4] = [65504.0, 1e-8, -2.0 ** -24 * 1.5, 0.5 + 2.0 ** -12]
+    assert np.array_equal(W.fp16_round(x), torch.from_numpy(x).to(torch.float16).float().numpy())

@@ -66,6 +66,23 @@ def test_paged_decode_matches_oracle(case):
     assert sab.device_status()[0] == 0
 
 
+def test_paged_decode_fp16():
+    """fp16 K/V through a shuffled 48-key table."""
+    lens = [47, 700, 1300]
+    d = W.random_decode(21, lens, 8, 2, 128, 128, dtype="fp16")
+    table, nb = W.paged_layout(22, lens, 48)
+    kc = W.to_paged(d.k, d.cu_seqlens_k, table, 48, nb)
+    vc = W.to_paged(d.v, d.cu_seqlens_k, table, 48, nb)
+    used = np.asarray(lens, np.int32)
+    out, lse = sab.attn_sink_decode_paged(
+        _dev(d.q, torch.float16), _dev(kc, torch.float16), _dev(vc, torch.float16), _dev(table),
+        _dev(used), max(lens), _dev(d.sink), d.softmax_scale, True)
+    torch.cuda.synchronize()
+    ro, rl = ref.decode_paged(d.q, kc, vc, table, used, 48, d.sink, d.softmax_scale, True)
+    check_out(to_np(out), ro, "fp16")
+    check_lse(to_np(lse), rl, "fp16")
+
+
 def test_paged_equals_packed_decode_bits():
     """The same keys read packed or through a shuffled block table give identical bits when
     the chunking is the same (one split)."""

@@ -60,6 +60,11 @@ FWD_CASES = [
     ("persistent_even_group", _LENS_B, _LENS_B, 8, 2, 128, 128, True, -1, -1, "normal", "bf16"),
     ("persistent_window_sk_gt_sq", _LENS_A, [n + 37 for n in _LENS_A], 4, 4, 128, 64, True, 200, 0,
      "uniform", "bf16"),
+    # fp16 inputs on the tensor-core path (both unit arrangements) and on the CUDA-core one
+    ("fp16_causal_gqa", _LENS_B[:8], _LENS_B[:8], 8, 2, 128, 128, True, -1, -1, "normal", "fp16"),
+    ("fp16_odd_group_window", [300, 129], [333, 200], 3, 1, 128, 64, True, 100, 0, "normal", "fp16"),
+    ("fp16_dk64", [257, 64], [257, 64], 4, 2, 64, 64, False, -1, -1, "uniform", "fp16"),
+    ("fp16_dv32_simt", [190], [190], 2, 1, 128, 32, True, -1, -1, "normal", "fp16"),
     # 9000 sequences: the item table would not fit in shared memory, so the forward runs one
     # CTA per item of the dense grid instead.
     ("grid_mode_many_sequences", _LENS_C, _LENS_C, 2, 1, 128, 128, True, -1, -1, "normal", "bf16"),
@@ -118,6 +123,10 @@ BWD_CASES = [
     ("neg_inf_sink_masked_rows", [5, 260], [2, 260], 4, 2, 128, 128, True, -1, -1, "neg_inf", "bf16"),
     ("fp32_gqa", [70, 33], [80, 33], 4, 2, 128, 64, True, -1, -1, "normal", "fp32"),
     ("fp32_window", [90], [90], 2, 2, 64, 64, False, 10, 5, "normal", "fp32"),
+    ("fp16_varlen_gqa", [1, 129, 0, 257], [1, 129, 0, 257], 8, 2, 128, 128, True, -1, -1, "normal", "fp16"),
+    ("fp16_dv64_window", [260], [300], 2, 1, 128, 64, True, 50, 0, "normal", "fp16"),
+    ("fp16_dk64", [300, 131], [300, 131], 4, 1, 64, 64, True, -1, -1, "normal", "fp16"),
+    ("fp16_dv32_simt", [150, 90], [160, 90], 2, 1, 64, 32, True, 40, 0, "normal", "fp16"),
 ]
 
 
@@ -156,13 +165,15 @@ DECODE_CASES = [
     ("no_sink", [257, 65], 8, 2, 128, 128, True, -1, -1, None, 0),
     ("neg_inf_sink_empty_seq", [0, 70], 8, 2, 128, 128, True, -1, -1, "neg_inf", 0),
     ("fp32", [300, 41], 8, 2, 128, 64, True, -1, -1, "normal", 0),
+    ("fp16_gqa8", [1, 63, 1000, 4097], 16, 2, 128, 128, True, -1, -1, "normal", 0),
+    ("fp16_dk64_dv32", [333, 1000], 8, 2, 64, 32, True, -1, -1, "normal", 3),
 ]
 
 
 @pytest.mark.parametrize("case", DECODE_CASES, ids=[c[0] for c in DECODE_CASES])
 def test_decode_matches_oracle(case):
     name, lk, hq, hkv, dk, dv, causal, wl, wr, sink, splits = case
-    dtype = "fp32" if name.startswith("fp32") else "bf16"
+    dtype = name.split("_")[0] if name.split("_")[0] in ("fp32", "fp16") else "bf16"
     d = W.random_decode(_seed(name) + 3, lk, hq, hkv, dk, dv, causal, wl, wr, sink, dtype)
     out, lse = run_decode(d, splits)
     ro, rl = ref.decode(d.q, d.k, d.v, d.cu_seqlens_k, d.sink, d.softmax_scale, causal, wl, wr)

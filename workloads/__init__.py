@@ -108,9 +108,16 @@ def cu_from_lengths(lengths: Sequence[int]) -> np.ndarray:
     return out
 
 
+def fp16_round(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest fp16 (ties to even, numpy's conversion); float32."""
+    return np.asarray(x, dtype=np.float32).astype(np.float16).astype(np.float32)
+
+
 def _normal(rng, shape, std=1.0, dtype="bf16") -> np.ndarray:
     x = (rng.standard_normal(size=shape, dtype=np.float32) * np.float32(std)).astype(np.float32)
-    return bf16_round(x) if dtype == "bf16" else x
+    if dtype == "bf16":
+        return bf16_round(x)
+    return fp16_round(x) if dtype == "fp16" else x
 
 
 def _draw_sink(rng, hq: int, kind) -> Optional[np.ndarray]:
@@ -170,17 +177,18 @@ def config2_lengths() -> np.ndarray:
     return rng.integers(64, 4096, size=16, endpoint=True)
 
 
-def config2() -> Problem:
+def config2(dtype: str = "bf16") -> Problem:
+    """The headline workload; dtype "fp16" rounds the same draws to fp16 instead of bf16."""
     rng = np.random.default_rng(1)
     lengths = rng.integers(64, 4096, size=16, endpoint=True)
     cu = cu_from_lengths(lengths)
     t = int(cu[-1])
-    q = _normal(rng, (t, 32, 128))
-    k = _normal(rng, (t, 8, 128))
-    v = _normal(rng, (t, 8, 128))
+    q = _normal(rng, (t, 32, 128), dtype=dtype)
+    k = _normal(rng, (t, 8, 128), dtype=dtype)
+    v = _normal(rng, (t, 8, 128), dtype=dtype)
     sink = rng.standard_normal(size=32, dtype=np.float32)
     return Problem(q, k, v, cu, cu.copy(), sink, _f32(1.0 / math.sqrt(128)), True, -1, -1,
-                   "bf16", None, "varlen16_gqa32x8_d128_causal")
+                   dtype, None, "varlen16_gqa32x8_d128_causal" + ("_fp16" if dtype == "fp16" else ""))
 
 
 def config3(with_dout: bool = True) -> Problem:
