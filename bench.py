@@ -380,9 +380,14 @@ def bench_fwd_bwd(args, world, peaks, peak_kind):
     b_per, b_total = time_steps(
         lambda: sab.attn_sink_bwd(q, k, v, out, do, lse, cu, cu, 8192, 8192, sink, p.softmax_scale,
                                   True, dq=dq, dk=dk, dv=dv, dsink=dsink), steps, args.warmup, world, flush)
+    d_per, d_total = time_steps(
+        lambda: sab.attn_sink_bwd(q, k, v, out, do, lse, cu, cu, 8192, 8192, sink, p.softmax_scale,
+                                  True, dq=dq, dk=dk, dv=dv, dsink=dsink, deterministic=True),
+        steps, args.warmup, world, flush)
     ff, bf = 2 * 256 * pairs, 2 * (3 * 128 + 2 * 128) * pairs
     fa = ff / (statistics.mean(f_per) * 1e-3) / 1e12
     ba = bf / (statistics.mean(b_per) * 1e-3) / 1e12
+    da = bf / (statistics.mean(d_per) * 1e-3) / 1e12
     pk = peaks["bf16_tflops"]
     return {
         "workload": f"train{args.seqs}x8192_h16_d128_causal", "pairs": pairs, "steps": steps,
@@ -397,6 +402,13 @@ def bench_fwd_bwd(args, world, peaks, peak_kind):
                              "unit": "TFLOP/s", "frac": round(ba / pk, 4),
                              "traffic": kernel_traffic("bwd_sm100.cu") if args.seqs == 4 else None,
                              "peak_source": f"bf16_tflops ({peak_kind}, burst)"}},
+        # the same algorithmic flops; the deterministic pass recomputes Q K^T and dout V^T
+        "bwd_deterministic": {"value": round(bf * world / (d_total / steps * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                              "ms_per_step": round(d_total / steps, 4), "flops": bf,
+                              "roofline": {"bound": "tensor", "achieved": round(da, 2), "peak": pk,
+                                           "unit": "TFLOP/s", "frac": round(da / pk, 4), "traffic": None,
+                                           "peak_source": f"bf16_tflops ({peak_kind}, burst)",
+                                           "kernels": "preprocess + key-stationary dK/dV + query-stationary dQ"}},
     }
 
 

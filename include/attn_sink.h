@@ -127,6 +127,21 @@ int attn_sink_bwd(const attn_sink_params* params, const void* q, const void* k, 
                   size_t workspace_bytes, attn_sink_stream_t stream);
 
 /*
+ * Deterministic backward: the same arguments, results and workspace size as
+ * attn_sink_bwd, and bit-identical outputs from run to run (the slime wrapper exposes a
+ * `deterministic` flag for the same purpose).  attn_sink_bwd adds the dQ contributions of
+ * different key tiles with fp32 atomics, whose order varies; here dQ is computed by a
+ * query-stationary pass that adds them in a fixed order (dK, dV and dsink are reduced in a
+ * fixed order by both entry points).  Slower than attn_sink_bwd: Q K^T and dout V^T are
+ * computed twice.
+ */
+int attn_sink_bwd_deterministic(const attn_sink_params* params, const void* q, const void* k,
+                                const void* v, const void* out, const void* dout, const float* lse,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                const float* sink, void* dq, void* dk, void* dv, float* dsink,
+                                void* workspace, size_t workspace_bytes, attn_sink_stream_t stream);
+
+/*
  * Decode: one query per sequence, q [batch, Hq, dk] (cu_seqlens_q = 0, 1, ..., batch is
  * implied; total_q == batch, max_seqlen_q == 1).  K/V are packed with cu_seqlens_k.
  * The keys of each (sequence, kv head) are cut into num_splits chunks (0 = choose

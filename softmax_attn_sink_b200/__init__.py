@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.attn_sink_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.attn_sink_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.attn_sink_decode.argtypes = [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]
+        L.attn_sink_bwd_deterministic.argtypes = list(L.attn_sink_bwd.argtypes)
+        L.attn_sink_bwd_deterministic.restype = i32
         L.attn_sink_decode_paged.argtypes = [P, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, sz, vp]
         for f in (L.attn_sink_fwd, L.attn_sink_bwd, L.attn_sink_decode, L.attn_sink_decode_paged):
             f.restype = i32
@@ -202,8 +204,9 @@ def attn_sink_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_se
 def attn_sink_bwd(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                   max_seqlen_k: int, sink=None, softmax_scale: Optional[float] = None,
                   causal: bool = False, window_size: Sequence[int] = (-1, -1), dq=None, dk=None,
-                  dv=None, dsink=None, stream=None):
-    """Backward for the loss sum(dout * out).  Returns (dq, dk, dv, dsink)."""
+                  dv=None, dsink=None, stream=None, deterministic: bool = False):
+    """Backward for the loss sum(dout * out).  Returns (dq, dk, dv, dsink).  With
+    deterministic=True the results are bit-identical from run to run (slower)."""
     torch = _torch()
     p = _common(q, k, v, cu_seqlens_q, cu_seqlens_k, sink, max_seqlen_q, max_seqlen_k,
                 softmax_scale, causal, window_size)
@@ -219,12 +222,13 @@ def attn_sink_bwd(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqle
     if ws_bytes == ctypes.c_size_t(-1).value:
         raise AttnSinkError("attn_sink_bwd_workspace_size", 1)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
-    st = lib().attn_sink_bwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                             out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
-                             cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), _ptr(sink),
-                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dsink.data_ptr(),
-                             ws.data_ptr(), ws_bytes, _stream(stream))
-    _check("attn_sink_bwd", st)
+    fn = lib().attn_sink_bwd_deterministic if deterministic else lib().attn_sink_bwd
+    st = fn(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+            out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+            cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), _ptr(sink),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dsink.data_ptr(),
+            ws.data_ptr(), ws_bytes, _stream(stream))
+    _check("attn_sink_bwd_deterministic" if deterministic else "attn_sink_bwd", st)
     return dq, dk, dv, dsink
 
 

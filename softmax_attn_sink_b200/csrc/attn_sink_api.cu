@@ -62,16 +62,19 @@ void effective_window(const attn_sink_params* p, int& left, int& right) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? ATTN_SINK_OK : ATTN_SINK_ERR_CUDA; }
 
-// workspace layout of the backward
+// workspace layout of the backward: D, lse_tot, the preprocess blocks' d_sink partials
+// ([hq][ceil(total_q / 64)]), then the fp32 dQ accumulator of the tensor-core path
 struct BwdLayout {
-  size_t D, lse_tot, dq_acc, total;
+  size_t D, lse_tot, dsink_part, dq_acc, total;
 };
 BwdLayout bwd_layout(const attn_sink_params* p) {
   BwdLayout l{};
   const size_t rows = (size_t)p->num_heads_q * p->total_q;
+  const size_t parts = (size_t)p->num_heads_q * ((p->total_q + 63) / 64);
   l.D = 0;
   l.lse_tot = align_up(l.D + rows * 4, 256);
-  l.dq_acc = align_up(l.lse_tot + rows * 4, 256);
+  l.dsink_part = align_up(l.lse_tot + rows * 4, 256);
+  l.dq_acc = align_up(l.dsink_part + parts * 4, 256);
   size_t end = l.dq_acc;
   if (p->dtype != ATTN_SINK_FP32) end += (size_t)p->total_q * p->num_heads_q * p->head_dim_qk * 4;
   l.total = align_up(end, 256);
@@ -120,6 +123,53 @@ int launch_decode(const attn_sink_params* p, DecodeArgs& a, int num_splits, void
   a.splits = splits; a.scale = p->softmax_scale; a.left = left; a.right = right;
   a.status = status_ptr();
   return from_cuda(launch_decode_split(a, p->dtype, s));
+}
+
+// The backward, with dQ reduced by fp32 atomics into a workspace accumulator (fast) or, in
+// the deterministic mode, computed by a query-stationary pass that adds the key tiles'
+// contributions in a fixed order.
+int run_bwd(const attn_sink_params* p, const void* q, const void* k, const void* v, const void* out,
+            const void* dout, const float* lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+            const float* sink, void* dq, void* dk, void* dv, float* dsink, void* workspace,
+            size_t workspace_bytes, attn_sink_stream_t stream, bool deterministic) {
+  int st = validate_params(p, false);
+  if (st != ATTN_SINK_OK) return st;
+  if (!q || !k || !v || !out || !dout || !lse || !cu_seqlens_q || !cu_seqlens_k || !dq || !dk || !dv)
+    return ATTN_SINK_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, out, dout, (const void*)lse, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
+  if ((sink && !aligned16(sink)) || (dsink && !aligned16(dsink))) return ATTN_SINK_ERR_INVALID_ARG;
+  const BwdLayout lay = bwd_layout(p);
+  if (!workspace || workspace_bytes < lay.total || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  BwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.lse = lse;
+  a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
+  a.grad_q = dq; a.grad_k = dk; a.grad_v = dv; a.dsink = dsink;
+  a.D = reinterpret_cast<float*>(ws + lay.D);
+  a.lse_tot = reinterpret_cast<float*>(ws + lay.lse_tot);
+  a.dsink_part = reinterpret_cast<float*>(ws + lay.dsink_part);
+  a.dq_acc = (p->dtype != ATTN_SINK_FP32 && !deterministic) ? reinterpret_cast<float*>(ws + lay.dq_acc) : nullptr;
+  a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
+  a.max_sq = p->max_seqlen_q; a.max_sk = p->max_seqlen_k;
+  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
+  a.scale = p->softmax_scale;
+  effective_window(p, a.left, a.right);
+  a.status = status_ptr();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
+  if (!deterministic) {
+    if (bwd_sm100_supported(a, dt)) return from_cuda(launch_bwd_sm100(a, dt, s));
+    return from_cuda(launch_bwd_simt(a, dt, s));
+  }
+  // deterministic: dK / dV on the key-stationary tensor-core kernel without its dQ part,
+  // then dQ query-stationary; the CUDA-core path has no atomics to begin with
+  if (bwd_sm100_supported(a, dt) && bwd_dq_sm100_supported(a, dt)) {
+    cudaError_t e = launch_bwd_sm100(a, dt, s);
+    if (e == cudaSuccess) e = launch_bwd_dq_sm100(a, dt, s);
+    return from_cuda(e);
+  }
+  return from_cuda(launch_bwd_simt(a, dt, s));
 }
 
 }  // namespace
@@ -188,38 +238,23 @@ int attn_sink_fwd(const attn_sink_params* p, const void* q, const void* k, const
   return from_cuda(launch_fwd_simt(a, dt, s));
 }
 
+
 int attn_sink_bwd(const attn_sink_params* p, const void* q, const void* k, const void* v,
                   const void* out, const void* dout, const float* lse,
                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
                   void* dq, void* dk, void* dv, float* dsink, void* workspace,
                   size_t workspace_bytes, attn_sink_stream_t stream) {
-  int st = validate_params(p, false);
-  if (st != ATTN_SINK_OK) return st;
-  if (!q || !k || !v || !out || !dout || !lse || !cu_seqlens_q || !cu_seqlens_k || !dq || !dk || !dv)
-    return ATTN_SINK_ERR_INVALID_ARG;
-  for (const void* ptr : {q, k, v, out, dout, (const void*)lse, (const void*)dq, (const void*)dk, (const void*)dv})
-    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
-  if ((sink && !aligned16(sink)) || (dsink && !aligned16(dsink))) return ATTN_SINK_ERR_INVALID_ARG;
-  const BwdLayout lay = bwd_layout(p);
-  if (!workspace || workspace_bytes < lay.total || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
-  BwdArgs a{};
-  a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.lse = lse;
-  a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
-  a.grad_q = dq; a.grad_k = dk; a.grad_v = dv; a.dsink = dsink;
-  a.D = reinterpret_cast<float*>(ws + lay.D);
-  a.lse_tot = reinterpret_cast<float*>(ws + lay.lse_tot);
-  a.dq_acc = p->dtype != ATTN_SINK_FP32 ? reinterpret_cast<float*>(ws + lay.dq_acc) : nullptr;
-  a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
-  a.max_sq = p->max_seqlen_q; a.max_sk = p->max_seqlen_k;
-  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
-  a.scale = p->softmax_scale;
-  effective_window(p, a.left, a.right);
-  a.status = status_ptr();
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
-  if (bwd_sm100_supported(a, dt)) return from_cuda(launch_bwd_sm100(a, dt, s));
-  return from_cuda(launch_bwd_simt(a, dt, s));
+  return run_bwd(p, q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, sink, dq, dk, dv, dsink, workspace,
+                 workspace_bytes, stream, false);
+}
+
+int attn_sink_bwd_deterministic(const attn_sink_params* p, const void* q, const void* k, const void* v,
+                                const void* out, const void* dout, const float* lse,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
+                                void* dq, void* dk, void* dv, float* dsink, void* workspace,
+                                size_t workspace_bytes, attn_sink_stream_t stream) {
+  return run_bwd(p, q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, sink, dq, dk, dv, dsink, workspace,
+                 workspace_bytes, stream, true);
 }
 
 int attn_sink_decode(const attn_sink_params* p, const void* q, const void* k, const void* v,

@@ -1,0 +1,368 @@
+// Query-stationary dQ for the deterministic backward on the sm_100a tensor cores.
+//
+// The gradient with respect to q of the sink attention (Huawei CANN ops-transformer
+// flash_attn doc, "Function", the formula after "After adding sink"; its exact gradient,
+// which the slime learnable_softmax_attention.py docstring states as
+// dS = P * s * (D - s * di) with s = sigmoid(lse - sink)) is
+//   dq_i = scale * sum_j dS_ij k_j,   dS_ij = P_ij (dP_ij - D_i),
+//   P_ij = e^{scale q_i.k_j - lse_tot_i},  dP_ij = dout_i . v_j,  D_i = dout_i . out_i,
+// with lse_tot = logaddexp(lse, sink) from the preprocess pass.  The key-stationary kernel
+// adds dQ contributions of different key tiles with fp32 atomics, whose order varies from
+// run to run.  Here one CTA owns a 128-row query tile of one q head and walks its visible
+// key tiles in increasing order, accumulating dQ in TMEM, so every run adds the same
+// numbers in the same order.
+//
+// Per key tile j (128 keys):
+//   MMA thread:   S = Q K_j^T -> S columns, dP = dout V_j^T -> dP columns (SS, K-major),
+//                 then, once the compute warps wrote dS, dQ += dS K_j (A = dS from TMEM,
+//                 B = K_j read MN-major from the same shared-memory tile).
+//   compute warps (thread = query row, TMEM lane): two 64-key halves; P = 2^{S scale log2e
+//                 - lse_tot log2e} (masked scores are -inf, so P = 0), dS = P (dP - D),
+//                 rounded to the input type and written over the S columns of its half.
+// TMEM columns: S [0,128) dP [128,256) dQ [256,256+DK).  dS of tile j sits in S's columns
+// until dQ(j) has read it; S(j+1) is issued after dQ(j) by the same thread, and MMAs from
+// one thread execute in issue order.  Every mbarrier wait is bounded; a timeout sets the
+// status word and the CTA drains and frees its TMEM instead of hanging.
+#include <cuda.h>
+
+#include <type_traits>
+
+#include "sm100_ptx.cuh"
+
+namespace attn_sink {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;       // query rows per CTA
+constexpr int kBN = 128;       // keys per tile
+constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 compute
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+
+template <int DK, int DV>
+struct DqLayout {
+  static constexpr int KH = DK / 64, VH = DV / 64;     // 64-element (128-byte) column halves
+  static constexpr int kHalf = 128 * 128;              // one 128-row x 64-column box
+  static constexpr int kQBytes = KH * kHalf, kOBytes = VH * kHalf;
+  static constexpr int kKBytes = KH * kHalf, kVBytes = VH * kHalf;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffO = kOffQ + kQBytes;
+  static constexpr int kOffK = kOffO + kOBytes;        // K ring, 2 stages
+  static constexpr int kOffV = kOffK + 2 * kKBytes;    // V ring, 2 stages
+  static constexpr int kOffBar = kOffV + 2 * kVBytes;
+  static constexpr int kNumBars = 9;  // qd_full, kv_full[2], kv_empty[2], sdp_full, ds_full, dq_done, drain
+  static constexpr int kOffSlot = kOffBar + kNumBars * 8;
+  // + slack to align the base to 1 KB; at least 116 KB so two CTAs never share an SM (each
+  // holds all 512 TMEM columns)
+  static constexpr int kSmem = (kOffSlot + 16 + 1024) > 118784 ? (kOffSlot + 16 + 1024) : 118784;
+};
+
+struct DqBars {
+  uint32_t base;
+  __device__ __forceinline__ uint32_t qd_full() const { return base; }
+  __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 8u * (1 + s); }
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8u * (3 + s); }
+  __device__ __forceinline__ uint32_t sdp_full() const { return base + 8u * 5; }
+  __device__ __forceinline__ uint32_t ds_full() const { return base + 8u * 6; }
+  __device__ __forceinline__ uint32_t dq_done() const { return base + 8u * 7; }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * 8; }
+};
+
+// CTA -> (row tile m, sequence b, q head h): the deepest row tiles first (under a causal mask
+// they see the most keys), heads fastest so the CTAs resident together share K/V tiles.
+__device__ __forceinline__ void dq_tile_of(const BwdArgs& a, int mtiles, int& m, int& b, int& h) {
+  const long long id = blockIdx.x;
+  const long long per_level = (long long)a.batch * a.hq;
+  const int zr = (int)(id / per_level);
+  const int rem = (int)(id - (long long)zr * per_level);
+  m = mtiles - 1 - zr;
+  b = rem / a.hq;
+  h = rem - b * a.hq;
+}
+
+template <typename Elem, int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do) {
+  using L = DqLayout<DK, DV>;
+  extern __shared__ unsigned char smem_raw[];
+
+  int m, b, h;
+  dq_tile_of(a, (a.max_sq + kBM - 1) / kBM, m, b, h);
+  const long long q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
+  const long long k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
+  const long long m0 = (long long)m * kBM;
+  if (m0 >= sq) return;
+  const int g = h / (a.hq / a.hkv);
+  const long long nrows = (sq - m0 < kBM) ? sq - m0 : kBM;
+  long long lo, hi, l2, h2;
+  row_key_range(m0, sq, sk, a.left, a.right, lo, hi);
+  row_key_range(m0 + nrows - 1, sq, sk, a.left, a.right, l2, h2);
+  hi = h2 > lo ? h2 : lo;   // key ranges move right with the row: the union is [lo(first), hi(last))
+  const int n = hi > lo ? (int)((hi - lo + kBN - 1) / kBN) : 0;
+
+  const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
+  const uint32_t sQ = base_u32 + L::kOffQ, sO = base_u32 + L::kOffO, sK = base_u32 + L::kOffK,
+                 sV = base_u32 + L::kOffV;
+  const DqBars bar{base_u32 + L::kOffBar};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar.qd_full(), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar.kv_full(s), 1);
+      mbar_init(bar.kv_empty(s), 1);
+    }
+    mbar_init(bar.sdp_full(), 1);
+    mbar_init(bar.ds_full(), 4);   // one arrival per compute warp
+    mbar_init(bar.dq_done(), 1);
+    mbar_init(bar.drain(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================================ TMA producer ======================================
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      const int row = (int)(q0 + m0);
+      mbar_arrive_expect_tx(bar.qd_full(), L::kQBytes + L::kOBytes);
+      for (int hf = 0; hf < L::KH; ++hf) tma_load_3d(sQ + hf * L::kHalf, &tm_q, bar.qd_full(), hf * 64, h, row);
+      for (int hf = 0; hf < L::VH; ++hf) tma_load_3d(sO + hf * L::kHalf, &tm_do, bar.qd_full(), hf * 64, h, row);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(bar.kv_empty(st), ((j >> 1) & 1) ^ 1, a.status)) break;
+        const int krow = (int)(k0 + lo + (long long)j * kBN);
+        mbar_arrive_expect_tx(bar.kv_full(st), L::kKBytes + L::kVBytes);
+        for (int hf = 0; hf < L::KH; ++hf)
+          tma_load_3d(sK + st * L::kKBytes + hf * L::kHalf, &tm_k, bar.kv_full(st), hf * 64, g, krow);
+        for (int hf = 0; hf < L::VH; ++hf)
+          tma_load_3d(sV + st * L::kVBytes + hf * L::kHalf, &tm_v, bar.kv_full(st), hf * 64, g, krow);
+        issued = j + 1;
+      }
+      // make sure no copy is still landing in shared memory when the CTA exits
+      mbar_wait(bar.qd_full(), 0, a.status);
+      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
+        mbar_wait(bar.kv_full(j & 1), (j >> 1) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    // ================================ MMA issuer =========================================
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t id_s = idesc_of<Elem>(kBM, kBN, 0, 0);   // S, dP: K-major A and B
+      constexpr uint32_t id_q = idesc_of<Elem>(kBM, DK, 0, 1);    // dS (TMEM) x K (MN-major)
+      // Shared-memory descriptors, built once; offsets add to the start field.  "k" = K-major
+      // view, "m" = MN-major view (LBO = the 16 KB between 64-column halves).
+      const uint64_t kQ = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t kO = smem_desc(sO, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t kK = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
+      const uint64_t mK = smem_desc(sK, L::kHalf, 1024, kLayoutSwizzle128B);
+      const uint64_t kV = smem_desc(sV, 16, 1024, kLayoutSwizzle128B);
+      bool ok = mbar_wait(bar.qd_full(), 0, a.status);
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j & 1;
+        if (!(ok = mbar_wait(bar.kv_full(st), (j >> 1) & 1, a.status))) break;
+        tc_fence_after();
+        const uint64_t koff = (uint64_t)((st * L::kKBytes) >> 4), voff = (uint64_t)((st * L::kVBytes) >> 4);
+        // S = Q K^T and dP = dout V^T.  S's columns held dS(j - 1), read by dQ(j - 1), which
+        // this thread issued earlier.
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + kColS, kQ + off16, kK + koff + off16, id_s, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < DV / 16; ++ks) {
+          const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + kColP, kO + off16, kV + voff + off16, id_s, ks > 0);
+        }
+        mma_commit(bar.sdp_full());
+        // dQ += dS K, once the compute warps have written dS
+        if (!(ok = mbar_wait(bar.ds_full(), j & 1, a.status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(tmem + kColQ, tmem + kColS + kk * 8, mK + koff + (uint64_t)((kk * 2048) >> 4), id_q,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar.kv_empty(st));
+      }
+      if (ok) mma_commit(bar.dq_done());
+      // every MMA must be complete before the TMEM is freed
+      mma_commit(bar.drain());
+      mbar_wait(bar.drain(), 0, a.status);
+    }
+  } else if (warp >= 4) {
+    // ================================ compute warps (thread = query row) =================
+    const int lg = warp & 3;
+    const int r = lg * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    const long long i = m0 + r;
+    const bool row_ok = i < sq;
+    int rlo = 0, rhi = 0;   // visible keys of this row relative to the first key of the loop
+    float neg_lt = 0.f, Dr = 0.f;
+    if (row_ok) {
+      long long l_, h_;
+      row_key_range(i, sq, sk, a.left, a.right, l_, h_);
+      rlo = (int)(l_ - lo);
+      rhi = (int)(h_ - lo);
+      const long long idx = (long long)h * a.total_q + q0 + i;
+      const float lt2 = a.lse_tot[idx] * kLog2e;
+      neg_lt = (lt2 == kNegInf) ? 0.f : -lt2;   // no key and no sink: every score is -inf, P = 0
+      Dr = a.D[idx];
+    }
+    const float scale2 = a.scale * kLog2e;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.sdp_full(), j & 1, a.status))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[64], pv[64];
+        tmem_ld32(tmem + lane_off + kColS + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tmem + lane_off + kColS + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tmem + lane_off + kColP + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+        tmem_ld32(tmem + lane_off + kColP + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+        tmem_wait_ld();
+        const int klo = rlo - j * kBN - hh * 64, khi = rhi - j * kBN - hh * 64;   // visible [klo, khi)
+        if (!(klo <= 0 && khi >= 64)) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < klo || c >= khi) sv[c] = __float_as_uint(kNegInf);
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), scale2, neg_lt));
+          const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), scale2, neg_lt));
+          pk[c] = pack2<Elem>(p0 * (__uint_as_float(pv[2 * c]) - Dr), p1 * (__uint_as_float(pv[2 * c + 1]) - Dr));
+        }
+        // dS of keys [64 hh, 64 hh + 64) over S columns [32 hh, 32 hh + 32): half 0 goes over
+        // S columns already read, half 1 over half 0's S columns
+        tmem_st32(tmem + lane_off + kColS + hh * 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.ds_full());
+    }
+    // ---- epilogue: dq = scale * dQ ------------------------------------------------------
+    const bool have = __all_sync(0xffffffffu, ok && n > 0 && mbar_wait(bar.dq_done(), 0, a.status));
+    tc_fence_after();
+    Elem* dqp = static_cast<Elem*>(a.grad_q) + ((q0 + i) * a.hq + h) * DK;
+#pragma unroll
+    for (int c = 0; c < DK / 32; ++c) {
+      uint32_t v[32];
+      if (n > 0) {
+        tmem_ld32(tmem + lane_off + kColQ + c * 32, v);
+        tmem_wait_ld();
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float x0 = (n > 0 && have) ? __uint_as_float(v[2 * e]) * a.scale : 0.f;
+        const float x1 = (n > 0 && have) ? __uint_as_float(v[2 * e + 1]) * a.scale : 0.f;
+        pk[e] = pack2<Elem>(x0, x1);
+      }
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(dqp) + c * 4;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- host -----------------------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, heads, d] of 16-bit elements as a 3-D tensor; boxes of 128 rows x 1 head x 64
+// columns (128 bytes), 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows, CUtensorMapDataType dt) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * heads};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename Elem, int DK, int DV>
+cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
+  using L = DqLayout<DK, DV>;
+  constexpr CUtensorMapDataType dt =
+      std::is_same<Elem, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
+      !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
+    return cudaErrorInvalidValue;
+  cudaError_t e =
+      cudaFuncSetAttribute(bwd_dq_sm100_kernel<Elem, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  if (e != cudaSuccess) return e;
+  const long long ctas = (long long)((a.max_sq + kBM - 1) / kBM) * a.batch * a.hq;
+  bwd_dq_sm100_kernel<Elem, DK, DV><<<(unsigned)ctas, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
+  return cudaGetLastError();
+}
+
+template <typename Elem>
+cudaError_t launch_dims(const BwdArgs& a, cudaStream_t s) {
+  if (a.dk == 128 && a.dv == 128) return launch_typed<Elem, 128, 128>(a, s);
+  if (a.dk == 128 && a.dv == 64) return launch_typed<Elem, 128, 64>(a, s);
+  if (a.dk == 64 && a.dv == 64) return launch_typed<Elem, 64, 64>(a, s);
+  if (a.dk == 64 && a.dv == 128) return launch_typed<Elem, 64, 128>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool bwd_dq_sm100_supported(const BwdArgs& a, int dtype) {
+  if (dtype != 0 && dtype != 2) return false;
+  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
+  if ((long long)((a.max_sq + kBM - 1) / kBM) * a.batch * a.hq > 0x7fffffffLL) return false;  // 1-D grid
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_bwd_dq_sm100(const BwdArgs& a, int dtype, cudaStream_t s) {
+  return dtype == 2 ? launch_dims<__half>(a, s) : launch_dims<__nv_bfloat16>(a, s);
+}
+
+}  // namespace attn_sink

@@ -52,8 +52,20 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
   if (threadIdx.x == 0 && a.dsink) {
     float s = 0.f;
     for (int w = 0; w < 8; ++w) s += red[w];
-    atomicAdd(a.dsink + h, s);
+    a.dsink_part[(long long)h * gridDim.x + blockIdx.x] = s;   // summed in a fixed order later
   }
+}
+
+// d_sink[h] = sum over the preprocess blocks of their partials, one warp per head: lane l
+// adds blocks l, l + 32, ... in order, then a fixed butterfly combines the lanes, so the
+// result does not depend on the order in which blocks ran.
+__global__ void __launch_bounds__(32) dsink_reduce_kernel(const BwdArgs a, int nblocks) {
+  const int h = blockIdx.x, lane = threadIdx.x;
+  const float* part = a.dsink_part + (long long)h * nblocks;
+  float s = 0.f;
+  for (int i = lane; i < nblocks; i += 32) s += part[i];
+  s = warp_sum(s);
+  if (lane == 0) a.dsink[h] = s;
 }
 
 // --- dK / dV: key-stationary -----------------------------------------------------------
@@ -297,8 +309,6 @@ cudaError_t dispatch_dims(const BwdArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s) {
-  cudaError_t e;
-  if (a.dsink && (e = cudaMemsetAsync(a.dsink, 0, sizeof(float) * a.hq, s)) != cudaSuccess) return e;
   dim3 grid((a.total_q + 63) / 64, a.hq);
   if (dtype == 1)
     bwd_preprocess_kernel<float><<<grid, 256, 0, s>>>(a);
@@ -306,6 +316,9 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s) {
     bwd_preprocess_kernel<__half><<<grid, 256, 0, s>>>(a);
   else
     bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !a.dsink) return e;
+  dsink_reduce_kernel<<<a.hq, 32, 0, s>>>(a, (int)grid.x);
   return cudaGetLastError();
 }
 

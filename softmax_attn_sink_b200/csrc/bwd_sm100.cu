@@ -105,7 +105,7 @@ struct BBars {
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * 11; }
 };
 
-template <typename Elem, int DK, int DV>
+template <typename Elem, int DK, int DV, bool DQ>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do) {
@@ -213,7 +213,7 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
           mma_ss(tmem + kColR0, smem_desc(sK + off, 16, 1024, kLayoutSwizzle128B),
                  smem_desc(q_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
         }
-        if (t >= 1 && !(ok = mbar_wait(bar.dq_free(), (t - 1) & 1, a.status))) break;   // R1 free
+        if (DQ && t >= 1 && !(ok = mbar_wait(bar.dq_free(), (t - 1) & 1, a.status))) break;   // R1 free
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DV / 16; ++ks) {
@@ -233,11 +233,13 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
         for (int kk = 0; kk < kBM / 16; ++kk)
           mma_ss(tmem + kColDK, smem_desc(sDS + (kk >> 2) * L::kHalf + (kk & 3) * 32, 16, 1024, kLayoutSwizzle128B),
                  smem_desc(q_s + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dk, (t > 0 || kk > 0));
+        if (DQ) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ss(tmem + kColR1, smem_desc(sDS + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B),
-                 smem_desc(sK + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dq, kk > 0);
-        mma_commit(bar.dq_full());
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ss(tmem + kColR1, smem_desc(sDS + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B),
+                   smem_desc(sK + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dq, kk > 0);
+          mma_commit(bar.dq_full());
+        }
         mma_commit(bar.ds_free());
         mma_commit(bar.qd_empty(st));
       }
@@ -345,7 +347,7 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
-    for (int t = 0; t < T; ++t) {
+    for (int t = 0; t < (DQ ? T : 0); ++t) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar.dq_full(), t & 1, a.status))) break;
       tc_fence_after();
       uint32_t v[DK];
@@ -434,7 +436,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <typename Elem, int DV>
+template <typename Elem, int DV, bool DQ>
 __global__ void __launch_bounds__(kThreadsP, 1)
 bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -558,7 +560,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
           const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
           mma_ss(cS, kK + off16, kQ + qoff + off16, id_s, ks > 0);
         }
-        if (t >= 1 && !mbar_wait(bar.dq_free(hh), (t - 1) & 1, a.status)) return false;   // dQ^T_h read
+        if (DQ && t >= 1 && !mbar_wait(bar.dq_free(hh), (t - 1) & 1, a.status)) return false;   // dQ^T_h read
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DV / 16; ++ks) {
@@ -582,10 +584,12 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem + kColDK, kDS + dsoff + (uint64_t)((kk * 32) >> 4),
                  mQ + qoff + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_dk, (t > 0 || hh > 0 || kk > 0));
+        if (DQ) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ss(cP, mK + (uint64_t)((kk * 2048) >> 4), mDS + dsoff + (uint64_t)((kk * 2048) >> 4), id_dq, kk > 0);
-        mma_commit(bar.dq_full(hh));
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ss(cP, mK + (uint64_t)((kk * 2048) >> 4), mDS + dsoff + (uint64_t)((kk * 2048) >> 4), id_dq, kk > 0);
+          mma_commit(bar.dq_full(hh));
+        }
         mma_commit(bar.ds_free(hh));
       };
       bool ok = mbar_wait(bar.kv_full(), 0, a.status);
@@ -744,7 +748,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     const int d = lg * 32 + lane;                     // TMEM lane = head-dim index of dQ^T
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     bool ok = true;
-    for (int t = 0; t < T && ok; ++t) {
+    for (int t = 0; t < (DQ ? T : 0) && ok; ++t) {
       const int h = head_of(t);
       const long long i0 = qbase_of(t);
       for (int hh = 0; hh < 2; ++hh) {
@@ -859,17 +863,19 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   if (!make_map(&tq, a.q, 128, a.hq, a.total_q, dt) || !make_map(&tk, a.k, 128, a.hkv, a.total_k, dt) ||
       !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * 128 * sizeof(float), s);
+  const bool dq = a.dq_acc != nullptr;
+  cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * 128 * sizeof(float), s) : cudaSuccess;
   if (e != cudaSuccess) return e;
   if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(bwd_sm100_d128_kernel<T, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                L::kSmem)) != cudaSuccess)
+  auto kernel = dq ? bwd_sm100_d128_kernel<T, DV, true> : bwd_sm100_d128_kernel<T, DV, false>;
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) != cudaSuccess)
     return e;
   BwdArgs ab = a;
   ab.band_groups = bwd_band_groups(a);
   const long long ctas = (long long)a.hkv * a.batch * ((a.max_sk + kBN - 1) / kBN);
-  bwd_sm100_d128_kernel<T, DV><<<(unsigned)ctas, kThreadsP, L::kSmem, s>>>(ab, tq, tk, tv, to);
+  kernel<<<(unsigned)ctas, kThreadsP, L::kSmem, s>>>(ab, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!dq) return cudaSuccess;
   const long long n8 = (long long)a.total_q * a.hq * 128 / 8;
   dq_convert_hmajor_kernel<T><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
       a.dq_acc, static_cast<T*>(a.grad_q), a.total_q, a.hq, n8);
@@ -884,17 +890,19 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
       !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * DK * sizeof(float), s);
+  const bool dq = a.dq_acc != nullptr;
+  cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * DK * sizeof(float), s) : cudaSuccess;
   if (e != cudaSuccess) return e;
   if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(bwd_sm100_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                L::kSmem)) != cudaSuccess)
+  auto kernel = dq ? bwd_sm100_kernel<T, DK, DV, true> : bwd_sm100_kernel<T, DK, DV, false>;
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) != cudaSuccess)
     return e;
   BwdArgs ab = a;
   ab.band_groups = bwd_band_groups(a);
   const long long ctas = (long long)a.hkv * a.batch * ((a.max_sk + kBN - 1) / kBN);
-  bwd_sm100_kernel<T, DK, DV><<<(unsigned)ctas, kThreads, L::kSmem, s>>>(ab, tq, tk, tv, to);
+  kernel<<<(unsigned)ctas, kThreads, L::kSmem, s>>>(ab, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!dq) return cudaSuccess;
   const long long n8 = (long long)a.total_q * a.hq * DK / 8;
   dq_convert_kernel<T><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.dq_acc, static_cast<T*>(a.grad_q), n8);
   return cudaGetLastError();
@@ -912,7 +920,7 @@ cudaError_t launch_dims(const BwdArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool bwd_sm100_supported(const BwdArgs& a, int dtype) {
-  if ((dtype != 0 && dtype != 2) || a.dq_acc == nullptr) return false;
+  if (dtype != 0 && dtype != 2) return false;
   if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
   if ((long long)a.batch * a.hkv * ((a.max_sk + kBN - 1) / kBN) > 0x7fffffffLL) return false;  // 1-D grid
   return encode_fn() != nullptr;

@@ -46,7 +46,8 @@ struct BwdArgs {
   float* dsink;          // may be nullptr
   float* D;              // workspace [hq, total_q]: rowsum(dout * out)
   float* lse_tot;        // workspace [hq, total_q]: logaddexp(lse, sink)
-  float* dq_acc;         // workspace [total_q, hq, dk] fp32 (tensor-core path only)
+  float* dq_acc;         // workspace [total_q, hq, dk] fp32 (tensor-core path; nullptr = no dQ there)
+  float* dsink_part;     // workspace [hq, preprocess blocks] fp32: per-block d_sink partials
   int batch, total_q, total_k, max_sq, max_sk, hq, hkv, dk, dv;
   float scale;
   int left, right;
@@ -85,7 +86,13 @@ cudaError_t launch_fwd_sm100(const FwdArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_bwd_simt(const BwdArgs& a, int dtype, cudaStream_t s);
 bool bwd_sm100_supported(const BwdArgs& a, int dtype);
+// With a.dq_acc == nullptr the tensor-core backward computes dK and dV only.
 cudaError_t launch_bwd_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
+// Query-stationary dQ without atomics (the deterministic backward's dQ pass).
+bool bwd_dq_sm100_supported(const BwdArgs& a, int dtype);
+cudaError_t launch_bwd_dq_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
+// d_sink from the preprocess pass's per-block partials, summed in a fixed order.
+cudaError_t launch_dsink_reduce(const BwdArgs& a, cudaStream_t s);
 
 cudaError_t launch_decode_split(const DecodeArgs& a, int dtype, cudaStream_t s);
 

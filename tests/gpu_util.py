@@ -30,7 +30,7 @@ def run_fwd(p):
     return out, lse
 
 
-def run_bwd(p):
+def run_bwd(p, deterministic=False):
     td = tdtype(p)
     q, k, v = dev(p.q, td), dev(p.k, td), dev(p.v, td)
     do = dev(p.dout, td)
@@ -39,7 +39,8 @@ def run_bwd(p):
     mq, mk = max(p.max_seqlen_q, 1), max(p.max_seqlen_k, 1)
     out, lse = sab.attn_sink_fwd(q, k, v, cu_q, cu_k, mq, mk, sink, p.softmax_scale, p.causal, window(p))
     dq, dk, dv, ds = sab.attn_sink_bwd(q, k, v, out, do, lse, cu_q, cu_k, mq, mk, sink,
-                                       p.softmax_scale, p.causal, window(p))
+                                       p.softmax_scale, p.causal, window(p),
+                                       deterministic=deterministic)
     torch.cuda.synchronize()
     return out, lse, dq, dk, dv, ds
 

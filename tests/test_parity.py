@@ -130,12 +130,13 @@ BWD_CASES = [
 ]
 
 
+@pytest.mark.parametrize("deterministic", [False, True], ids=["atomic_dq", "deterministic"])
 @pytest.mark.parametrize("case", BWD_CASES, ids=[c[0] for c in BWD_CASES])
-def test_bwd_matches_oracle(case):
+def test_bwd_matches_oracle(case, deterministic):
     name, lq, lk, hq, hkv, dk, dv, causal, wl, wr, sink, dtype = case
     p = W.random_problem(_seed(name) + 7, lq, lk, hq, hkv, dk, dv, causal, wl, wr, sink,
                          dtype, with_dout=True)
-    out, lse, dq, dk_, dv_, ds = run_bwd(p)
+    out, lse, dq, dk_, dv_, ds = run_bwd(p, deterministic)
     a = (p.cu_seqlens_q, p.cu_seqlens_k, p.sink, p.softmax_scale, p.causal, wl, wr)
     rdq, rdk, rdv, rds = ref.bwd(p.q, p.k, p.v, p.dout, *a)
     check_grad(to_np(dq), rdq, dtype, "dq")
@@ -150,6 +151,22 @@ def test_bwd_fully_masked_rows_have_zero_dq():
     out, lse, dq, dk, dv, ds = run_bwd(p)
     assert np.all(to_np(dq)[[0, 1, 2, 5, 6, 7]] == 0.0)
     assert np.all(np.isfinite(to_np(ds)))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_bwd_deterministic_is_bitwise_repeatable(dtype):
+    """The deterministic backward gives the same bits on every run (dq summed over 7 key
+    tiles in a fixed order, GQA heads, a sink); its results match the atomic path within
+    the gradient tolerance."""
+    p = W.random_problem(31, [900, 300], [900, 300], 8, 2, 128, 128, True, dtype=dtype, with_dout=True)
+    runs = [run_bwd(p, True) for _ in range(3)]
+    for name, idx in (("dq", 2), ("dk", 3), ("dv", 4), ("dsink", 5)):
+        first = to_np(runs[0][idx])
+        for r in runs[1:]:
+            assert np.array_equal(first, to_np(r[idx])), f"{name} differs between runs"
+    fast = run_bwd(p, False)
+    check_grad(to_np(runs[0][2]), to_np(fast[2]), dtype, "dq vs atomic dq")
+
 
 
 DECODE_CASES = [
