@@ -223,10 +223,24 @@ const char* attn_sink_status_string(int status);
 /*
  * Synchronises `stream`, then reads and clears the calling device's status word.
  * Returns ATTN_SINK_OK, ATTN_SINK_ERR_TIMEOUT (a bounded wait ran out; bit 0),
- * ATTN_SINK_ERR_BAD_INDEX (an index or length outside its table was skipped; bit 1) or
- * ATTN_SINK_ERR_CUDA.  *bits (if not NULL) receives the raw word.
+ * ATTN_SINK_ERR_BAD_INDEX (an index or length outside its table was skipped, bit 1, or
+ * attn_sink_check_seqlens found a broken cu_seqlens, bit 2) or ATTN_SINK_ERR_CUDA.  *bits
+ * (if not NULL) receives the raw word.
  */
 int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits);
+
+/*
+ * Debug check of the cu_seqlens contract, which the other entry points take on trust (the
+ * CANN doc leaves invalid values undefined; "SeqLengths Parameter Group"): both arrays
+ * start at 0, never decrease and end at total_q / total_k, and no sequence is longer than
+ * max_seqlen_q / max_seqlen_k.  cu_seqlens_q may be NULL (decode).  One small kernel on
+ * `stream`, asynchronous; a violation sets the device status, which
+ * attn_sink_get_device_status() then reports as ATTN_SINK_ERR_BAD_INDEX (bit 2).  Returns
+ * ATTN_SINK_ERR_INVALID_ARG for a NULL params / cu_seqlens_k or batch <= 0, else the launch
+ * status.
+ */
+int attn_sink_check_seqlens(const attn_sink_params* params, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, attn_sink_stream_t stream);
 
 /*
  * Diagnostics, with no counterpart on the pages: launches a one-thread kernel whose bounded

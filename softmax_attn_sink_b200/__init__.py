@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.attn_sink_status_string.restype = ctypes.c_char_p
         L.attn_sink_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.attn_sink_get_device_status.restype = i32
+        L.attn_sink_check_seqlens.argtypes = [P, vp, vp, vp]
+        L.attn_sink_check_seqlens.restype = i32
         L.attn_sink_selftest_wait_timeout.argtypes = [vp]
         L.attn_sink_selftest_wait_timeout.restype = i32
         L.attn_sink_version.argtypes = []
@@ -320,6 +322,22 @@ def device_status(stream=None) -> Tuple[int, int]:
     return int(st), int(bits.value)
 
 
+def check_seqlens(cu_seqlens_q, cu_seqlens_k, total_q: int, total_k: int, max_seqlen_q: int,
+                  max_seqlen_k: int, stream=None) -> Tuple[int, int]:
+    """Check the cu_seqlens contract on the device (cu_seqlens_q may be None), then read and
+    clear the device status: (status, raw bits); status 6 means a broken contract."""
+    torch = _torch()
+    _require(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    if cu_seqlens_q is not None:
+        _require(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    p = make_params(batch=cu_seqlens_k.shape[0] - 1, total_q=total_q, total_k=total_k,
+                    max_seqlen_q=max_seqlen_q, max_seqlen_k=max_seqlen_k, num_heads_q=1, num_heads_kv=1,
+                    head_dim_qk=128, head_dim_v=128, softmax_scale=1.0)
+    _check("attn_sink_check_seqlens", lib().attn_sink_check_seqlens(
+        ctypes.byref(p), _ptr(cu_seqlens_q), cu_seqlens_k.data_ptr(), _stream(stream)))
+    return device_status(stream)
+
+
 def selftest_wait_timeout(stream=None) -> None:
     """Launch the diagnostics kernel whose bounded wait runs out (about 2 s)."""
     _check("attn_sink_selftest_wait_timeout", lib().attn_sink_selftest_wait_timeout(_stream(stream)))
@@ -360,5 +378,6 @@ class SinkAttention:
 
 
 __all__ = ["attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "attn_sink_decode_paged", "decode_num_splits",
+           "check_seqlens",
            "device_status", "selftest_wait_timeout", "SinkAttention", "AttnSinkError", "AttnSinkParams", "make_params",
            "lib", "LIB_PATH", "ATTN_SINK_BF16", "ATTN_SINK_FP32", "ATTN_SINK_FP16"]

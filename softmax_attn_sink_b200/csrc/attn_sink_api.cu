@@ -333,4 +333,13 @@ int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits) {
   return host ? ATTN_SINK_ERR_BAD_INDEX : ATTN_SINK_OK;
 }
 
+int attn_sink_check_seqlens(const attn_sink_params* p, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            attn_sink_stream_t stream) {
+  if (!p || !cu_seqlens_k || p->batch <= 0) return ATTN_SINK_ERR_INVALID_ARG;
+  unsigned* sp = status_ptr();
+  if (!sp) return ATTN_SINK_ERR_CUDA;
+  return from_cuda(launch_check_seqlens(cu_seqlens_q, cu_seqlens_k, p->batch, p->total_q, p->total_k,
+                                        p->max_seqlen_q, p->max_seqlen_k, sp, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -14,6 +14,7 @@ constexpr int kUnbounded = 1 << 30;
 // Bits of the per-device status word.
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBadIndex = 2u;  // a paged block id or key count outside its table
+constexpr unsigned kStatusBadSeqlens = 4u;  // cu_seqlens broke its contract (attn_sink_check_seqlens)
 
 struct FwdArgs {
   const void* q;
@@ -91,6 +92,9 @@ cudaError_t launch_bwd_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
 // Query-stationary dQ without atomics (the deterministic backward's dQ pass).
 bool bwd_dq_sm100_supported(const BwdArgs& a, int dtype);
 cudaError_t launch_bwd_dq_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
+// Contract check of cu_seqlens_q (may be nullptr) and cu_seqlens_k; sets kStatusBadSeqlens.
+cudaError_t launch_check_seqlens(const int32_t* cu_q, const int32_t* cu_k, int batch, int total_q, int total_k,
+                                 int max_sq, int max_sk, unsigned* status, cudaStream_t s);
 // d_sink from the preprocess pass's per-block partials, summed in a fixed order.
 cudaError_t launch_dsink_reduce(const BwdArgs& a, cudaStream_t s);
 

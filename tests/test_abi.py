@@ -133,3 +133,9 @@ def test_paged_decode_rejects_bad_arguments_on_host(change, status):
                                           a["num_blocks"], a["block_size"], a["max_blocks"], None, 0,
                                           fake, None, fake, 1 << 20, None)
     assert st == status
+
+
+def test_check_seqlens_rejects_null_arrays_on_host():
+    p = _params()
+    assert sab.lib().attn_sink_check_seqlens(ctypes.byref(p), None, None, None) == 1
+    assert sab.lib().attn_sink_check_seqlens(None, None, 4096, None) == 1
