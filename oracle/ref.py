@@ -33,6 +33,11 @@ Sources, by page and section:
 * Decode split + LSE merge -- CANN doc, the ``softmax_lse`` note (partial results of
   ring attention are combined through max / sum / log); the sink enters once, after
   the partials are combined.
+* Dropout -- slime wrapper (``dropout_p`` passed to flash attention, whose probabilities
+  are then scaled by sigmoid(lse - offset)): dropout applies to the sink-normalised
+  probabilities, kept ones scaled so the expectation is unchanged, lse untouched.  The keep
+  decisions come from Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
+  As Easy as 1, 2, 3", SC 2011), on the counter layout ``dropout_keep`` defines.
 * Paged K/V -- CANN doc, "Paged Attention Parameter Group" (block_table (B,
   max_num_blocks_per_seq) int32, block_size in [16, 1024] and a multiple of 16, seqused_kv)
   and the PA_BBND layout of k / v, (num_blocks, block_size, KV_N, D).
@@ -72,10 +77,12 @@ def allowed_mask(sq: int, sk: int, causal: bool, window_left: int = -1,
     return (j <= i + off + right) & (j >= i + off - left)
 
 
-def attend_head(qh, kh, vh, sink_h: float, scale: float, allowed: np.ndarray) -> Dict[str, np.ndarray]:
+def attend_head(qh, kh, vh, sink_h: float, scale: float, allowed: np.ndarray,
+                drop: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Forward of one (sequence, head): the CANN sink formula, written out.
 
-    qh [sq, dk], kh [sk, dk], vh [sk, dv]; sink_h a float (may be -inf).
+    qh [sq, dk], kh [sk, dk], vh [sk, dv]; sink_h a float (may be -inf).  drop, when given,
+    is the dropout weight Z [sq, sk] (keep mask x 256 / T): out = (P o Z) V.
     Returns out [sq, dv], lse [sq] (vanilla: sink excluded), P [sq, sk],
     p_sink [sq] (the probability the sink column takes), S [sq, sk].
     """
@@ -94,13 +101,58 @@ def attend_head(qh, kh, vh, sink_h: float, scale: float, allowed: np.ndarray) ->
     inv = np.where(den > 0, 1.0 / np.where(den > 0, den, 1.0), 0.0)
     P = E * inv[:, None]
     p_sink = e_sink * inv
-    out = P @ vh
+    out = (P if drop is None else P * drop) @ vh
     # vanilla lse: log sum_j e^{S_j - max S} + max S over the visible keys
     with np.errstate(divide="ignore", invalid="ignore"):
         smax_ref = np.where(np.isfinite(smax), smax, 0.0)
         z = np.exp(S_vis - smax_ref[:, None]).sum(axis=1)
         lse = np.where(np.isfinite(smax), np.log(z) + smax_ref, NEG_INF)
     return {"out": out, "lse": lse, "P": P, "p_sink": p_sink, "S": S}
+
+
+# --- dropout --------------------------------------------------------------------------
+
+PHILOX_M = (0xD2511F53, 0xCD9E8D57)   # round multipliers of Philox4x32 (Salmon et al. 2011)
+PHILOX_W = (0x9E3779B9, 0xBB67AE85)   # key increments (Weyl sequence) of Philox4x32
+_U32 = np.uint64(0xFFFFFFFF)
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32 with 10 rounds on numpy arrays of 32-bit values (held as uint64).
+    ctr: 4 arrays (or ints), key: 2 arrays (or ints); returns the 4 output words."""
+    c = [np.asarray(x, dtype=np.uint64) & _U32 for x in ctr]
+    k = [np.asarray(x, dtype=np.uint64) & _U32 for x in key]
+    for _ in range(10):
+        p0 = np.uint64(PHILOX_M[0]) * c[0]
+        p1 = np.uint64(PHILOX_M[1]) * c[2]
+        hi0, lo0 = p0 >> np.uint64(32), p0 & _U32
+        hi1, lo1 = p1 >> np.uint64(32), p1 & _U32
+        c = [hi1 ^ c[1] ^ k[0], lo1, hi0 ^ c[3] ^ k[1], lo0]
+        k = [(k[0] + np.uint64(PHILOX_W[0])) & _U32, (k[1] + np.uint64(PHILOX_W[1])) & _U32]
+    return c
+
+
+def dropout_threshold(p: float) -> int:
+    """Keep threshold T: an element is kept when its random byte is below T, so the keep
+    probability is T / 256 (T = round(256 (1 - p)), 1 <= T <= 256)."""
+    t = int(round(256.0 * (1.0 - float(p))))
+    if not 1 <= t <= 256:
+        raise ValueError("dropout p must satisfy 1 <= round(256 (1 - p)) <= 256")
+    return t
+
+
+def dropout_keep(seed: int, offset: int, threshold: int, rows, head: int, nkeys: int) -> np.ndarray:
+    """Keep mask [len(rows), nkeys] of query rows `rows` (packed row indices) of q head
+    `head` against keys 0 .. nkeys-1 of their sequence.  Key j of row r uses byte j % 16 of
+    Philox4x32-10 with counter (j // 16, r, head, offset) and key (seed low 32 bits, seed
+    high 32 bits); byte t is bits 8 (t % 4) .. 8 (t % 4) + 7 of output word t // 4."""
+    rows = np.asarray(rows, dtype=np.uint64)[:, None]
+    j = np.arange(nkeys, dtype=np.uint64)[None, :]
+    words = philox4x32_10((j >> np.uint64(4), rows, head, offset), (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
+    t = j & np.uint64(15)
+    w = np.choose((t >> np.uint64(2)).astype(np.int64), [np.broadcast_to(x, np.broadcast(rows, j).shape) for x in words])
+    byte = (w >> (np.uint64(8) * (t & np.uint64(3)))) & np.uint64(0xFF)
+    return byte < np.uint64(threshold)
 
 
 def _sink_of(sink: Optional[np.ndarray], h: int) -> float:
@@ -111,9 +163,21 @@ def _seq_ranges(cu: np.ndarray, b: int) -> Tuple[int, int]:
     return int(cu[b]), int(cu[b + 1])
 
 
+def _drop_weights(dropout, q0: int, q1: int, h: int, nkeys: int) -> Optional[np.ndarray]:
+    """Dropout weights Z [q1 - q0, nkeys] (keep x 256 / T) of rows q0 .. q1-1 of head h, or
+    None without dropout.  dropout = (p, seed, offset)."""
+    if dropout is None:
+        return None
+    p, seed, offset = dropout
+    t = dropout_threshold(p)
+    keep = dropout_keep(seed, offset, t, np.arange(q0, q1), h, nkeys)
+    return keep * (256.0 / t)
+
+
 def fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, sink, softmax_scale: float, causal: bool = False,
-        window_left: int = -1, window_right: int = -1) -> Tuple[np.ndarray, np.ndarray]:
+        window_left: int = -1, window_right: int = -1, dropout=None) -> Tuple[np.ndarray, np.ndarray]:
     """Packed THD forward.  q [T_q,Hq,dk], k [T_k,Hkv,dk], v [T_k,Hkv,dv], sink [Hq] or None.
+    dropout = (p, seed, offset) or None.
 
     Returns out [T_q, Hq, dv] float64 and lse [Hq, T_q] float64 (vanilla lse).
     """
@@ -131,37 +195,45 @@ def fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, sink, softmax_scale: float, causal:
         mask = allowed_mask(q1 - q0, k1 - k0, causal, window_left, window_right)
         for h in range(hq):
             r = attend_head(q[q0:q1, h], k[k0:k1, h // group], v[k0:k1, h // group],
-                            _sink_of(sink, h), softmax_scale, mask)
+                            _sink_of(sink, h), softmax_scale, mask,
+                            _drop_weights(dropout, q0, q1, h, k1 - k0))
             out[q0:q1, h] = r["out"]
             lse[h, q0:q1] = r["lse"]
     return out, lse
 
 
-def bwd_head(qh, kh, vh, dout_h, sink_h: float, scale: float, allowed: np.ndarray) -> Dict[str, np.ndarray]:
+def bwd_head(qh, kh, vh, dout_h, sink_h: float, scale: float, allowed: np.ndarray,
+             drop: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Gradients of one (sequence, head) for the loss sum(dout * out).
 
     With P the sink-normalised probabilities and p_sink the sink's share of each row:
       dP = dO V^T,  D_i = dO_i . out_i,  dS = P * (dP - D),
       dq = scale dS K,  dk = scale dS^T Q,  dv = P^T dO,  d_sink = -sum_i p_sink_i D_i.
+    With dropout weights Z (out = (P o Z) V): dP = Z o (dO V^T) and dv = (P o Z)^T dO; D and
+    the rest are unchanged (D = dO . out still equals sum_j P_ij dP_ij).
     """
-    r = attend_head(qh, kh, vh, sink_h, scale, allowed)
+    r = attend_head(qh, kh, vh, sink_h, scale, allowed, drop)
     qh, kh, vh, do = _f64(qh), _f64(kh), _f64(vh), _f64(dout_h)
     P, out = r["P"], r["out"]
+    PZ = P if drop is None else P * drop
     dP = do @ vh.T
+    if drop is not None:
+        dP = dP * drop
     D = (do * out).sum(axis=1)
     dS = P * (dP - D[:, None])
     return {
         "dq": float(scale) * (dS @ kh),
         "dk": float(scale) * (dS.T @ qh),
-        "dv": P.T @ do,
+        "dv": PZ.T @ do,
         "dsink": -float((r["p_sink"] * D).sum()),
         "D": D, "out": out, "lse": r["lse"],
     }
 
 
 def bwd(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, sink, softmax_scale: float,
-        causal: bool = False, window_left: int = -1, window_right: int = -1):
+        causal: bool = False, window_left: int = -1, window_right: int = -1, dropout=None):
     """Packed THD backward.  Returns dq, dk, dv (float64, input layouts) and dsink [Hq].
+    dropout = (p, seed, offset) or None (the forward's keep decisions are drawn again).
 
     dk / dv of a kv head sum the contributions of the q heads of its group.
     """
@@ -179,7 +251,8 @@ def bwd(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, sink, softmax_scale: float,
         for h in range(hq):
             g = h // group
             r = bwd_head(q[q0:q1, h], k[k0:k1, g], v[k0:k1, g], dout[q0:q1, h],
-                         _sink_of(sink, h), softmax_scale, mask)
+                         _sink_of(sink, h), softmax_scale, mask,
+                         _drop_weights(dropout, q0, q1, h, k1 - k0))
             dq[q0:q1, h] = r["dq"]
             dk[k0:k1, g] += r["dk"]
             dv[k0:k1, g] += r["dv"]

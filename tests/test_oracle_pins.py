@@ -497,3 +497,79 @@ def test_fp16_rounding_matches_torch():
     x = np.random.default_rng(3).standard_normal(10000).astype(np.float32) * 100
     x[:4] = [65504.0, 1e-8, -2.0 ** -24 * 1.5, 0.5 + 2.0 ** -12]
     assert np.array_equal(W.fp16_round(x), torch.from_numpy(x).to(torch.float16).float().numpy())
+
+
+# --- P14: dropout (Philox4x32-10; slime wrapper's dropout_p) ------------------------------
+
+def test_p14_philox_known_answers():
+    """The oracle's Philox4x32-10 reproduces the published known-answer vectors."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "philox4x32_10_kat.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert len(rows) == 3
+    for r in rows:
+        v = [int(x, 16) for x in r]
+        got = [int(x) for x in ref.philox4x32_10(v[0:4], v[4:6])]
+        assert got == v[6:10]
+
+
+def test_p14_keep_rate_and_threshold():
+    """Bytes below T are kept: over 2^18 decisions the kept share is T/256 within 4 sigma,
+    and T = 256 keeps everything."""
+    for p in (0.1, 0.5, 0.9):
+        t = ref.dropout_threshold(p)
+        keep = ref.dropout_keep(2024, 3, t, np.arange(256), 5, 1024)
+        q = t / 256.0
+        sigma = math.sqrt(q * (1 - q) / keep.size)
+        assert abs(keep.mean() - q) < 4 * sigma
+    assert ref.dropout_keep(1, 0, 256, np.arange(8), 0, 100).all()
+    with pytest.raises(ValueError):
+        ref.dropout_threshold(0.999)
+
+
+def test_p14_no_dropout_is_identity():
+    """p = 0 (T = 256) gives exactly the forward and backward without dropout."""
+    p = W.random_problem(140, [9, 5], [11, 5], 4, 2, 8, 6, True, dtype="fp32", with_dout=True)
+    a = (p.cu_seqlens_q, p.cu_seqlens_k, p.sink, p.softmax_scale, True)
+    o1, l1 = ref.fwd(p.q, p.k, p.v, *a)
+    o2, l2 = ref.fwd(p.q, p.k, p.v, *a, dropout=(0.0, 9, 1))
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    g1 = ref.bwd(p.q, p.k, p.v, p.dout, *a)
+    g2 = ref.bwd(p.q, p.k, p.v, p.dout, *a, dropout=(0.0, 9, 1))
+    for x, y in zip(g1, g2):
+        assert np.array_equal(x, y)
+
+
+def test_p14_dropout_gradients_match_finite_differences():
+    """With the keep decisions fixed (they depend on positions, seed and offset only), the
+    dropout backward is the exact gradient of the dropout forward: central differences in
+    fp64 for q, k, v and the sink."""
+    p = W.random_problem(141, [6, 4], [7, 4], 4, 2, 4, 3, True, window_left=4, dtype="fp32", with_dout=True)
+    drop = (0.3, 77, 5)
+    a = (p.cu_seqlens_q, p.cu_seqlens_k)
+    loss = lambda q, k, v, s: float((ref.fwd(q, k, v, *a, s, p.softmax_scale, True, 4, -1, drop)[0] * p.dout).sum())
+    dq, dk, dv, ds = ref.bwd(p.q, p.k, p.v, p.dout, *a, p.sink, p.softmax_scale, True, 4, -1, drop)
+    base = [p.q.astype(np.float64), p.k.astype(np.float64), p.v.astype(np.float64), p.sink.astype(np.float64)]
+    h = 1e-6
+    for which, grad in enumerate((dq, dk, dv, ds)):
+        x = base[which]
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [xp if i == which else base[i] for i in range(4)]
+            args_m = [xm if i == which else base[i] for i in range(4)]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        err = np.abs(num - grad).max() / max(1e-12, np.abs(grad).max())
+        assert err < 1e-6, (which, err)
+
+
+def test_p14_dropout_is_unbiased_on_average():
+    """Averaged over seeds, the dropout output approaches the output without dropout."""
+    p = W.random_problem(142, [8], [8], 2, 2, 4, 4, True, dtype="fp32")
+    a = (p.cu_seqlens_q, p.cu_seqlens_k, p.sink, p.softmax_scale, True)
+    o_ref, _ = ref.fwd(p.q, p.k, p.v, *a)
+    n = 400
+    outs = np.stack([ref.fwd(p.q, p.k, p.v, *a, dropout=(0.5, 1000 + s, 0))[0] for s in range(n)])
+    se = outs.std(axis=0) / math.sqrt(n)          # standard error of each element's mean
+    assert np.all(np.abs(outs.mean(axis=0) - o_ref) <= 5 * se + 1e-12)
