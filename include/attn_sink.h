@@ -101,6 +101,23 @@ typedef struct {
 typedef void* attn_sink_stream_t;
 
 /*
+ * Dropout on the attention probabilities (slime wrapper's `dropout_p`, which it passes to
+ * flash attention before the sigmoid(lse - offset) scaling, i.e. dropout acts on the
+ * sink-normalised probabilities).  Key j of packed query row r and q head h is kept when
+ * byte j % 16 of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+ * Easy as 1, 2, 3", SC 2011) with counter (j / 16, r, h, offset) and key (seed low 32 bits,
+ * seed high 32 bits) is below T = round(256 (1 - p)); byte t is bits 8 (t % 4) .. +7 of
+ * output word t / 4.  Kept probabilities are scaled by 256 / T (keep probability T / 256),
+ * so the output's expectation is the output without dropout; lse is not affected.
+ * 1 <= T <= 256 is required (0 <= p < 1 - 1/512).  The backward draws the same decisions.
+ */
+typedef struct {
+  float p;          /* dropout probability                                          */
+  uint64_t seed;    /* Philox key                                                   */
+  uint32_t offset;  /* fourth counter word, e.g. a step counter for fresh masks     */
+} attn_sink_dropout;
+
+/*
  * Forward (CANN doc, "Function" formula and softmax_lse formula; slime
  * learnable_softmax_flash_attn_varlen).  Writes out [total_q, Hq, dv] (dtype) and, when
  * `lse` is not NULL, lse [Hq, total_q] fp32.  sink may be NULL (= -inf).  The workspace
@@ -125,6 +142,24 @@ int attn_sink_bwd(const attn_sink_params* params, const void* q, const void* k, 
                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
                   void* dq, void* dk, void* dv, float* dsink, void* workspace,
                   size_t workspace_bytes, attn_sink_stream_t stream);
+
+/*
+ * Forward and backward with dropout (see attn_sink_dropout); otherwise the arguments of
+ * attn_sink_fwd / attn_sink_bwd.  Tensor-core paths only: bf16 or fp16, and for the
+ * backward head_dim_qk == 128 with head_dim_v in {64, 128} (ATTN_SINK_ERR_UNSUPPORTED
+ * otherwise; ATTN_SINK_ERR_INVALID_ARG for a NULL dropout or p out of range).  The backward
+ * takes the deterministic path (bit-identical results from run to run) and the workspace
+ * attn_sink_bwd_workspace_size() gives.
+ */
+int attn_sink_fwd_dropout(const attn_sink_params* params, const void* q, const void* k,
+                          const void* v, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                          const float* sink, const attn_sink_dropout* dropout, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, attn_sink_stream_t stream);
+int attn_sink_bwd_dropout(const attn_sink_params* params, const void* q, const void* k,
+                          const void* v, const void* out, const void* dout, const float* lse,
+                          const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
+                          const attn_sink_dropout* dropout, void* dq, void* dk, void* dv, float* dsink,
+                          void* workspace, size_t workspace_bytes, attn_sink_stream_t stream);
 
 /*
  * Deterministic backward: the same arguments, results and workspace size as

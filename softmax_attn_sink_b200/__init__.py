@@ -45,6 +45,20 @@ class AttnSinkParams(ctypes.Structure):
                 ("dtype", ctypes.c_int)]
 
 
+class AttnSinkDropout(ctypes.Structure):
+    """Mirror of ``attn_sink_dropout`` (include/attn_sink.h)."""
+
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint32)]
+
+
+def _dropout(dropout):
+    """(p, seed, offset) -> AttnSinkDropout, or None."""
+    if dropout is None:
+        return None
+    p, seed, offset = dropout
+    return AttnSinkDropout(float(p), int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFF)
+
+
 class AttnSinkError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
@@ -69,6 +83,11 @@ def lib() -> ctypes.CDLL:
         L.attn_sink_decode.argtypes = [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]
         L.attn_sink_bwd_deterministic.argtypes = list(L.attn_sink_bwd.argtypes)
         L.attn_sink_bwd_deterministic.restype = i32
+        D = ctypes.POINTER(AttnSinkDropout)
+        L.attn_sink_fwd_dropout.argtypes = [P, vp, vp, vp, vp, vp, vp, D, vp, vp, vp, sz, vp]
+        L.attn_sink_fwd_dropout.restype = i32
+        L.attn_sink_bwd_dropout.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, D, vp, vp, vp, vp, vp, sz, vp]
+        L.attn_sink_bwd_dropout.restype = i32
         L.attn_sink_decode_paged.argtypes = [P, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, sz, vp]
         for f in (L.attn_sink_fwd, L.attn_sink_bwd, L.attn_sink_decode, L.attn_sink_decode_paged):
             f.restype = i32
@@ -177,8 +196,9 @@ def _common(q, k, v, cu_seqlens_q, cu_seqlens_k, sink, max_seqlen_q, max_seqlen_
 def attn_sink_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                   sink=None, softmax_scale: Optional[float] = None, causal: bool = False,
                   window_size: Sequence[int] = (-1, -1), out=None, lse=None, return_lse=True,
-                  stream=None):
-    """Sink-attention forward on packed THD tensors.  Returns (out, lse).
+                  stream=None, dropout=None):
+    """Sink-attention forward on packed THD tensors.  Returns (out, lse).  dropout, when
+    given, is (p, seed, offset) (tensor-core path; see attn_sink_dropout).
 
     q [T_q, Hq, dk], k [T_k, Hkv, dk], v [T_k, Hkv, dv] (bf16 or fp32, CUDA, contiguous);
     cu_seqlens_q / cu_seqlens_k int32 [B + 1]; sink fp32 [Hq] or None (= -inf);
@@ -196,19 +216,28 @@ def attn_sink_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_se
     if ws_bytes == ctypes.c_size_t(-1).value:
         raise AttnSinkError("attn_sink_fwd_workspace_size", 1)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device) if ws_bytes else None
-    st = lib().attn_sink_fwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                             cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), _ptr(sink),
-                             out.data_ptr(), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
-    _check("attn_sink_fwd", st)
+    if dropout is None:
+        st = lib().attn_sink_fwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                 cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), _ptr(sink),
+                                 out.data_ptr(), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
+        _check("attn_sink_fwd", st)
+    else:
+        d = _dropout(dropout)
+        st = lib().attn_sink_fwd_dropout(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), _ptr(sink),
+                                         ctypes.byref(d), out.data_ptr(), _ptr(lse), _ptr(ws), ws_bytes,
+                                         _stream(stream))
+        _check("attn_sink_fwd_dropout", st)
     return out, lse
 
 
 def attn_sink_bwd(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                   max_seqlen_k: int, sink=None, softmax_scale: Optional[float] = None,
                   causal: bool = False, window_size: Sequence[int] = (-1, -1), dq=None, dk=None,
-                  dv=None, dsink=None, stream=None, deterministic: bool = False):
+                  dv=None, dsink=None, stream=None, deterministic: bool = False, dropout=None):
     """Backward for the loss sum(dout * out).  Returns (dq, dk, dv, dsink).  With
-    deterministic=True the results are bit-identical from run to run (slower)."""
+    deterministic=True the results are bit-identical from run to run (slower).  dropout:
+    the forward's (p, seed, offset) (implies the deterministic path)."""
     torch = _torch()
     p = _common(q, k, v, cu_seqlens_q, cu_seqlens_k, sink, max_seqlen_q, max_seqlen_k,
                 softmax_scale, causal, window_size)
@@ -224,6 +253,15 @@ def attn_sink_bwd(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqle
     if ws_bytes == ctypes.c_size_t(-1).value:
         raise AttnSinkError("attn_sink_bwd_workspace_size", 1)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    if dropout is not None:
+        d = _dropout(dropout)
+        st = lib().attn_sink_bwd_dropout(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                                         cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), _ptr(sink),
+                                         ctypes.byref(d), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                         dsink.data_ptr(), ws.data_ptr(), ws_bytes, _stream(stream))
+        _check("attn_sink_bwd_dropout", st)
+        return dq, dk, dv, dsink
     fn = lib().attn_sink_bwd_deterministic if deterministic else lib().attn_sink_bwd
     st = fn(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(),
             out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
@@ -380,4 +418,4 @@ class SinkAttention:
 __all__ = ["attn_sink_fwd", "attn_sink_bwd", "attn_sink_decode", "attn_sink_decode_paged", "decode_num_splits",
            "check_seqlens",
            "device_status", "selftest_wait_timeout", "SinkAttention", "AttnSinkError", "AttnSinkParams", "make_params",
-           "lib", "LIB_PATH", "ATTN_SINK_BF16", "ATTN_SINK_FP32", "ATTN_SINK_FP16"]
+           "lib", "LIB_PATH", "ATTN_SINK_BF16", "ATTN_SINK_FP32", "ATTN_SINK_FP16", "AttnSinkDropout"]

@@ -125,13 +125,58 @@ int launch_decode(const attn_sink_params* p, DecodeArgs& a, int num_splits, void
   return from_cuda(launch_decode_split(a, p->dtype, s));
 }
 
+// Keep threshold and scale of a dropout request (round(256 (1 - p)) in [1, 256]); false
+// when p is outside that range.
+bool dropout_of(const attn_sink_dropout* d, Dropout& out) {
+  out = Dropout{};
+  if (!d) return true;
+  if (!(d->p >= 0.f) || !isfinite(d->p)) return false;
+  const long t = lroundf(256.f * (1.f - d->p));
+  if (t < 1 || t > 256) return false;
+  out.threshold = (uint32_t)t;
+  out.seed_lo = (uint32_t)(d->seed & 0xFFFFFFFFu);
+  out.seed_hi = (uint32_t)(d->seed >> 32);
+  out.offset = d->offset;
+  out.scale = 256.f / (float)t;
+  return true;
+}
+
+int run_fwd(const attn_sink_params* p, const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+            const int32_t* cu_seqlens_k, const float* sink, const attn_sink_dropout* dropout, void* out, float* lse,
+            void* workspace, size_t workspace_bytes, attn_sink_stream_t stream) {
+  int st = validate_params(p, false);
+  if (st != ATTN_SINK_OK) return st;
+  if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !out) return ATTN_SINK_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
+  if ((lse && !aligned16(lse)) || (sink && !aligned16(sink))) return ATTN_SINK_ERR_INVALID_ARG;
+  (void)workspace;
+  (void)workspace_bytes;
+  FwdArgs a{};
+  if (!dropout_of(dropout, a.drop)) return ATTN_SINK_ERR_INVALID_ARG;
+  a.q = q; a.k = k; a.v = v; a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
+  a.out = out; a.lse = lse;
+  a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
+  a.max_sq = p->max_seqlen_q; a.max_sk = p->max_seqlen_k;
+  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
+  a.scale = p->softmax_scale;
+  effective_window(p, a.left, a.right);
+  a.status = status_ptr();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
+  if (fwd_sm100_supported(a, dt)) return from_cuda(launch_fwd_sm100(a, dt, s));
+  if (a.drop.threshold) return ATTN_SINK_ERR_UNSUPPORTED;   // dropout runs on the tensor-core path only
+  return from_cuda(launch_fwd_simt(a, dt, s));
+}
+
 // The backward, with dQ reduced by fp32 atomics into a workspace accumulator (fast) or, in
 // the deterministic mode, computed by a query-stationary pass that adds the key tiles'
 // contributions in a fixed order.
 int run_bwd(const attn_sink_params* p, const void* q, const void* k, const void* v, const void* out,
             const void* dout, const float* lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
             const float* sink, void* dq, void* dk, void* dv, float* dsink, void* workspace,
-            size_t workspace_bytes, attn_sink_stream_t stream, bool deterministic) {
+            size_t workspace_bytes, attn_sink_stream_t stream, bool deterministic,
+            const attn_sink_dropout* dropout = nullptr) {
   int st = validate_params(p, false);
   if (st != ATTN_SINK_OK) return st;
   if (!q || !k || !v || !out || !dout || !lse || !cu_seqlens_q || !cu_seqlens_k || !dq || !dk || !dv)
@@ -143,6 +188,8 @@ int run_bwd(const attn_sink_params* p, const void* q, const void* k, const void*
   if (!workspace || workspace_bytes < lay.total || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   BwdArgs a{};
+  if (!dropout_of(dropout, a.drop)) return ATTN_SINK_ERR_INVALID_ARG;
+  if (a.drop.threshold) deterministic = true;   // dropout runs on the query-stationary dQ path
   a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.lse = lse;
   a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
   a.grad_q = dq; a.grad_k = dk; a.grad_v = dv; a.dsink = dsink;
@@ -164,7 +211,9 @@ int run_bwd(const attn_sink_params* p, const void* q, const void* k, const void*
   }
   // deterministic: dK / dV on the key-stationary tensor-core kernel without its dQ part,
   // then dQ query-stationary; the CUDA-core path has no atomics to begin with
-  if (bwd_sm100_supported(a, dt) && bwd_dq_sm100_supported(a, dt)) {
+  const bool tc = bwd_sm100_supported(a, dt) && bwd_dq_sm100_supported(a, dt);
+  if (a.drop.threshold && !(tc && a.dk == 128)) return ATTN_SINK_ERR_UNSUPPORTED;   // dropout: d = 128 kernels
+  if (tc) {
     cudaError_t e = launch_bwd_sm100(a, dt, s);
     if (e == cudaSuccess) e = launch_bwd_dq_sm100(a, dt, s);
     return from_cuda(e);
@@ -215,27 +264,17 @@ int attn_sink_fwd(const attn_sink_params* p, const void* q, const void* k, const
                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
                   void* out, float* lse, void* workspace, size_t workspace_bytes,
                   attn_sink_stream_t stream) {
-  int st = validate_params(p, false);
-  if (st != ATTN_SINK_OK) return st;
-  if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !out) return ATTN_SINK_ERR_INVALID_ARG;
-  for (const void* ptr : {q, k, v, (const void*)out})
-    if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
-  if ((lse && !aligned16(lse)) || (sink && !aligned16(sink))) return ATTN_SINK_ERR_INVALID_ARG;
-  (void)workspace;
-  (void)workspace_bytes;
-  FwdArgs a{};
-  a.q = q; a.k = k; a.v = v; a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
-  a.out = out; a.lse = lse;
-  a.batch = p->batch; a.total_q = p->total_q; a.total_k = p->total_k;
-  a.max_sq = p->max_seqlen_q; a.max_sk = p->max_seqlen_k;
-  a.hq = p->num_heads_q; a.hkv = p->num_heads_kv; a.dk = p->head_dim_qk; a.dv = p->head_dim_v;
-  a.scale = p->softmax_scale;
-  effective_window(p, a.left, a.right);
-  a.status = status_ptr();
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
-  if (fwd_sm100_supported(a, dt)) return from_cuda(launch_fwd_sm100(a, dt, s));
-  return from_cuda(launch_fwd_simt(a, dt, s));
+  return run_fwd(p, q, k, v, cu_seqlens_q, cu_seqlens_k, sink, nullptr, out, lse, workspace, workspace_bytes,
+                 stream);
+}
+
+int attn_sink_fwd_dropout(const attn_sink_params* p, const void* q, const void* k, const void* v,
+                          const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
+                          const attn_sink_dropout* dropout, void* out, float* lse, void* workspace,
+                          size_t workspace_bytes, attn_sink_stream_t stream) {
+  if (!dropout) return ATTN_SINK_ERR_INVALID_ARG;
+  return run_fwd(p, q, k, v, cu_seqlens_q, cu_seqlens_k, sink, dropout, out, lse, workspace, workspace_bytes,
+                 stream);
 }
 
 
@@ -255,6 +294,16 @@ int attn_sink_bwd_deterministic(const attn_sink_params* p, const void* q, const 
                                 size_t workspace_bytes, attn_sink_stream_t stream) {
   return run_bwd(p, q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, sink, dq, dk, dv, dsink, workspace,
                  workspace_bytes, stream, true);
+}
+
+int attn_sink_bwd_dropout(const attn_sink_params* p, const void* q, const void* k, const void* v,
+                          const void* out, const void* dout, const float* lse, const int32_t* cu_seqlens_q,
+                          const int32_t* cu_seqlens_k, const float* sink, const attn_sink_dropout* dropout,
+                          void* dq, void* dk, void* dv, float* dsink, void* workspace, size_t workspace_bytes,
+                          attn_sink_stream_t stream) {
+  if (!dropout) return ATTN_SINK_ERR_INVALID_ARG;
+  return run_bwd(p, q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, sink, dq, dk, dv, dsink, workspace,
+                 workspace_bytes, stream, true, dropout);
 }
 
 int attn_sink_decode(const attn_sink_params* p, const void* q, const void* k, const void* v,

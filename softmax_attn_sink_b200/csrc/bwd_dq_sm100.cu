@@ -81,7 +81,7 @@ __device__ __forceinline__ void dq_tile_of(const BwdArgs& a, int mtiles, int& m,
   h = rem - b * a.hq;
 }
 
-template <typename Elem, int DK, int DV>
+template <typename Elem, int DK, int DV, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -101,6 +101,7 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
   row_key_range(m0, sq, sk, a.left, a.right, lo, hi);
   row_key_range(m0 + nrows - 1, sq, sk, a.left, a.right, l2, h2);
   hi = h2 > lo ? h2 : lo;   // key ranges move right with the row: the union is [lo(first), hi(last))
+  if (DROP && hi > lo) lo &= ~15LL;   // dropout draws keep bytes for 16-key blocks
   const int n = hi > lo ? (int)((hi - lo + kBN - 1) / kBN) : 0;
 
   const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -244,11 +245,27 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (c < klo || c >= khi) sv[c] = __float_as_uint(kNegInf);
         }
         uint32_t pk[32];
+        // dropout: dS = P (Z dP - D) with Z = 256 / T for kept keys and 0 otherwise, the keep
+        // bytes drawn as in the forward
+        uint4 kb4[DROP ? 4 : 1];
+        if constexpr (DROP) {
+          const uint32_t kb0 = (uint32_t)(lo + (long long)j * kBN + hh * 64) >> 4;
+#pragma unroll
+          for (int gq = 0; gq < 4; ++gq) kb4[gq] = dropout_bytes(a.drop, kb0 + gq, (uint32_t)(q0 + i), (uint32_t)h);
+        }
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), scale2, neg_lt));
           const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), scale2, neg_lt));
-          pk[c] = pack2<Elem>(p0 * (__uint_as_float(pv[2 * c]) - Dr), p1 * (__uint_as_float(pv[2 * c + 1]) - Dr));
+          float dp0 = __uint_as_float(pv[2 * c]), dp1 = __uint_as_float(pv[2 * c + 1]);
+          if constexpr (DROP) {
+            const uint4 w4 = kb4[c >> 3];
+            const int t = (2 * c) & 15;
+            const uint32_t w = (t >> 2) == 0 ? w4.x : (t >> 2) == 1 ? w4.y : (t >> 2) == 2 ? w4.z : w4.w;
+            dp0 = ((w >> (8 * (t & 3))) & 0xFFu) < a.drop.threshold ? dp0 * a.drop.scale : 0.f;
+            dp1 = ((w >> (8 * (t & 3) + 8)) & 0xFFu) < a.drop.threshold ? dp1 * a.drop.scale : 0.f;
+          }
+          pk[c] = pack2<Elem>(p0 * (dp0 - Dr), p1 * (dp1 - Dr));
         }
         // dS of keys [64 hh, 64 hh + 64) over S columns [32 hh, 32 hh + 32): half 0 goes over
         // S columns already read, half 1 over half 0's S columns
@@ -335,11 +352,11 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
       !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
     return cudaErrorInvalidValue;
-  cudaError_t e =
-      cudaFuncSetAttribute(bwd_dq_sm100_kernel<Elem, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  auto kernel = a.drop.threshold ? bwd_dq_sm100_kernel<Elem, DK, DV, true> : bwd_dq_sm100_kernel<Elem, DK, DV, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   const long long ctas = (long long)((a.max_sq + kBM - 1) / kBM) * a.batch * a.hq;
-  bwd_dq_sm100_kernel<Elem, DK, DV><<<(unsigned)ctas, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
+  kernel<<<(unsigned)ctas, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
   return cudaGetLastError();
 }
 

@@ -436,7 +436,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <typename Elem, int DV, bool DQ>
+template <typename Elem, int DV, bool DQ, bool DROP>
 __global__ void __launch_bounds__(kThreadsP, 1)
 bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -643,16 +643,56 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       named_bar_sync(1, 128);
       if (t + 1 < T) prefetch(t + 1);   // in flight while this tile is computed
 #pragma unroll 1
-      for (int hh = 0; hh < 2 && ok; ++hh) {
+      for (int hh = 0; hh < 2; ++hh) {
         const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar.sdp_full(hh), t & 1, a.status))) { ok = false; break; }
-        if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar.ds_free(hh), (t - 1) & 1, a.status))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // every (key, query) pair of this half visible?  (then skip the per-element mask)
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar.sdp_full(hh), t & 1, a.status));
+        if (ok && t >= 1) ok = __all_sync(0xffffffffu, mbar_wait(bar.ds_free(hh), (t - 1) & 1, a.status));
+        if (ok) tc_fence_after();
         const long long qa = i0 + 64 * hh;
+        // Dropout keep bytes of this thread's key for the half's 64 queries.  A Philox call
+        // gives the bytes of 16 keys for one query, so the 16 threads of a 16-key block share
+        // the block's 64 calls (4 each) and swap bytes through the (still free) dS staging
+        // area of this half: word [block][key t][u] holds, in byte k, the keep byte of query
+        // u + 16 k for key t.  Both barriers are passed by every compute warp, also after a
+        // timed-out wait (ok = false), like the named barriers of the tile loop.
+        uint32_t zb[DROP ? 16 : 1];
+        if constexpr (DROP) {
+          const uint32_t stage = sDS + hh * L::kHalf;
+          const int blk = r >> 4, u = r & 15;
+          constexpr int kBlockWords = 16 * 16 + 16;   // + 16 words: blocks 2w, 2w+1 in other banks
+          if (ok) {
+            const uint32_t kb = (uint32_t)((n0 >> 4) + blk);
+            uint4 w[4];
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4)
+              w[s4] = dropout_bytes(a.drop, kb, (uint32_t)(q0 + qa + u + 16 * s4), (uint32_t)h);
+#pragma unroll
+            for (int tk = 0; tk < 16; ++tk) {
+              auto word_of = [&](const uint4& x) {
+                return (tk >> 2) == 0 ? x.x : (tk >> 2) == 1 ? x.y : (tk >> 2) == 2 ? x.z : x.w;
+              };
+              const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
+              const uint32_t lo2 = __byte_perm(word_of(w[0]), word_of(w[1]), sel);
+              const uint32_t hi2 = __byte_perm(word_of(w[2]), word_of(w[3]), sel);
+              const uint32_t word = __byte_perm(lo2, hi2, 0x5410);
+              asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage + 4u * (blk * kBlockWords + tk * 16 + u)), "r"(word)
+                           : "memory");
+            }
+          }
+          named_bar_sync(2, 128);
+          if (ok) {
+            const uint32_t src = stage + 4u * (blk * kBlockWords + (r & 15) * 16);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(zb[4 * v4]), "=r"(zb[4 * v4 + 1]), "=r"(zb[4 * v4 + 2]), "=r"(zb[4 * v4 + 3])
+                           : "r"(src + 16u * v4)
+                           : "memory");
+          }
+          named_bar_sync(2, 128);   // every thread has its bytes before dS overwrites the area
+        }
+        if (!ok) continue;
+        // every (key, query) pair of this half visible?  (then skip the per-element mask)
         bool full = (nkeys == kBN) && (qa + 63 < sq);
         if (a.right < kUnbounded) full = full && (n0 + kBN - 1 <= qa + off + a.right);
         if (a.left < kUnbounded) full = full && (n0 >= qa + 63 + off - a.left);
@@ -672,7 +712,23 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
             dd[e] = y.x; dd[e + 1] = y.y; dd[e + 2] = y.z; dd[e + 3] = y.w;
           }
           float p[32], ds[32];
-          if (full) {
+          if constexpr (DROP) {
+            // dropout: dV takes the kept probabilities scaled by 256 / T, dS = P (Z dP - D)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const long long qi = i0 + qc + e;
+              bool vis = key_ok && qi < sq;
+              const long long d = j - (qi + off);
+              if (a.right < kUnbounded) vis = vis && d <= a.right;
+              if (a.left < kUnbounded) vis = vis && d >= -(long long)a.left;
+              // query 32 c + e of the half: word (e % 16), byte (2 c + e / 16)
+              const bool keep = ((zb[e & 15] >> (8 * (2 * c + (e >> 4)))) & 0xFFu) < a.drop.threshold;
+              const float pe = vis ? ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e])) : 0.f;
+              const float z = keep ? a.drop.scale : 0.f;
+              p[e] = pe * z;
+              ds[e] = pe * (__uint_as_float(dpv[e]) * z - dd[e]);
+            }
+          } else if (full) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               p[e] = ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e]));
@@ -867,7 +923,8 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * 128 * sizeof(float), s) : cudaSuccess;
   if (e != cudaSuccess) return e;
   if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
-  auto kernel = dq ? bwd_sm100_d128_kernel<T, DV, true> : bwd_sm100_d128_kernel<T, DV, false>;
+  auto kernel = dq ? bwd_sm100_d128_kernel<T, DV, true, false>
+                  : (a.drop.threshold ? bwd_sm100_d128_kernel<T, DV, false, true> : bwd_sm100_d128_kernel<T, DV, false, false>);
   if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) != cudaSuccess)
     return e;
   BwdArgs ab = a;

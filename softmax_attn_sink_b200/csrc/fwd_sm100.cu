@@ -235,8 +235,10 @@ struct Item {
   Unit un[2];
 };
 
+// align16: start the key loop at a multiple of 16 keys (dropout draws its keep bytes for
+// 16-key blocks; the extra leading keys are masked like any invisible key).
 __device__ __forceinline__ void setup_item(const FwdArgs& a, bool even, int group, int b, int x, int z,
-                                           Item& it) {
+                                           Item& it, bool align16 = false) {
   int hA, hB, mA, mB;
   if (even) {
     const int g_ = x / (group / 2), p_ = x % (group / 2);
@@ -275,6 +277,7 @@ __device__ __forceinline__ void setup_item(const FwdArgs& a, bool even, int grou
     if (hi <= lo) { lo = it.un[1].lo; hi = it.un[1].hi; }
     else { lo = lo < it.un[1].lo ? lo : it.un[1].lo; hi = hi > it.un[1].hi ? hi : it.un[1].hi; }
   }
+  if (align16 && hi > lo) lo &= ~15;
   it.lo = lo;
   it.n_tiles = hi > lo ? (hi - lo + kBN - 1) / kBN : 0;
 #pragma unroll
@@ -299,7 +302,7 @@ struct ItemDesc {
 };
 static_assert(sizeof(ItemDesc) == 128, "item slot size");
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -516,7 +519,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         d.kind = more ? 1 : 0;
         if (more) {
           Item it;
-          setup_item(a, even, group, b, x, z, it);
+          setup_item(a, even, group, b, x, z, it, DROP);
           d.q0 = it.q0;
           d.sq = it.sq;
           d.k0 = it.k0;
@@ -616,13 +619,31 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t pk[32];
+          // dropout: keep bytes of this half's four 16-key blocks (the key loop starts at a
+          // multiple of 16); the row sum keeps every probability, the P V operand only the
+          // kept ones, scaled by 256 / T
+          uint4 kb4[DROP ? 4 : 1];
+          if constexpr (DROP) {
+            const uint32_t kb0 = (uint32_t)(klo0 + j * kBN + hh * 64) >> 4;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) kb4[gq] = dropout_bytes(a.drop, kb0 + gq, (uint32_t)(q0 + i), (uint32_t)h);
+          }
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float2 x = ffma2(make_float2(__uint_as_float(sr[hh * 64 + 2 * c]), __uint_as_float(sr[hh * 64 + 2 * c + 1])),
                                    sc2, nm2);
             const float2 pp = make_float2(ex2(x.x), ex2(x.y));
             sv[c & 1] = fadd2(sv[c & 1], pp);
-            pk[c] = pack2<T>(pp.x, pp.y);
+            if constexpr (DROP) {
+              const uint4 w4 = kb4[c >> 3];
+              const int t = (2 * c) & 15;   // byte of the pair's first key in its 16-key block
+              const uint32_t w = (t >> 2) == 0 ? w4.x : (t >> 2) == 1 ? w4.y : (t >> 2) == 2 ? w4.z : w4.w;
+              const uint32_t b0 = (w >> (8 * (t & 3))) & 0xFFu, b1 = (w >> (8 * (t & 3) + 8)) & 0xFFu;
+              pk[c] = pack2<T>(b0 < a.drop.threshold ? pp.x * a.drop.scale : 0.f,
+                               b1 < a.drop.threshold ? pp.y * a.drop.scale : 0.f);
+            } else {
+              pk[c] = pack2<T>(pp.x, pp.y);
+            }
           }
           tmem_st32(tS + hh * 32, pk);
         }
@@ -794,9 +815,10 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   Sched sc{zmax, width, smem_p <= dev.smem_optin ? 1 : 0};
   const long long smem = sc.persistent ? smem_p : L::smem_bytes(0);
   const long long grid = sc.persistent ? (items_ub < dev.sms ? items_ub : dev.sms) : items_ub;
-  e = cudaFuncSetAttribute(fwd_sm100_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kernel = a.drop.threshold ? fwd_sm100_kernel<T, DK, DV, true> : fwd_sm100_kernel<T, DK, DV, false>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  fwd_sm100_kernel<T, DK, DV><<<(unsigned)grid, kThreads, (size_t)smem, s>>>(a, sc, tq, tk, tv);
+  kernel<<<(unsigned)grid, kThreads, (size_t)smem, s>>>(a, sc, tq, tk, tv);
   return cudaGetLastError();
 }
 

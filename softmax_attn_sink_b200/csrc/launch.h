@@ -16,6 +16,16 @@ constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBadIndex = 2u;  // a paged block id or key count outside its table
 constexpr unsigned kStatusBadSeqlens = 4u;  // cu_seqlens broke its contract (attn_sink_check_seqlens)
 
+// Dropout keep decisions: key j of packed query row r and q head h is kept when byte j % 16
+// of Philox4x32-10(counter = (j / 16, r, h, offset), key = (seed_lo, seed_hi)) is below the
+// threshold T (keep probability T / 256); kept values are scaled by 256 / T.  Byte t is bits
+// 8 (t % 4) .. +7 of output word t / 4.
+struct Dropout {
+  uint32_t threshold;   // T in [1, 256]; 0 = no dropout
+  uint32_t seed_lo, seed_hi, offset;
+  float scale;          // 256 / T
+};
+
 struct FwdArgs {
   const void* q;
   const void* k;
@@ -29,6 +39,7 @@ struct FwdArgs {
   float scale;
   int left, right;       // effective window (causal folded into right), kUnbounded = none
   unsigned* status;
+  Dropout drop;          // threshold 0 = none (tensor-core path only)
 };
 
 struct BwdArgs {
@@ -54,6 +65,7 @@ struct BwdArgs {
   int left, right;
   unsigned* status;
   int band_groups;       // tensor-core path: (sequence, kv head) groups whose key tiles run together
+  Dropout drop;          // threshold 0 = none (deterministic tensor-core path only)
 };
 
 struct DecodeArgs {

@@ -19,28 +19,29 @@ def window(p):
     return (p.window_left, p.window_right)
 
 
-def run_fwd(p):
+def run_fwd(p, dropout=None):
     td = tdtype(p)
     q, k, v = dev(p.q, td), dev(p.k, td), dev(p.v, td)
     cu_q, cu_k = dev(p.cu_seqlens_q), dev(p.cu_seqlens_k)
     sink = None if p.sink is None else dev(p.sink)
     out, lse = sab.attn_sink_fwd(q, k, v, cu_q, cu_k, max(p.max_seqlen_q, 1), max(p.max_seqlen_k, 1),
-                                 sink, p.softmax_scale, p.causal, window(p))
+                                 sink, p.softmax_scale, p.causal, window(p), dropout=dropout)
     torch.cuda.synchronize()
     return out, lse
 
 
-def run_bwd(p, deterministic=False):
+def run_bwd(p, deterministic=False, dropout=None):
     td = tdtype(p)
     q, k, v = dev(p.q, td), dev(p.k, td), dev(p.v, td)
     do = dev(p.dout, td)
     cu_q, cu_k = dev(p.cu_seqlens_q), dev(p.cu_seqlens_k)
     sink = None if p.sink is None else dev(p.sink)
     mq, mk = max(p.max_seqlen_q, 1), max(p.max_seqlen_k, 1)
-    out, lse = sab.attn_sink_fwd(q, k, v, cu_q, cu_k, mq, mk, sink, p.softmax_scale, p.causal, window(p))
+    out, lse = sab.attn_sink_fwd(q, k, v, cu_q, cu_k, mq, mk, sink, p.softmax_scale, p.causal, window(p),
+                                 dropout=dropout)
     dq, dk, dv, ds = sab.attn_sink_bwd(q, k, v, out, do, lse, cu_q, cu_k, mq, mk, sink,
                                        p.softmax_scale, p.causal, window(p),
-                                       deterministic=deterministic)
+                                       deterministic=deterministic, dropout=dropout)
     torch.cuda.synchronize()
     return out, lse, dq, dk, dv, ds
 

@@ -139,3 +139,42 @@ def test_check_seqlens_rejects_null_arrays_on_host():
     p = _params()
     assert sab.lib().attn_sink_check_seqlens(ctypes.byref(p), None, None, None) == 1
     assert sab.lib().attn_sink_check_seqlens(None, None, 4096, None) == 1
+
+
+@pytest.mark.parametrize("drop,change,status", [
+    (None, {}, 1),                                    # NULL dropout
+    ((1.0, 1, 0), {}, 1), ((-0.1, 1, 0), {}, 1),      # p out of range (T = 0, T > 256)
+    ((float("nan"), 1, 0), {}, 1),
+    ((0.1, 1, 0), dict(dtype=sab.ATTN_SINK_FP32), 2),  # tensor-core path only
+])
+def test_dropout_entry_points_validate_on_host(drop, change, status):
+    """attn_sink_fwd_dropout / attn_sink_bwd_dropout reject a missing or out-of-range dropout
+    and unsupported dtypes before any launch (fake, aligned device addresses)."""
+    L = sab.lib()
+    p = _params(**change)
+    d = None if drop is None else ctypes.byref(sab.AttnSinkDropout(*drop))
+    a = 1 << 20
+    ws = L.attn_sink_bwd_workspace_size(ctypes.byref(p))
+    assert L.attn_sink_fwd_dropout(ctypes.byref(p), a, a, a, a, a, None, d, a, None, None, 0,
+                                   None) == status
+    assert L.attn_sink_bwd_dropout(ctypes.byref(p), a, a, a, a, a, a, a, a, None, d, a, a, a, None,
+                                   a, ws, None) == status
+
+
+def test_bwd_dropout_needs_head_dim_128():
+    L = sab.lib()
+    p = _params(head_dim_qk=64, head_dim_v=64)
+    a = 1 << 20
+    d = sab.AttnSinkDropout(0.1, 1, 0)
+    ws = L.attn_sink_bwd_workspace_size(ctypes.byref(p))
+    assert L.attn_sink_bwd_dropout(ctypes.byref(p), a, a, a, a, a, a, a, a, None, ctypes.byref(d),
+                                   a, a, a, None, a, ws, None) == 2
+
+
+def test_dropout_struct_matches_header():
+    text = open(HEADER).read()
+    body = re.search(r"typedef struct \{([^{}]*)\} attn_sink_dropout;", text).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\b([a-z_]+)\s*;", body)
+    assert names == [f[0] for f in sab.AttnSinkDropout._fields_]
+    assert ctypes.sizeof(sab.AttnSinkDropout) == 24
