@@ -327,12 +327,16 @@ def bench_fwd(args, world, peaks, peak_kind, sampler):
             "pairs": pairs, "flops": flops, "p": p}
 
 
-def bench_fwd_fp16(args, world, peaks, peak_kind):
-    """The headline forward with fp16 inputs (the same draws rounded to fp16)."""
+DROPOUT = (0.1, 0x5EED5EED1234ABCD, 0)   # p, Philox key, counter offset of the dropout legs
+
+
+def bench_fwd_variant(args, world, peaks, peak_kind, dtype="fp16", dropout=None):
+    """The headline forward with fp16 inputs (the same draws rounded to fp16), or with
+    dropout; the algorithmic flops are those of the plain forward."""
     import torch
     import softmax_attn_sink_b200 as sab
-    p = W.config2("fp16")
-    td = torch.float16
+    p = W.config2(dtype)
+    td = torch.float16 if dtype == "fp16" else torch.bfloat16
     q, k, v = (torch.from_numpy(x).to(td).cuda() for x in (p.q, p.k, p.v))
     cu = torch.from_numpy(p.cu_seqlens_q).cuda()
     sink = torch.from_numpy(p.sink).cuda()
@@ -343,11 +347,13 @@ def bench_fwd_fp16(args, world, peaks, peak_kind):
     flush = Flusher()
     steps = max(3, min(args.steps, 50))
     per, total = time_steps(lambda: sab.attn_sink_fwd(q, k, v, cu, cu, p.max_seqlen_q, p.max_seqlen_k, sink,
-                                                      p.softmax_scale, True, out=out, lse=lse),
+                                                      p.softmax_scale, True, out=out, lse=lse,
+                                                      dropout=dropout),
                             steps, args.warmup, world, flush)
     achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
     pk = peaks["bf16_tflops"]   # dense fp16 and bf16 tensor rates are equal (nominal ratio 1)
-    return {"workload": p.name, "unit": "TFLOP/s", "steps": steps,
+    name = p.name + (f"_dropout{dropout[0]}" if dropout else "")
+    return {"workload": name, "unit": "TFLOP/s", "steps": steps,
             "value": round(weak_scaling_value(flops, world, total, steps) / 1e12, 2),
             "ms_per_step": round(total / steps, 4), "flops": flops,
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk, "unit": "TFLOP/s",
@@ -384,11 +390,27 @@ def bench_fwd_bwd(args, world, peaks, peak_kind):
         lambda: sab.attn_sink_bwd(q, k, v, out, do, lse, cu, cu, 8192, 8192, sink, p.softmax_scale,
                                   True, dq=dq, dk=dk, dv=dv, dsink=dsink, deterministic=True),
         steps, args.warmup, world, flush)
+    fd_per, fd_total = time_steps(
+        lambda: sab.attn_sink_fwd(q, k, v, cu, cu, 8192, 8192, sink, p.softmax_scale, True,
+                                  out=out, lse=lse, dropout=DROPOUT), steps, args.warmup, world, flush)
+    bd_per, bd_total = time_steps(
+        lambda: sab.attn_sink_bwd(q, k, v, out, do, lse, cu, cu, 8192, 8192, sink, p.softmax_scale,
+                                  True, dq=dq, dk=dk, dv=dv, dsink=dsink, dropout=DROPOUT),
+        steps, args.warmup, world, flush)
     ff, bf = 2 * 256 * pairs, 2 * (3 * 128 + 2 * 128) * pairs
     fa = ff / (statistics.mean(f_per) * 1e-3) / 1e12
     ba = bf / (statistics.mean(b_per) * 1e-3) / 1e12
     da = bf / (statistics.mean(d_per) * 1e-3) / 1e12
+    fda = ff / (statistics.mean(fd_per) * 1e-3) / 1e12
+    bda = bf / (statistics.mean(bd_per) * 1e-3) / 1e12
     pk = peaks["bf16_tflops"]
+
+    def leg(total, flops, achieved, **kw):
+        return {"value": round(flops * world / (total / steps * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(total / steps, 4), "flops": flops,
+                "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk,
+                             "unit": "TFLOP/s", "frac": round(achieved / pk, 4), "traffic": None,
+                             "peak_source": f"bf16_tflops ({peak_kind}, burst)", **kw}}
     return {
         "workload": f"train{args.seqs}x8192_h16_d128_causal", "pairs": pairs, "steps": steps,
         "fwd": {"value": round(ff * world / (f_total / steps * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
@@ -409,6 +431,11 @@ def bench_fwd_bwd(args, world, peaks, peak_kind):
                                            "unit": "TFLOP/s", "frac": round(da / pk, 4), "traffic": None,
                                            "peak_source": f"bf16_tflops ({peak_kind}, burst)",
                                            "kernels": "preprocess + key-stationary dK/dV + query-stationary dQ"}},
+        # dropout p = 0.1 (Philox keep bytes drawn in the forward, redrawn in the backward);
+        # the flops counted are the plain ones
+        "fwd_dropout": leg(fd_total, ff, fda, dropout=list(DROPOUT[:1])),
+        "bwd_dropout": leg(bd_total, bf, bda, dropout=list(DROPOUT[:1]),
+                           kernels="preprocess + key-stationary dK/dV + query-stationary dQ"),
     }
 
 
@@ -551,7 +578,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all", "fwd", "fwd_fp16", "fwd_bwd", "decode"], default="all")
+    ap.add_argument("--workload", choices=["all", "fwd", "fwd_fp16", "fwd_dropout", "fwd_bwd", "decode"],
+                    default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", type=int, default=4, choices=[1, 2, 3, 4],
                     help="sequences of the fwd_bwd leg (4 = the full training workload)")
@@ -588,7 +616,9 @@ def main():
             if sampler is not None:
                 line["clocks"] = sampler.summary()
         if args.workload in ("all", "fwd_fp16"):
-            extra["fwd_fp16"] = bench_fwd_fp16(args, world, peaks, peak_kind)
+            extra["fwd_fp16"] = bench_fwd_variant(args, world, peaks, peak_kind, "fp16")
+        if args.workload in ("all", "fwd_dropout"):
+            extra["fwd_dropout"] = bench_fwd_variant(args, world, peaks, peak_kind, "bf16", DROPOUT)
         if args.workload in ("all", "fwd_bwd"):
             extra["fwd_bwd"] = bench_fwd_bwd(args, world, peaks, peak_kind)
         if args.workload in ("all", "decode"):
