@@ -37,10 +37,17 @@ using namespace sm100;
 constexpr int kBM = 128;       // query rows per CTA
 constexpr int kBN = 128;       // keys per tile
 constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 compute
+// With dropout a fourth warpgroup (warps 8-11, one warp per SM sub-partition) draws the keep
+// bytes of each key tile one tile ahead of the compute warps, into a two-stage shared-memory
+// ring.  Launched at 168 registers (384 x 168 = 64512): the first and the dropout warpgroups
+// drop to 136, the compute warps take 232 (128 x (136 + 136 + 232) = 64512).
+constexpr int kThreadsDrop = 384;
+constexpr int kRegsLowD = 136, kRegsHighD = 232;
+static_assert(128 * (2 * kRegsLowD + kRegsHighD) <= kThreadsDrop * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
 
-template <int DK, int DV>
+template <int DK, int DV, bool DROP>
 struct DqLayout {
   static constexpr int KH = DK / 64, VH = DV / 64;     // 64-element (128-byte) column halves
   static constexpr int kHalf = 128 * 128;              // one 128-row x 64-column box
@@ -50,8 +57,14 @@ struct DqLayout {
   static constexpr int kOffO = kOffQ + kQBytes;
   static constexpr int kOffK = kOffO + kOBytes;        // K ring, 2 stages
   static constexpr int kOffV = kOffK + 2 * kKBytes;    // V ring, 2 stages
-  static constexpr int kOffBar = kOffV + 2 * kVBytes;
-  static constexpr int kNumBars = 9;  // qd_full, kv_full[2], kv_empty[2], sdp_full, ds_full, dq_done, drain
+  // dropout keep bytes, 2 stages x 128 rows x 128 keys; row r's 16-byte block u sits at
+  // slot u ^ (r % 8), so that the compute warps' 16-byte row reads hit distinct banks
+  static constexpr int kZStage = 128 * 128;
+  static constexpr int kOffZ = kOffV + 2 * kVBytes;
+  static constexpr int kOffBar = kOffZ + (DROP ? 2 * kZStage : 0);
+  // qd_full, kv_full[2], kv_empty[2], sdp_full, ds_full, dq_done, drain (+ rng_full[2],
+  // rng_empty[2] with dropout)
+  static constexpr int kNumBars = DROP ? 13 : 9;
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   // + slack to align the base to 1 KB; at least 116 KB so two CTAs never share an SM (each
   // holds all 512 TMEM columns)
@@ -67,6 +80,8 @@ struct DqBars {
   __device__ __forceinline__ uint32_t ds_full() const { return base + 8u * 6; }
   __device__ __forceinline__ uint32_t dq_done() const { return base + 8u * 7; }
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * 8; }
+  __device__ __forceinline__ uint32_t rng_full(int s) const { return base + 8u * (9 + s); }
+  __device__ __forceinline__ uint32_t rng_empty(int s) const { return base + 8u * (11 + s); }
 };
 
 // CTA -> (row tile m, sequence b, q head h): the deepest row tiles first (under a causal mask
@@ -82,11 +97,11 @@ __device__ __forceinline__ void dq_tile_of(const BwdArgs& a, int mtiles, int& m,
 }
 
 template <typename Elem, int DK, int DV, bool DROP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
 bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_do) {
-  using L = DqLayout<DK, DV>;
+  using L = DqLayout<DK, DV, DROP>;
   extern __shared__ unsigned char smem_raw[];
 
   int m, b, h;
@@ -107,7 +122,7 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
   const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
   const uint32_t sQ = base_u32 + L::kOffQ, sO = base_u32 + L::kOffO, sK = base_u32 + L::kOffK,
-                 sV = base_u32 + L::kOffV;
+                 sV = base_u32 + L::kOffV, sZ = base_u32 + L::kOffZ;
   const DqBars bar{base_u32 + L::kOffBar};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -122,6 +137,12 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar.ds_full(), 4);   // one arrival per compute warp
     mbar_init(bar.dq_done(), 1);
     mbar_init(bar.drain(), 1);
+    if (DROP) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(bar.rng_full(s), 128);    // every dropout thread, after storing its row
+        mbar_init(bar.rng_empty(s), 128);   // every compute thread, after reading its row
+      }
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -135,6 +156,7 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == 0) {
     // ================================ TMA producer ======================================
+    if constexpr (DROP) regs_dec<kRegsLowD>();
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -163,6 +185,7 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
+    if constexpr (DROP) regs_dec<kRegsLowD>();
     if (lane == 0 && n > 0) {
       constexpr uint32_t id_s = idesc_of<Elem>(kBM, kBN, 0, 0);   // S, dP: K-major A and B
       constexpr uint32_t id_q = idesc_of<Elem>(kBM, DK, 0, 1);    // dS (TMEM) x K (MN-major)
@@ -206,8 +229,11 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       mma_commit(bar.drain());
       mbar_wait(bar.drain(), 0, a.status);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    if constexpr (DROP) regs_dec<kRegsLowD>();   // warps 2-3: no role, but part of the first warpgroup
+  } else if (warp < 8) {
     // ================================ compute warps (thread = query row) =================
+    if constexpr (DROP) regs_inc<kRegsHighD>();
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
@@ -229,6 +255,10 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar.sdp_full(), j & 1, a.status))) { ok = false; break; }
+      if (DROP && !__all_sync(0xffffffffu, mbar_wait(bar.rng_full(j & 1), (j >> 1) & 1, a.status))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -245,27 +275,35 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (c < klo || c >= khi) sv[c] = __float_as_uint(kNegInf);
         }
         uint32_t pk[32];
-        // dropout: dS = P (Z dP - D) with Z = 256 / T for kept keys and 0 otherwise, the keep
-        // bytes drawn as in the forward
+        // dropout: dS = P (Z dP - D) with Z = 256 / T for kept keys and 0 otherwise; the drop
+        // flags of this row's keys [64 hh, 64 hh + 64), drawn by the dropout warps
         uint4 kb4[DROP ? 4 : 1];
         if constexpr (DROP) {
-          const uint32_t kb0 = (uint32_t)(lo + (long long)j * kBN + hh * 64) >> 4;
+          const uint32_t zrow = sZ + (j & 1) * L::kZStage + r * 128;
 #pragma unroll
-          for (int gq = 0; gq < 4; ++gq) kb4[gq] = dropout_bytes(a.drop, kb0 + gq, (uint32_t)(q0 + i), (uint32_t)h);
+          for (int gq = 0; gq < 4; ++gq)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(kb4[gq].x), "=r"(kb4[gq].y), "=r"(kb4[gq].z), "=r"(kb4[gq].w)
+                         : "r"(zrow + (((4 * hh + gq) ^ (r & 7)) << 4))
+                         : "memory");
+          if (hh == 1) mbar_arrive(bar.rng_empty(j & 1));
         }
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), scale2, neg_lt));
           const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), scale2, neg_lt));
-          float dp0 = __uint_as_float(pv[2 * c]), dp1 = __uint_as_float(pv[2 * c + 1]);
           if constexpr (DROP) {
+            // keys 2c, 2c + 1: bytes 0-1 (c even) or 2-3 (c odd) of flag word c / 2
             const uint4 w4 = kb4[c >> 3];
-            const int t = (2 * c) & 15;
-            const uint32_t w = (t >> 2) == 0 ? w4.x : (t >> 2) == 1 ? w4.y : (t >> 2) == 2 ? w4.z : w4.w;
-            dp0 = ((w >> (8 * (t & 3))) & 0xFFu) < a.drop.threshold ? dp0 * a.drop.scale : 0.f;
-            dp1 = ((w >> (8 * (t & 3) + 8)) & 0xFFu) < a.drop.threshold ? dp1 * a.drop.scale : 0.f;
+            const int t = ((2 * c) & 15) >> 2;
+            const uint32_t w = t == 0 ? w4.x : t == 1 ? w4.y : t == 2 ? w4.z : w4.w;
+            const uint32_t d0 = (c & 1) ? prmt_sign<0xAAAA>(w) : prmt_sign<0x8888>(w);
+            const uint32_t d1 = (c & 1) ? prmt_sign<0xBBBB>(w) : prmt_sign<0x9999>(w);
+            pk[c] = pack2<Elem>(p0 * fmaf(__uint_as_float(pv[2 * c] & ~d0), a.drop.scale, -Dr),
+                                p1 * fmaf(__uint_as_float(pv[2 * c + 1] & ~d1), a.drop.scale, -Dr));
+          } else {
+            pk[c] = pack2<Elem>(p0 * (__uint_as_float(pv[2 * c]) - Dr), p1 * (__uint_as_float(pv[2 * c + 1]) - Dr));
           }
-          pk[c] = pack2<Elem>(p0 * (dp0 - Dr), p1 * (dp1 - Dr));
         }
         // dS of keys [64 hh, 64 hh + 64) over S columns [32 hh, 32 hh + 32): half 0 goes over
         // S columns already read, half 1 over half 0's S columns
@@ -299,6 +337,28 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
+    }
+  } else if constexpr (DROP) {
+    // ================================ dropout warps (thread = query row) =================
+    // Philox keep bytes of row r for the 8 16-key blocks of key tile j (counter: key block,
+    // packed row, q head, offset), turned into drop flags (bit 7 of a byte set = dropped) and
+    // stored for the compute thread of the same row.
+    regs_dec<kRegsLowD>();
+    const int r = (warp - 8) * 32 + lane;
+    const uint32_t row = (uint32_t)(q0 + m0 + r);
+    const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
+    for (int j = 0; j < n; ++j) {
+      const int st = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.rng_empty(st), ((j >> 1) & 1) ^ 1, a.status))) break;
+      const uint32_t kb0 = (uint32_t)((lo + (long long)j * kBN) >> 4);
+      const uint32_t zrow = sZ + st * L::kZStage + r * 128;
+#pragma unroll
+      for (int gq = 0; gq < 8; ++gq) {
+        const uint4 w = dropout_bytes(a.drop, kb0 + gq, row, (uint32_t)h);
+        st_shared_v4(zrow + ((gq ^ (r & 7)) << 4), drop_flags4(w.x, t4, t4h), drop_flags4(w.y, t4, t4h),
+                     drop_flags4(w.z, t4, t4h), drop_flags4(w.w, t4, t4h));
+      }
+      mbar_arrive(bar.rng_full(st));
     }
   }
 
@@ -345,18 +405,19 @@ bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows, CU
 
 template <typename Elem, int DK, int DV>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
-  using L = DqLayout<DK, DV>;
   constexpr CUtensorMapDataType dt =
       std::is_same<Elem, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tq, tk, tv, to;
   if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
       !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
     return cudaErrorInvalidValue;
-  auto kernel = a.drop.threshold ? bwd_dq_sm100_kernel<Elem, DK, DV, true> : bwd_dq_sm100_kernel<Elem, DK, DV, false>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  const bool drop = a.drop.threshold != 0;
+  auto kernel = drop ? bwd_dq_sm100_kernel<Elem, DK, DV, true> : bwd_dq_sm100_kernel<Elem, DK, DV, false>;
+  const int smem = drop ? DqLayout<DK, DV, true>::kSmem : DqLayout<DK, DV, false>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long ctas = (long long)((a.max_sq + kBM - 1) / kBM) * a.batch * a.hq;
-  kernel<<<(unsigned)ctas, kThreads, L::kSmem, s>>>(a, tq, tk, tv, to);
+  kernel<<<(unsigned)ctas, drop ? kThreadsDrop : kThreads, smem, s>>>(a, tq, tk, tv, to);
   return cudaGetLastError();
 }
 

@@ -645,35 +645,42 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
+        const long long qa = i0 + 64 * hh;
+        // Dropout drop flags of this half, drawn before the waits so that the Philox work
+        // overlaps the tensor pipe: a call gives the bytes of 16 keys for one query, so the 16
+        // threads of a 16-key block share the block's 64 calls (4 each).
+        uint32_t fw[DROP ? 16 : 1];
+        if constexpr (DROP) {
+          const uint32_t kb = (uint32_t)((n0 >> 4) + (r >> 4));
+          const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
+#pragma unroll
+          for (int s4 = 0; s4 < 4; ++s4) {
+            const uint4 w = dropout_bytes(a.drop, kb, (uint32_t)(q0 + qa + (r & 15) + 16 * s4), (uint32_t)h);
+            fw[4 * s4] = drop_flags4(w.x, t4, t4h);
+            fw[4 * s4 + 1] = drop_flags4(w.y, t4, t4h);
+            fw[4 * s4 + 2] = drop_flags4(w.z, t4, t4h);
+            fw[4 * s4 + 3] = drop_flags4(w.w, t4, t4h);
+          }
+        }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar.sdp_full(hh), t & 1, a.status));
         if (ok && t >= 1) ok = __all_sync(0xffffffffu, mbar_wait(bar.ds_free(hh), (t - 1) & 1, a.status));
         if (ok) tc_fence_after();
-        const long long qa = i0 + 64 * hh;
-        // Dropout keep bytes of this thread's key for the half's 64 queries.  A Philox call
-        // gives the bytes of 16 keys for one query, so the 16 threads of a 16-key block share
-        // the block's 64 calls (4 each) and swap bytes through the (still free) dS staging
-        // area of this half: word [block][key t][u] holds, in byte k, the keep byte of query
-        // u + 16 k for key t.  Both barriers are passed by every compute warp, also after a
-        // timed-out wait (ok = false), like the named barriers of the tile loop.
+        // The flag bytes are swapped through the (now free) dS staging area of this half:
+        // word [block][key t][u] holds, in byte k, the flag byte of query u + 16 k for key t.
+        // Both barriers are passed by every compute warp, also after a timed-out wait
+        // (ok = false), like the named barriers of the tile loop.
         uint32_t zb[DROP ? 16 : 1];
         if constexpr (DROP) {
           const uint32_t stage = sDS + hh * L::kHalf;
           const int blk = r >> 4, u = r & 15;
           constexpr int kBlockWords = 16 * 16 + 16;   // + 16 words: blocks 2w, 2w+1 in other banks
           if (ok) {
-            const uint32_t kb = (uint32_t)((n0 >> 4) + blk);
-            uint4 w[4];
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4)
-              w[s4] = dropout_bytes(a.drop, kb, (uint32_t)(q0 + qa + u + 16 * s4), (uint32_t)h);
 #pragma unroll
             for (int tk = 0; tk < 16; ++tk) {
-              auto word_of = [&](const uint4& x) {
-                return (tk >> 2) == 0 ? x.x : (tk >> 2) == 1 ? x.y : (tk >> 2) == 2 ? x.z : x.w;
-              };
+              // flag byte of key tk of query u + 16 s4 is byte tk % 4 of fw[4 s4 + tk / 4]
               const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
-              const uint32_t lo2 = __byte_perm(word_of(w[0]), word_of(w[1]), sel);
-              const uint32_t hi2 = __byte_perm(word_of(w[2]), word_of(w[3]), sel);
+              const uint32_t lo2 = __byte_perm(fw[tk >> 2], fw[4 + (tk >> 2)], sel);
+              const uint32_t hi2 = __byte_perm(fw[8 + (tk >> 2)], fw[12 + (tk >> 2)], sel);
               const uint32_t word = __byte_perm(lo2, hi2, 0x5410);
               asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage + 4u * (blk * kBlockWords + tk * 16 + u)), "r"(word)
                            : "memory");
@@ -712,28 +719,9 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
             dd[e] = y.x; dd[e + 1] = y.y; dd[e + 2] = y.z; dd[e + 3] = y.w;
           }
           float p[32], ds[32];
-          if constexpr (DROP) {
-            // dropout: dV takes the kept probabilities scaled by 256 / T, dS = P (Z dP - D)
+          if (full) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const long long qi = i0 + qc + e;
-              bool vis = key_ok && qi < sq;
-              const long long d = j - (qi + off);
-              if (a.right < kUnbounded) vis = vis && d <= a.right;
-              if (a.left < kUnbounded) vis = vis && d >= -(long long)a.left;
-              // query 32 c + e of the half: word (e % 16), byte (2 c + e / 16)
-              const bool keep = ((zb[e & 15] >> (8 * (2 * c + (e >> 4)))) & 0xFFu) < a.drop.threshold;
-              const float pe = vis ? ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e])) : 0.f;
-              const float z = keep ? a.drop.scale : 0.f;
-              p[e] = pe * z;
-              ds[e] = pe * (__uint_as_float(dpv[e]) * z - dd[e]);
-            }
-          } else if (full) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              p[e] = ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e]));
-              ds[e] = p[e] * (__uint_as_float(dpv[e]) - dd[e]);
-            }
+            for (int e = 0; e < 32; ++e) p[e] = ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e]));
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -743,8 +731,23 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
               if (a.right < kUnbounded) vis = vis && d <= a.right;
               if (a.left < kUnbounded) vis = vis && d >= -(long long)a.left;
               p[e] = vis ? ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e])) : 0.f;
-              ds[e] = p[e] * (__uint_as_float(dpv[e]) - dd[e]);
             }
+          }
+          if constexpr (DROP) {
+            // dropout: dV takes the kept probabilities (its 256 / T scale is applied to the
+            // result), dS = P (Z dP - D).  Query 32 c + e of the half is byte 2 c + e / 16 of
+            // word e % 16; its flag widened to 32 bits clears a dropped element.
+            const uint32_t sel0 = (8u | (2u * c)) * 0x1111u, sel1 = (8u | (2u * c + 1u)) * 0x1111u;
+            const float zs = a.drop.scale;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const uint32_t drop = prmt_sign_r(zb[e & 15], (e >> 4) ? sel1 : sel0);
+              ds[e] = p[e] * fmaf(__uint_as_float(dpv[e] & ~drop), zs, -dd[e]);
+              p[e] = __uint_as_float(__float_as_uint(p[e]) & ~drop);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ds[e] = p[e] * (__uint_as_float(dpv[e]) - dd[e]);
           }
           uint32_t pk[16], dk_[16];
 #pragma unroll
@@ -776,7 +779,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     for (int pass = 0; pass < 2; ++pass) {
       const int ncol = pass == 0 ? DK : DV;
       const uint32_t col = pass == 0 ? kColDK : kColDV;
-      const float mul = pass == 0 ? a.scale : 1.f;
+      const float mul = pass == 0 ? a.scale : (DROP ? a.drop.scale : 1.f);
       uint4* dst = reinterpret_cast<uint4*>(pass == 0 ? dkp : dvp);
       for (int c = 0; c < ncol / 32; ++c) {
         uint32_t v[32];

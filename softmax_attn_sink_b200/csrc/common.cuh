@@ -61,6 +61,31 @@ __device__ __forceinline__ uint4 dropout_bytes(const Dropout& d, uint32_t kb, ui
   return philox4x32_10(kb, r, h, d.offset, d.seed_lo, d.seed_hi);
 }
 
+// Drop flags of the four keep bytes in x: bit 7 of byte b of the result is set iff byte b of
+// x is >= T (the element is dropped); the other bits are unspecified.  t4 = (T - 1) in every
+// byte, t4h = t4 | 0x80808080.  Per byte, d = (T - 1 | 0x80) - (x & 0x7F) cannot borrow from
+// the next byte, and its bit 7 says (T - 1) mod 128 >= x mod 128; combined with the top bits
+// of x and T - 1 that decides T - 1 < x.  Valid for every 1 <= T <= 256.
+__device__ __forceinline__ uint32_t drop_flags4(uint32_t x, uint32_t t4, uint32_t t4h) {
+  const uint32_t d = t4h - (x & 0x7F7F7F7Fu);
+  return (~t4 & x) | (~(x ^ t4) & ~d);
+}
+
+// prmt.b32 with sign replication: selector nibble 8 | b fills the result byte with bit 7 of
+// byte b of `a`.  Used to widen drop flags into element masks.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "n"(SEL));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t prmt_sign_r(uint32_t a, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "r"(sel));
+  return r;
+}
+
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));

@@ -615,18 +615,25 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         const float neg_m = (m == kNegInf) ? 0.f : -m;
         // two columns per packed multiply-add and per packed sum update
         const float2 sc2 = make_float2(scale2, scale2), nm2 = make_float2(neg_m, neg_m);
+        const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
         float2 sv[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t pk[32];
-          // dropout: keep bytes of this half's four 16-key blocks (the key loop starts at a
+          // dropout: drop flags of this half's four 16-key blocks (the key loop starts at a
           // multiple of 16); the row sum keeps every probability, the P V operand only the
-          // kept ones, scaled by 256 / T
-          uint4 kb4[DROP ? 4 : 1];
+          // kept ones (the 256 / T scale is applied to the output)
+          uint32_t fl[DROP ? 16 : 1];
           if constexpr (DROP) {
             const uint32_t kb0 = (uint32_t)(klo0 + j * kBN + hh * 64) >> 4;
 #pragma unroll
-            for (int gq = 0; gq < 4; ++gq) kb4[gq] = dropout_bytes(a.drop, kb0 + gq, (uint32_t)(q0 + i), (uint32_t)h);
+            for (int gq = 0; gq < 4; ++gq) {
+              const uint4 w = dropout_bytes(a.drop, kb0 + gq, (uint32_t)(q0 + i), (uint32_t)h);
+              fl[4 * gq] = drop_flags4(w.x, t4, t4h);
+              fl[4 * gq + 1] = drop_flags4(w.y, t4, t4h);
+              fl[4 * gq + 2] = drop_flags4(w.z, t4, t4h);
+              fl[4 * gq + 3] = drop_flags4(w.w, t4, t4h);
+            }
           }
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -634,15 +641,12 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
                                    sc2, nm2);
             const float2 pp = make_float2(ex2(x.x), ex2(x.y));
             sv[c & 1] = fadd2(sv[c & 1], pp);
+            pk[c] = pack2<T>(pp.x, pp.y);
             if constexpr (DROP) {
-              const uint4 w4 = kb4[c >> 3];
-              const int t = (2 * c) & 15;   // byte of the pair's first key in its 16-key block
-              const uint32_t w = (t >> 2) == 0 ? w4.x : (t >> 2) == 1 ? w4.y : (t >> 2) == 2 ? w4.z : w4.w;
-              const uint32_t b0 = (w >> (8 * (t & 3))) & 0xFFu, b1 = (w >> (8 * (t & 3) + 8)) & 0xFFu;
-              pk[c] = pack2<T>(b0 < a.drop.threshold ? pp.x * a.drop.scale : 0.f,
-                               b1 < a.drop.threshold ? pp.y * a.drop.scale : 0.f);
-            } else {
-              pk[c] = pack2<T>(pp.x, pp.y);
+              // keys 2c, 2c + 1 are bytes 0-1 (c even) or 2-3 (c odd) of flag word c / 2:
+              // widen their flags to the two 16-bit halves and clear the dropped ones
+              const uint32_t mask = (c & 1) ? prmt_sign<0xBBAA>(fl[c >> 1]) : prmt_sign<0x9988>(fl[c >> 1]);
+              pk[c] &= ~mask;
             }
           }
           tmem_st32(tS + hh * 32, pk);
@@ -686,7 +690,8 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       const float sink2 = a.sink ? a.sink[h] * kLog2e : kNegInf;
       const float e_sink = (sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m);
       const float den = l + e_sink;
-      const float inv = den > 0.f ? 1.f / den : 0.f;
+      // with dropout, O summed the kept probabilities unscaled: the 256 / T factor goes here
+      const float inv = den > 0.f ? (DROP ? a.drop.scale : 1.f) / den : 0.f;
       const long long grow = (long long)q0 + i;   // packed row of this thread's query
       T* out = static_cast<T*>(a.out);
       uint4* orow = reinterpret_cast<uint4*>(out + (grow * a.hq + h) * DV);
