@@ -106,7 +106,8 @@ typedef void* attn_sink_stream_t;
  * sink-normalised probabilities).  Key j of packed query row r and q head h is kept when
  * byte j % 16 of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
  * Easy as 1, 2, 3", SC 2011) with counter (j / 16, r, h, offset) and key (seed low 32 bits,
- * seed high 32 bits) is below T = round(256 (1 - p)); byte t is bits 8 (t % 4) .. +7 of
+ * seed high 32 bits) is below T = floor(256 (1 - p) + 1/2) (p as passed, evaluated
+ * exactly); byte t is bits 8 (t % 4) .. +7 of
  * output word t / 4.  Kept probabilities are scaled by 256 / T (keep probability T / 256),
  * so the output's expectation is the output without dropout; lse is not affected.
  * 1 <= T <= 256 is required (0 <= p < 1 - 1/512).  The backward draws the same decisions.

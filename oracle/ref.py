@@ -48,6 +48,7 @@ from the bottom-right diagonal and causal clamps right to min(right, 0).
 """
 from __future__ import annotations
 
+import math
 from typing import Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
@@ -134,8 +135,9 @@ def philox4x32_10(ctr, key):
 
 def dropout_threshold(p: float) -> int:
     """Keep threshold T: an element is kept when its random byte is below T, so the keep
-    probability is T / 256 (T = round(256 (1 - p)), 1 <= T <= 256)."""
-    t = int(round(256.0 * (1.0 - float(p))))
+    probability is T / 256.  T = floor(256 (1 - p) + 1/2) for the float32 value of p (the
+    call passes p as a float), evaluated exactly (halves round up); 1 <= T <= 256."""
+    t = int(math.floor(256.0 * (1.0 - float(np.float32(p))) + 0.5))
     if not 1 <= t <= 256:
         raise ValueError("dropout p must satisfy 1 <= round(256 (1 - p)) <= 256")
     return t

@@ -125,13 +125,14 @@ int launch_decode(const attn_sink_params* p, DecodeArgs& a, int num_splits, void
   return from_cuda(launch_decode_split(a, p->dtype, s));
 }
 
-// Keep threshold and scale of a dropout request (round(256 (1 - p)) in [1, 256]); false
-// when p is outside that range.
+// Keep threshold and scale of a dropout request: T = floor(256 (1 - p) + 1/2) from the float
+// p, evaluated exactly in double (halves round up), in [1, 256]; false when p is outside
+// that range.
 bool dropout_of(const attn_sink_dropout* d, Dropout& out) {
   out = Dropout{};
   if (!d) return true;
   if (!(d->p >= 0.f) || !isfinite(d->p)) return false;
-  const long t = lroundf(256.f * (1.f - d->p));
+  const long t = (long)floor(256.0 * (1.0 - (double)d->p) + 0.5);
   if (t < 1 || t > 256) return false;
   out.threshold = (uint32_t)t;
   out.seed_lo = (uint32_t)(d->seed & 0xFFFFFFFFu);

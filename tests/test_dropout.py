@@ -144,6 +144,8 @@ MASK_CASES = [
      0.1),
     ("causal_sk_gt_sq_p50", [260, 190], [297, 400], 2, 1, True, 127, 0, "bf16", 0.5),
     ("causal_mha_p90", [385, 128], [385, 128], 3, 3, True, 100, 0, "fp16", 0.9),
+    # 256 (1 - p) = 230.5 exactly: T = 231 on both sides (halves round up)
+    ("half_way_threshold", [200], [200], 2, 2, False, 50, 50, "bf16", 25.5 / 256),
 ]
 
 

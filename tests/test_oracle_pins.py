@@ -526,6 +526,16 @@ def test_p14_keep_rate_and_threshold():
         ref.dropout_threshold(0.999)
 
 
+def test_p14_threshold_rounds_halves_up_from_the_float_p():
+    """T = floor(256 (1 - p) + 1/2) of the float32 p, exactly: 256 (1 - p) = 230.5 gives 231,
+    0.5 gives 1, and a p whose float is just above a half-way point rounds down."""
+    assert ref.dropout_threshold(25.5 / 256) == 231
+    assert ref.dropout_threshold(1 - 0.5 / 256) == 1
+    assert ref.dropout_threshold(0.75) == 64 and ref.dropout_threshold(0.0) == 256
+    p = float(np.nextafter(np.float32(25.5 / 256), np.float32(1)))   # 256 (1 - p) just below 230.5
+    assert ref.dropout_threshold(p) == 230
+
+
 def test_p14_no_dropout_is_identity():
     """p = 0 (T = 256) gives exactly the forward and backward without dropout."""
     p = W.random_problem(140, [9, 5], [11, 5], 4, 2, 8, 6, True, dtype="fp32", with_dout=True)
