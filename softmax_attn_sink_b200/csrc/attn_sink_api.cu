@@ -34,8 +34,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// (dk, dv): 64 or 128 with 32, 64 or 128; and 256 with 256 (the CANN flash_attn doc lists
+// head dims 64, 128 and 256)
 bool dims_supported(int dk, int dv) {
-  return (dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128);
+  return ((dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128)) || (dk == 256 && dv == 256);
 }
 
 int validate_params(const attn_sink_params* p, bool decode) {
@@ -166,6 +168,7 @@ int run_fwd(const attn_sink_params* p, const void* q, const void* k, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
   if (fwd_sm100_supported(a, dt)) return from_cuda(launch_fwd_sm100(a, dt, s));
+  if (fwd_d256_sm100_supported(a, dt)) return from_cuda(launch_fwd_d256_sm100(a, dt, s));
   if (a.drop.threshold) return ATTN_SINK_ERR_UNSUPPORTED;   // dropout runs on the tensor-core path only
   return from_cuda(launch_fwd_simt(a, dt, s));
 }

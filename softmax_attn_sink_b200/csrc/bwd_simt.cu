@@ -76,14 +76,22 @@ constexpr int kWarps = 4;
 constexpr int kBlockKeys = kKeysPerWarp * kWarps;
 constexpr int kTile = 32;
 
+// Shared-memory bytes of the dK/dV kernel (dynamic: at head dim 256 it exceeds 48 KB).
+template <int DK, int DV>
+constexpr int dkdv_smem_bytes() {
+  return 4 * (kBlockKeys * DK + kBlockKeys * DV + kTile * (DK + 1) + kTile * (DV + 1) + 2 * kTile);
+}
+
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kWarps * 32) bwd_dkdv_simt_kernel(const BwdArgs a) {
   constexpr int KPL = DK / 32, VPL = DV / 32;
-  __shared__ float s_k[kBlockKeys][DK];
-  __shared__ float s_v[kBlockKeys][DV];
-  __shared__ float s_q[kTile][DK + 1];
-  __shared__ float s_do[kTile][DV + 1];
-  __shared__ float s_lt[kTile], s_D[kTile];
+  extern __shared__ float smem_f[];
+  float(*s_k)[DK] = reinterpret_cast<float(*)[DK]>(smem_f);
+  float(*s_v)[DV] = reinterpret_cast<float(*)[DV]>(smem_f + kBlockKeys * DK);
+  float(*s_q)[DK + 1] = reinterpret_cast<float(*)[DK + 1]>(smem_f + kBlockKeys * (DK + DV));
+  float(*s_do)[DV + 1] = reinterpret_cast<float(*)[DV + 1]>(smem_f + kBlockKeys * (DK + DV) + kTile * (DK + 1));
+  float* s_lt = smem_f + kBlockKeys * (DK + DV) + kTile * (DK + 1) + kTile * (DV + 1);
+  float* s_D = s_lt + kTile;
 
   const int b = blockIdx.z, g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,13 +196,19 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_dkdv_simt_kernel(const BwdArg
 constexpr int kRowsPerWarp = 2;
 constexpr int kBlockRows = kRowsPerWarp * kWarps;
 
+template <int DK, int DV>
+constexpr int dq_smem_bytes() {
+  return 4 * (kBlockRows * DK + kBlockRows * DV + kTile * (DK + 1) + kTile * (DV + 1));
+}
+
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kWarps * 32) bwd_dq_simt_kernel(const BwdArgs a) {
   constexpr int KPL = DK / 32;
-  __shared__ float s_q[kBlockRows][DK];
-  __shared__ float s_do[kBlockRows][DV];
-  __shared__ float s_k[kTile][DK + 1];
-  __shared__ float s_v[kTile][DV + 1];
+  extern __shared__ float smem_f[];
+  float(*s_q)[DK] = reinterpret_cast<float(*)[DK]>(smem_f);
+  float(*s_do)[DV] = reinterpret_cast<float(*)[DV]>(smem_f + kBlockRows * DK);
+  float(*s_k)[DK + 1] = reinterpret_cast<float(*)[DK + 1]>(smem_f + kBlockRows * (DK + DV));
+  float(*s_v)[DV + 1] = reinterpret_cast<float(*)[DV + 1]>(smem_f + kBlockRows * (DK + DV) + kTile * (DK + 1));
 
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -283,12 +297,19 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_dq_simt_kernel(const BwdArgs 
 // it) and every query row by the dq pass, so no output needs clearing first.
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
+  constexpr int smem1 = dkdv_smem_bytes<DK, DV>(), smem2 = dq_smem_bytes<DK, DV>();
   cudaError_t e;
+  if ((e = cudaFuncSetAttribute(bwd_dkdv_simt_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem1)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(bwd_dq_simt_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem2)) != cudaSuccess)
+    return e;
   dim3 g1((a.max_sk + kBlockKeys - 1) / kBlockKeys, a.hkv, a.batch);
-  bwd_dkdv_simt_kernel<T, DK, DV><<<g1, kWarps * 32, 0, s>>>(a);
+  bwd_dkdv_simt_kernel<T, DK, DV><<<g1, kWarps * 32, smem1, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 g2((a.max_sq + kBlockRows - 1) / kBlockRows, a.hq, a.batch);
-  bwd_dq_simt_kernel<T, DK, DV><<<g2, kWarps * 32, 0, s>>>(a);
+  bwd_dq_simt_kernel<T, DK, DV><<<g2, kWarps * 32, smem2, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -302,6 +323,7 @@ cudaError_t dispatch_dims(const BwdArgs& a, cudaStream_t s) {
   ATTN_SINK_BWD_CASE(128, 32)
   ATTN_SINK_BWD_CASE(128, 64)
   ATTN_SINK_BWD_CASE(128, 128)
+  ATTN_SINK_BWD_CASE(256, 256)
 #undef ATTN_SINK_BWD_CASE
   return cudaErrorInvalidValue;
 }

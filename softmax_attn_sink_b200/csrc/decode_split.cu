@@ -30,7 +30,11 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kStageKeys = 64;     // keys per pipeline stage (16 per warp)
-constexpr int kStages = 3;
+// pipeline depth: 3 stages up to head dim 128; 2 at 256 (64 KB a stage), one CTA per SM
+template <int DK, int DV>
+__host__ __device__ constexpr int stages_of() { return DK + DV > 256 ? 2 : 3; }
+template <int DK, int DV>
+__host__ __device__ constexpr int ctas_per_sm() { return DK + DV > 256 ? 1 : 2; }
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -113,8 +117,9 @@ __device__ __forceinline__ void decode_range(const DecodeArgs& a, int b, long lo
 enum KvMode { kPacked = 0, kPagedSmemTable = 1, kPagedGlobalTable = 2 };
 
 template <typename T, int DK, int DV, int MODE>
-__global__ void __launch_bounds__(kWarps * 32, 2) decode_split_kernel(const DecodeArgs a, int chunk,
-                                                                       int extra_off) {
+__global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_split_kernel(const DecodeArgs a,
+                                                                                        int chunk, int extra_off) {
+  constexpr int kStages = stages_of<DK, DV>();
   constexpr bool PAGED = MODE != kPacked;
   constexpr int KCH = DK / 8, VCH = DV / 8;        // 16-byte chunks per row
   constexpr int KSTEPS = DK / 16, VTILES = DV / 8;
@@ -442,6 +447,7 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
   // chunk length so that `splits` chunks cover the longest visible range
   const int chunk = (a.max_sk + a.splits - 1) / a.splits;
   constexpr int STAGE_BYTES = kStageKeys * (DK + DV) * 2;
+  constexpr int kStages = stages_of<DK, DV>();
   constexpr int PIPE = kStages * STAGE_BYTES;
   constexpr int COMBINE = kWarps * 16 * (DV + 2) * 4;
   constexpr int SMEM = PIPE > COMBINE ? PIPE : COMBINE;
@@ -452,11 +458,13 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
     e = launch_split<T, DK, DV, kPacked>(a, ch, SMEM, 0, s);
   } else {
     // a chunk spans at most ch / block_size + 2 blocks; stage their ids in shared memory
-    // when that keeps two CTAs per SM (113 KB each), else read the table from global memory
+    // when that keeps the CTAs per SM (two of 113 KB, or one of 227 KB at head dim 256),
+    // else read the table from global memory
     const long long rows = kStages * kStageKeys * 8;
     const long long ids = (long long)ch / a.block_size + 2;
     const long long smem_t = (long long)SMEM + rows + 4 * ((ids + 31) / 32 * 32);
-    e = smem_t <= 113 * 1024 ? launch_split<T, DK, DV, kPagedSmemTable>(a, ch, (int)smem_t, SMEM, s)
+    const long long cap = ctas_per_sm<DK, DV>() == 2 ? 113 * 1024 : 227 * 1024;
+    e = smem_t <= cap ? launch_split<T, DK, DV, kPagedSmemTable>(a, ch, (int)smem_t, SMEM, s)
                              : launch_split<T, DK, DV, kPagedGlobalTable>(a, ch, SMEM + (int)rows, SMEM, s);
   }
   if (e != cudaSuccess) return e;
@@ -468,7 +476,8 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool decode_split_supported(int dk, int dv, int dtype) {
-  return (dtype == 0 || dtype == 2) && (dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128);
+  return (dtype == 0 || dtype == 2) &&
+         (((dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128)) || (dk == 256 && dv == 256));
 }
 
 namespace {
@@ -482,6 +491,7 @@ cudaError_t launch_dims(const DecodeArgs& a, cudaStream_t s) {
   ATTN_SINK_DEC_CASE(128, 32)
   ATTN_SINK_DEC_CASE(128, 64)
   ATTN_SINK_DEC_CASE(128, 128)
+  ATTN_SINK_DEC_CASE(256, 256)
 #undef ATTN_SINK_DEC_CASE
   return cudaErrorInvalidValue;
 }

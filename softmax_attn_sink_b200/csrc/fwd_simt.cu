@@ -18,13 +18,20 @@ constexpr int kWarps = 4;
 constexpr int kRows = kRowsPerWarp * kWarps;   // query rows per block
 constexpr int kKeys = 32;                      // keys per tile (one per lane)
 
+// Shared-memory bytes (dynamic: at head dim 256 they exceed 48 KB).
+template <int DK, int DV>
+constexpr int fwd_smem_bytes() {
+  return 4 * (kRows * DK + kKeys * (DK + 1) + kKeys * DV);
+}
+
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kWarps * 32)
 fwd_simt_kernel(const FwdArgs a) {
   constexpr int VPL = DV / 32;  // output dims per lane
-  __shared__ float s_q[kRows][DK];
-  __shared__ float s_k[kKeys][DK + 1];
-  __shared__ float s_v[kKeys][DV];
+  extern __shared__ float smem_f[];
+  float(*s_q)[DK] = reinterpret_cast<float(*)[DK]>(smem_f);
+  float(*s_k)[DK + 1] = reinterpret_cast<float(*)[DK + 1]>(smem_f + kRows * DK);
+  float(*s_v)[DV] = reinterpret_cast<float(*)[DV]>(smem_f + kRows * DK + kKeys * (DK + 1));
 
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,8 +135,11 @@ fwd_simt_kernel(const FwdArgs a) {
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   const int max_sq = a.cu_q ? a.max_sq : 1;
+  constexpr int smem = fwd_smem_bytes<DK, DV>();
+  cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
   dim3 grid((max_sq + kRows - 1) / kRows, a.hq, a.batch);
-  fwd_simt_kernel<T, DK, DV><<<grid, kWarps * 32, 0, s>>>(a);
+  fwd_simt_kernel<T, DK, DV><<<grid, kWarps * 32, smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -143,6 +153,7 @@ cudaError_t dispatch_dims(const FwdArgs& a, cudaStream_t s) {
   ATTN_SINK_FWD_CASE(128, 32)
   ATTN_SINK_FWD_CASE(128, 64)
   ATTN_SINK_FWD_CASE(128, 128)
+  ATTN_SINK_FWD_CASE(256, 256)
 #undef ATTN_SINK_FWD_CASE
   return cudaErrorInvalidValue;
 }

@@ -94,6 +94,9 @@ struct DecodeArgs {
 cudaError_t launch_fwd_simt(const FwdArgs& a, int dtype, cudaStream_t s);
 bool fwd_sm100_supported(const FwdArgs& a, int dtype);
 cudaError_t launch_fwd_sm100(const FwdArgs& a, int dtype, cudaStream_t s);
+// head dim 256 (dk = dv = 256), bf16 / fp16
+bool fwd_d256_sm100_supported(const FwdArgs& a, int dtype);
+cudaError_t launch_fwd_d256_sm100(const FwdArgs& a, int dtype, cudaStream_t s);
 
 // D, lse_tot and dsink (dsink cleared first); shared by both backward paths.
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s);

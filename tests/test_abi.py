@@ -56,7 +56,7 @@ SIZE_MAX = ctypes.c_size_t(-1).value
 
 @pytest.mark.parametrize("bad,status", [
     (dict(num_heads_kv=3), 1), (dict(batch=0), 1), (dict(total_q=0), 1),
-    (dict(head_dim_qk=96), 2), (dict(head_dim_v=256), 2), (dict(dtype=7), 2),
+    (dict(head_dim_qk=96), 2), (dict(head_dim_v=256), 2), (dict(head_dim_qk=256), 2), (dict(dtype=7), 2),
     (dict(window_left=-2), 1), (dict(softmax_scale=float("inf")), 1),
     (dict(max_seqlen_q=0), 1), (dict(max_seqlen_k=65), 1),
 ])

@@ -50,6 +50,9 @@ FWD_CASES = [
     ("persistent_many_items_p15", _LENS_P, _LENS_P, 6, 2, 128, 128, True, -1, -1, "normal", "bf16",
      0.15),
     ("grid_mode_p10", _LENS_G, _LENS_G, 2, 1, 128, 128, True, -1, -1, "normal", "bf16", 0.1),
+    ("d256_causal_gqa_p20", [300, 129, 0, 257], [300, 129, 0, 257], 4, 2, 256, 256, True, -1, -1,
+     "normal", "bf16", 0.2),
+    ("d256_fp16_window_p10", [200, 65], [230, 90], 2, 1, 256, 256, True, 70, 0, "normal", "fp16", 0.1),
 ]
 
 
@@ -110,14 +113,13 @@ def _visible_pairs(p):
         yield b, q0, q1, k0, k1, vis
 
 
-def _structured(lens_q, lens_k, hq, hkv, causal, wl, wr, dtype, for_bwd):
+def _structured(lens_q, lens_k, hq, hkv, causal, wl, wr, dtype, for_bwd, d=128):
     """q = 0 (every visible key equally likely), sink = -inf.  Forward: v one-hot on key
     position mod 128, so out[i, h, j % 128] = P Z for the one visible key j there.  Backward:
     k one-hot on key position, v = 1, dout one-hot on query position, so dv[j, :, i % 128]
     collects P Z of row i and dq[i, h, j % 128] = scale dS_ij."""
     cu_q, cu_k = W.cu_from_lengths(lens_q), W.cu_from_lengths(lens_k)
     tq, tk = int(cu_q[-1]), int(cu_k[-1])
-    d = 128
     q = np.zeros((tq, hq, d), np.float32)
     k = np.zeros((tk, hkv, d), np.float32)
     v = np.zeros((tk, hkv, d), np.float32)
@@ -139,7 +141,7 @@ def _structured(lens_q, lens_k, hq, hkv, causal, wl, wr, dtype, for_bwd):
 
 
 MASK_CASES = [
-    # name, lens_q, lens_k, hq, hkv, causal, wl, wr, dtype, p
+    # name, lens_q, lens_k, hq, hkv, causal, wl, wr, dtype, p (head dim 128)
     ("two_sided_gqa_p10", [300, 517, 129, 0, 1], [300, 517, 129, 0, 1], 4, 2, False, 60, 60, "bf16",
      0.1),
     ("causal_sk_gt_sq_p50", [260, 190], [297, 400], 2, 1, True, 127, 0, "bf16", 0.5),
@@ -149,16 +151,18 @@ MASK_CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", MASK_CASES, ids=[c[0] for c in MASK_CASES])
-def test_fwd_dropout_keep_mask_is_exact(case):
+@pytest.mark.parametrize("case,d", [(c, 128) for c in MASK_CASES] + [
+    (("d256_two_sided_p30", [300, 517], [300, 517], 2, 1, False, 120, 120, "bf16", 0.3), 256)],
+    ids=[c[0] for c in MASK_CASES] + ["d256_two_sided_p30"])
+def test_fwd_dropout_keep_mask_is_exact(case, d):
     name, lq, lk, hq, hkv, causal, wl, wr, dtype, pdrop = case
-    p = _structured(lq, lk, hq, hkv, causal, wl, wr, dtype, for_bwd=False)
+    p = _structured(lq, lk, hq, hkv, causal, wl, wr, dtype, for_bwd=False, d=d)
     drop = (pdrop, BIG_SEED + _seed(name), 11)
     t = ref.dropout_threshold(pdrop)
-    want = np.zeros((int(p.cu_seqlens_q[-1]), hq, 128), bool)
+    want = np.zeros((int(p.cu_seqlens_q[-1]), hq, d), bool)
     for b, q0, q1, k0, k1, vis in _visible_pairs(p):
-        cols = np.arange(k1 - k0) % 128
-        for i in range(q1 - q0):   # a row sees at most 128 consecutive keys: one per column
+        cols = np.arange(k1 - k0) % d
+        for i in range(q1 - q0):   # a row sees at most d consecutive keys: one per column
             assert len(set(cols[vis[i]])) == int(vis[i].sum())
         for h in range(hq):
             keep = ref.dropout_keep(drop[1], drop[2], t, np.arange(q0, q1), h, k1 - k0) & vis

@@ -46,6 +46,8 @@ PAGED_CASES = [
     # one split over 70000 keys: 4377 block ids do not fit next to the pipeline in shared
     # memory, so the kernel reads the table from global memory
     ("bs16_splits1_global_table", [70000, 3], 8, 1, 128, 128, 16, -1, "normal", 1),
+    # head dim 256: two pipeline stages, one CTA per SM
+    ("d256_bs64_gqa4", [700, 65, 1], 8, 2, 256, 256, 64, -1, "normal", 0),
 ]
 
 

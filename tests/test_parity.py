@@ -68,6 +68,14 @@ FWD_CASES = [
     # 9000 sequences: the item table would not fit in shared memory, so the forward runs one
     # CTA per item of the dense grid instead.
     ("grid_mode_many_sequences", _LENS_C, _LENS_C, 2, 1, 128, 128, True, -1, -1, "normal", "bf16"),
+    # head dim 256: the one-unit tensor-core forward (Q in TMEM, 64-key tiles), its fp16
+    # variant, and the CUDA-core kernel for fp32
+    ("d256_causal_gqa", [1, 63, 64, 65, 0, 300, 700], [1, 63, 64, 65, 0, 300, 700], 8, 2, 256, 256,
+     True, -1, -1, "normal", "bf16"),
+    ("d256_sq_ne_sk_full", [5, 200, 129], [2, 333, 150], 4, 4, 256, 256, False, -1, -1, "uniform", "bf16"),
+    ("d256_window_neg_inf_sink", [400, 3], [420, 260], 4, 1, 256, 256, True, 100, 0, "neg_inf", "bf16"),
+    ("d256_fp16_causal", [300, 257], [300, 257], 4, 2, 256, 256, True, -1, -1, "normal", "fp16"),
+    ("d256_fp32", [70, 33], [90, 33], 2, 1, 256, 256, True, -1, -1, "normal", "fp32"),
 ]
 
 
@@ -127,6 +135,10 @@ BWD_CASES = [
     ("fp16_dv64_window", [260], [300], 2, 1, 128, 64, True, 50, 0, "normal", "fp16"),
     ("fp16_dk64", [300, 131], [300, 131], 4, 1, 64, 64, True, -1, -1, "normal", "fp16"),
     ("fp16_dv32_simt", [150, 90], [160, 90], 2, 1, 64, 32, True, 40, 0, "normal", "fp16"),
+    # head dim 256 runs on the CUDA-core backward
+    ("d256_causal_gqa", [1, 100, 0, 131], [1, 100, 0, 131], 4, 2, 256, 256, True, -1, -1, "normal", "bf16"),
+    ("d256_fp16_window", [120], [150], 2, 2, 256, 256, True, 40, 0, "normal", "fp16"),
+    ("d256_fp32", [40, 9], [50, 9], 2, 1, 256, 256, True, -1, -1, "normal", "fp32"),
 ]
 
 
@@ -184,6 +196,8 @@ DECODE_CASES = [
     ("fp32", [300, 41], 8, 2, 128, 64, True, -1, -1, "normal", 0),
     ("fp16_gqa8", [1, 63, 1000, 4097], 16, 2, 128, 128, True, -1, -1, "normal", 0),
     ("fp16_dk64_dv32", [333, 1000], 8, 2, 64, 32, True, -1, -1, "normal", 3),
+    ("d256_gqa8", [1, 63, 700, 3000], 16, 2, 256, 256, True, -1, -1, "normal", 0),
+    ("fp16_d256_splits3", [500, 65], 8, 1, 256, 256, True, -1, -1, "normal", 3),
 ]
 
 
