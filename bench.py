@@ -361,6 +361,76 @@ def bench_fwd_variant(args, world, peaks, peak_kind, dtype="fp16", dropout=None)
                          "peak_source": f"bf16_tflops x 1 (nominal fp16 / bf16 dense ratio; {peak_kind}, burst)"}}
 
 
+def bench_fwd_d256(args, world, peaks, peak_kind):
+    """Head dim 256: the headline workload's 16 sequence lengths with 16 q / 4 kv heads at
+    d = 256, causal, bf16 N(0, 1) drawn on the device from a seeded generator."""
+    import torch
+    import softmax_attn_sink_b200 as sab
+    lens = W.config2_lengths()
+    cu_np = W.cu_from_lengths(lens)
+    tq, hq, hkv, d = int(cu_np[-1]), 16, 4, 256
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    q, k, v = (torch.randn((tq, h, d), generator=gen, device="cuda").to(torch.bfloat16) for h in (hq, hkv, hkv))
+    sink = torch.randn(hq, generator=gen, device="cuda")
+    cu = torch.from_numpy(cu_np).cuda()
+    mx = int(lens.max())
+    pairs = visible_pairs(cu_np, cu_np, hq, True)
+    flops = 2 * (d + d) * pairs
+    out = torch.empty((tq, hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((hq, tq), dtype=torch.float32, device="cuda")
+    flush = Flusher()
+    steps = max(3, min(args.steps, 50))
+    per, total = time_steps(lambda: sab.attn_sink_fwd(q, k, v, cu, cu, mx, mx, sink, 1.0 / 16.0, True,
+                                                      out=out, lse=lse),
+                            steps, args.warmup, world, flush)
+    achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
+    pk = peaks["bf16_tflops"]
+    # backward (CUDA cores at this head dim): a few steps
+    do = torch.randn((tq, hq, d), generator=gen, device="cuda").to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dsink = torch.empty(hq, dtype=torch.float32, device="cuda")
+    bflops = 2 * (3 * d + 2 * d) * pairs
+    b_per, b_total = time_steps(lambda: sab.attn_sink_bwd(q, k, v, out, do, lse, cu, cu, mx, mx, sink, 1.0 / 16.0,
+                                                          True, dq=dq, dk=dk, dv=dv, dsink=dsink),
+                                3, 1, world, flush)
+    ba = bflops / (statistics.mean(b_per) * 1e-3) / 1e12
+    # decode: 16 sequences of the decode workload's lengths, 32 q / 4 kv heads at d = 256
+    dl = W.config5_meta().cu_seqlens_k
+    dlens = np.diff(dl)[:16]
+    dcu_np = W.cu_from_lengths(dlens)
+    dk_ = torch.randn((int(dcu_np[-1]), 4, d), generator=gen, device="cuda").to(torch.bfloat16)
+    dv_ = torch.randn((int(dcu_np[-1]), 4, d), generator=gen, device="cuda").to(torch.bfloat16)
+    dq_ = torch.randn((16, 32, d), generator=gen, device="cuda").to(torch.bfloat16)
+    dsk = torch.randn(32, generator=gen, device="cuda")
+    dcu = torch.from_numpy(dcu_np).cuda()
+    dout = torch.empty((16, 32, d), dtype=torch.bfloat16, device="cuda")
+    dlse = torch.empty((32, 16), dtype=torch.float32, device="cuda")
+    dbytes = 2 * int(dcu_np[-1]) * 4 * d * 2 + dq_.numel() * 2 + dout.numel() * 2 + dlse.numel() * 4
+    d_per, d_total = time_steps(lambda: sab.attn_sink_decode(dq_, dk_, dv_, dcu, int(dlens.max()), dsk, 1.0 / 16.0,
+                                                             out=dout, lse=dlse),
+                                steps, args.warmup, world, flush)
+    da = dbytes / (statistics.mean(d_per) * 1e-3) / 1e9
+    pb = peaks["hbm_gbs"]
+    return {"workload": "varlen16_gqa16x4_d256_causal", "unit": "TFLOP/s", "steps": steps,
+            "value": round(weak_scaling_value(flops, world, total, steps) / 1e12, 2),
+            "ms_per_step": round(total / steps, 4), "flops": flops, "pairs": pairs,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk, "unit": "TFLOP/s",
+                         "frac": round(achieved / pk, 4), "traffic": None,
+                         "peak_source": f"bf16_tflops ({peak_kind}, burst)",
+                         "kernel": "fwd_d256_sm100 (one launch per step)"},
+            "bwd": {"value": round(bflops * world / (b_total / 3 * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "ms_per_step": round(b_total / 3, 3), "flops": bflops, "steps": 3,
+                    "roofline": {"bound": "tensor", "achieved": round(ba, 2), "peak": pk, "unit": "TFLOP/s",
+                                 "frac": round(ba / pk, 4), "traffic": None,
+                                 "kernels": "preprocess + CUDA-core dK/dV + CUDA-core dQ"}},
+            "decode": {"workload": "decode16_gqa32x4_d256_L8k-32k", "value": round(dbytes * world / (d_total / steps * 1e-3) / 1e9, 1),
+                       "unit": "GB/s", "ms_per_step": round(d_total / steps, 4), "bytes_per_step": dbytes,
+                       "roofline": {"bound": "hbm", "achieved": round(da, 1), "peak": pb, "unit": "GB/s",
+                                    "frac": round(da / pb, 4), "traffic": None,
+                                    "kernels": "split + merge (two launches per step)"}}}
+
+
 def bench_fwd_bwd(args, world, peaks, peak_kind):
     import torch
     import softmax_attn_sink_b200 as sab
@@ -578,7 +648,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all", "fwd", "fwd_fp16", "fwd_dropout", "fwd_bwd", "decode"],
+    ap.add_argument("--workload", choices=["all", "fwd", "fwd_fp16", "fwd_dropout", "fwd_d256", "fwd_bwd", "decode"],
                     default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", type=int, default=4, choices=[1, 2, 3, 4],
@@ -619,6 +689,8 @@ def main():
             extra["fwd_fp16"] = bench_fwd_variant(args, world, peaks, peak_kind, "fp16")
         if args.workload in ("all", "fwd_dropout"):
             extra["fwd_dropout"] = bench_fwd_variant(args, world, peaks, peak_kind, "bf16", DROPOUT)
+        if args.workload in ("all", "fwd_d256"):
+            extra["fwd_d256"] = bench_fwd_d256(args, world, peaks, peak_kind)
         if args.workload in ("all", "fwd_bwd"):
             extra["fwd_bwd"] = bench_fwd_bwd(args, world, peaks, peak_kind)
         if args.workload in ("all", "decode"):

@@ -209,6 +209,11 @@ int run_bwd(const attn_sink_params* p, const void* q, const void* k, const void*
   a.status = status_ptr();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
+  if (bwd_d256_sm100_supported(a, dt)) {   // head dim 256: no atomics in either mode
+    cudaError_t e = launch_bwd_preprocess(a, dt, s);
+    if (e == cudaSuccess) e = launch_bwd_d256_sm100(a, dt, s);
+    return from_cuda(e);
+  }
   if (!deterministic) {
     if (bwd_sm100_supported(a, dt)) return from_cuda(launch_bwd_sm100(a, dt, s));
     return from_cuda(launch_bwd_simt(a, dt, s));

@@ -49,8 +49,9 @@ __host__ __device__ constexpr uint32_t col_S(int b) { return 128u + 64u * (uint3
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kStages * kTileBytes;
 constexpr int kOffBar = kOffV + kStages * kTileBytes;
-// q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], pv_done, drain
-constexpr int kNumBars = 1 + 4 * kStages + 6;
+// q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], pv_done, drain,
+// o_done
+constexpr int kNumBars = 1 + 4 * kStages + 7;
 constexpr int kOffSlot = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffSlot + 16 + 1024;  // + slack to align the base to 1 KB
 
@@ -65,6 +66,9 @@ struct Bars {
   __device__ __forceinline__ uint32_t p_full(int b) const { return base + 8u * (3 + 4 * kStages + b); }
   __device__ __forceinline__ uint32_t pv_done() const { return base + 8u * (5 + 4 * kStages); }
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * (6 + 4 * kStages); }
+  // after the last PV only: the epilogue cannot use pv_done's parity, because when the last
+  // S is ready PV(n - 2) may still be running (S(j) is issued behind PV(j - 2), not PV(j - 1))
+  __device__ __forceinline__ uint32_t o_done() const { return base + 8u * (7 + 4 * kStages); }
 };
 
 // CTA -> (row tile z, sequence b, q head h): the deepest row tiles first (under a causal mask
@@ -122,6 +126,7 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
     }
     mbar_init(bar.pv_done(), 1);
     mbar_init(bar.drain(), 1);
+    mbar_init(bar.o_done(), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -201,6 +206,7 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
         mma_commit(bar.v_empty(st));
         if (j + 2 < n) ok = issue_s(j + 2);
       }
+      if (ok) mma_commit(bar.o_done());
       // every MMA must be complete before the TMEM is freed
       mma_commit(bar.drain());
       mbar_wait(bar.drain(), 0, a.status);
@@ -331,7 +337,7 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
       if (lane == 0) mbar_arrive(bar.p_full(j & 1));
     }
     // ---- epilogue: out = O / (l + 2^{sink2 - m}),  lse = (m + log2 l) ln 2 ----------------
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar.pv_done(), (n - 1) & 1, a.status));
+    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar.o_done(), 0, a.status));
     if (ok) {
       tc_fence_after();
       const float sink2 = a.sink ? a.sink[h] * kLog2e : kNegInf;

@@ -107,6 +107,10 @@ cudaError_t launch_bwd_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
 // Query-stationary dQ without atomics (the deterministic backward's dQ pass).
 bool bwd_dq_sm100_supported(const BwdArgs& a, int dtype);
 cudaError_t launch_bwd_dq_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
+// head dim 256 (dk = dv = 256), bf16 / fp16: dQ, dK and dV kernels after the preprocess;
+// deterministic (no atomics)
+bool bwd_d256_sm100_supported(const BwdArgs& a, int dtype);
+cudaError_t launch_bwd_d256_sm100(const BwdArgs& a, int dtype, cudaStream_t s);
 // Contract check of cu_seqlens_q (may be nullptr) and cu_seqlens_k; sets kStatusBadSeqlens.
 cudaError_t launch_check_seqlens(const int32_t* cu_q, const int32_t* cu_k, int batch, int total_q, int total_k,
                                  int max_sq, int max_sk, unsigned* status, cudaStream_t s);

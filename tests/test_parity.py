@@ -135,9 +135,12 @@ BWD_CASES = [
     ("fp16_dv64_window", [260], [300], 2, 1, 128, 64, True, 50, 0, "normal", "fp16"),
     ("fp16_dk64", [300, 131], [300, 131], 4, 1, 64, 64, True, -1, -1, "normal", "fp16"),
     ("fp16_dv32_simt", [150, 90], [160, 90], 2, 1, 64, 32, True, 40, 0, "normal", "fp16"),
-    # head dim 256 runs on the CUDA-core backward
+    # head dim 256: the dQ / dK / dV tensor-core kernels (bf16, fp16); fp32 on the CUDA cores
     ("d256_causal_gqa", [1, 100, 0, 131], [1, 100, 0, 131], 4, 2, 256, 256, True, -1, -1, "normal", "bf16"),
     ("d256_fp16_window", [120], [150], 2, 2, 256, 256, True, 40, 0, "normal", "fp16"),
+    ("d256_sq_ne_sk_full", [5, 130], [2, 200], 4, 2, 256, 256, False, -1, -1, "uniform", "bf16"),
+    ("d256_long_gqa4_window", [700, 300], [700, 300], 8, 2, 256, 256, True, 200, 0, "normal", "bf16"),
+    ("d256_neg_inf_sink_masked_rows", [5, 260], [2, 260], 4, 2, 256, 256, True, -1, -1, "neg_inf", "bf16"),
     ("d256_fp32", [40, 9], [50, 9], 2, 1, 256, 256, True, -1, -1, "normal", "fp32"),
 ]
 
@@ -165,12 +168,14 @@ def test_bwd_fully_masked_rows_have_zero_dq():
     assert np.all(np.isfinite(to_np(ds)))
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16", "bf16_d256"])
 def test_bwd_deterministic_is_bitwise_repeatable(dtype):
     """The deterministic backward gives the same bits on every run (dq summed over 7 key
     tiles in a fixed order, GQA heads, a sink); its results match the atomic path within
     the gradient tolerance."""
-    p = W.random_problem(31, [900, 300], [900, 300], 8, 2, 128, 128, True, dtype=dtype, with_dout=True)
+    d = 256 if dtype.endswith("d256") else 128
+    dtype = dtype.split("_")[0]
+    p = W.random_problem(31, [900, 300], [900, 300], 8, 2, d, d, True, dtype=dtype, with_dout=True)
     runs = [run_bwd(p, True) for _ in range(3)]
     for name, idx in (("dq", 2), ("dk", 3), ("dv", 4), ("dsink", 5)):
         first = to_np(runs[0][idx])
