@@ -30,9 +30,9 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kStageKeys = 64;     // keys per pipeline stage (16 per warp)
-// pipeline depth: 3 stages up to head dim 128; 2 at 256 (64 KB a stage), one CTA per SM
+// pipeline depth: 3 stages (at head dim 256 64 KB a stage, 192 KB, one CTA per SM)
 template <int DK, int DV>
-__host__ __device__ constexpr int stages_of() { return DK + DV > 256 ? 2 : 3; }
+__host__ __device__ constexpr int stages_of() { return 3; }
 template <int DK, int DV>
 __host__ __device__ constexpr int ctas_per_sm() { return DK + DV > 256 ? 1 : 2; }
 
