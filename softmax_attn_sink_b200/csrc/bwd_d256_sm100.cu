@@ -128,15 +128,23 @@ struct Bars {
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_dq_d256_kernel(const BwdArgs a, int mtiles, const __grid_constant__ CUtensorMap tm_o,
+bwd_dq_d256_kernel(const BwdArgs a, int mtiles, int band, const __grid_constant__ CUtensorMap tm_o,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using namespace dq;
   extern __shared__ unsigned char smem_raw[];
-  // CTA -> (row tile, sequence, q head): deepest row tiles first, heads fastest
-  const long long per_level = (long long)a.batch * a.hq;
-  const int zr = (int)(blockIdx.x / per_level);
-  const int rem = (int)(blockIdx.x - (long long)zr * per_level);
-  const int m = mtiles - 1 - zr, b = rem / a.hq, h = rem - (rem / a.hq) * a.hq;
+  // CTA -> (row tile, sequence, q head), in bands of `band` (sequence, kv head) groups whose
+  // K / V fit in L2 together; within a band the deepest row tiles first, then the groups and
+  // their q heads
+  const int group = a.hq / a.hkv, G = a.batch * a.hkv;
+  const long long per_band = (long long)band * group * mtiles;
+  const int bi = (int)(blockIdx.x / per_band);
+  const int first = bi * band, members = (G - first < band) ? G - first : band;
+  const long long rem = blockIdx.x - (long long)bi * per_band;
+  const int zr = (int)(rem / ((long long)members * group));
+  const int r2 = (int)(rem - (long long)zr * members * group);
+  const int grp = first + r2 / group;
+  const int m = mtiles - 1 - zr, b = grp / a.hkv;
+  const int h = (grp - b * a.hkv) * group + r2 % group;
   const int q0 = a.cu_q[b], sq = a.cu_q[b + 1] - q0;
   const int k0 = a.cu_k[b], sk = a.cu_k[b + 1] - k0;
   const int m0 = m * kBM;
@@ -307,17 +315,23 @@ bwd_dq_d256_kernel(const BwdArgs a, int mtiles, const __grid_constant__ CUtensor
 namespace ks {
 constexpr int kBN = 128;   // keys per CTA
 constexpr int kBM = 64;    // queries per tile
-// CTA -> (key tile, sequence, kv head): key tiles in increasing order (under a bottom-right
-// causal mask the first key tiles are seen by the most queries), kv heads fastest.
+// CTA -> (key tile, sequence, kv head).  Under a bottom-right causal mask the first key tiles
+// are seen by the most queries, so they go first.
+// In bands of `band` (sequence, kv head) groups whose Q / dout fit in L2 together; within a
+// band key tiles in increasing order, then the groups.
 struct Tile {
   int b, g, q0, sq, k0, sk, n0, nkeys, qlo, n_m, T;
 };
-__device__ __forceinline__ bool tile_of(const BwdArgs& a, Tile& t) {
-  const long long per_level = (long long)a.batch * a.hkv;
-  const int nt = (int)(blockIdx.x / per_level);
-  const int rem = (int)(blockIdx.x - (long long)nt * per_level);
-  t.b = rem / a.hkv;
-  t.g = rem - t.b * a.hkv;
+__device__ __forceinline__ bool tile_of(const BwdArgs& a, int ntiles, int band, Tile& t) {
+  const int G = a.batch * a.hkv;
+  const long long per_band = (long long)band * ntiles;
+  const int bi = (int)(blockIdx.x / per_band);
+  const int first = bi * band, members = (G - first < band) ? G - first : band;
+  const long long rem = blockIdx.x - (long long)bi * per_band;
+  const int nt = (int)(rem / members);
+  const int grp = first + (int)(rem - (long long)nt * members);
+  t.b = grp / a.hkv;
+  t.g = grp - t.b * a.hkv;
   t.q0 = a.cu_q[t.b];
   t.sq = a.cu_q[t.b + 1] - t.q0;
   t.k0 = a.cu_k[t.b];
@@ -362,12 +376,13 @@ struct Bars {
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_dv_d256_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o) {
+bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_o) {
   using namespace dvk;
   using ks::kBM;
   extern __shared__ unsigned char smem_raw[];
   ks::Tile tl;
-  if (!ks::tile_of(a, tl)) return;
+  if (!ks::tile_of(a, ntiles, band, tl)) return;
   const int group = a.hq / a.hkv, T_ = tl.T;
   auto head_of = [&](int t) { return tl.g * group + t / tl.n_m; };
   auto qbase_of = [&](int t) { return tl.qlo + (t % tl.n_m) * kBM; };
@@ -553,13 +568,13 @@ struct Bars {
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_dk_d256_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
-                   const __grid_constant__ CUtensorMap tm_v) {
+bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_v) {
   using namespace dkk;
   using ks::kBM;
   extern __shared__ unsigned char smem_raw[];
   ks::Tile tl;
-  if (!ks::tile_of(a, tl)) return;
+  if (!ks::tile_of(a, ntiles, band, tl)) return;
   const int group = a.hq / a.hkv, T_ = tl.T;
   auto head_of = [&](int t) { return tl.g * group + t / tl.n_m; };
   auto qbase_of = [&](int t) { return tl.qlo + (t % tl.n_m) * kBM; };
@@ -765,6 +780,16 @@ bool make_map(CUtensorMap* map, const void* base, int heads, int rows, int box_r
 long long dq_grid(const BwdArgs& a) { return (long long)((a.max_sq + dq::kBM - 1) / dq::kBM) * a.batch * a.hq; }
 long long ks_grid(const BwdArgs& a) { return (long long)((a.max_sk + ks::kBN - 1) / ks::kBN) * a.batch * a.hkv; }
 
+// (sequence, kv head) groups per band: as many as fit `per_group` bytes each in about half of
+// the 126 MB L2
+int band_of(const BwdArgs& a, long long per_group) {
+  long long s = (64LL << 20) / (per_group > 0 ? per_group : 1);
+  const long long G = (long long)a.batch * a.hkv;
+  if (s < 1) s = 1;
+  if (s > G) s = G;
+  return (int)s;
+}
+
 template <typename T>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   constexpr CUtensorMapDataType dt =
@@ -779,15 +804,19 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
       (e = cudaFuncSetAttribute(bwd_dv_d256_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dvk::kSmem)) ||
       (e = cudaFuncSetAttribute(bwd_dk_d256_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dkk::kSmem)))
     return e;
-  const int mtiles = (a.max_sq + dq::kBM - 1) / dq::kBM;
+  const int mtiles = (a.max_sq + dq::kBM - 1) / dq::kBM, ntiles = (a.max_sk + ks::kBN - 1) / ks::kBN;
+  const int group = a.hq / a.hkv;
+  // per group: K and V of the sequence (dQ); Q and dout of the group's q heads (dK, dV)
+  const int band_q = band_of(a, (long long)(a.max_sk > 0 ? a.max_sk : 1) * 2 * D * 2);
+  const int band_k = band_of(a, (long long)(a.max_sq > 0 ? a.max_sq : 1) * group * 2 * D * 2);
   if (mtiles > 0) {
-    bwd_dq_d256_kernel<T><<<(unsigned)dq_grid(a), kThreads, dq::kSmem, s>>>(a, mtiles, o128, k64, v64);
+    bwd_dq_d256_kernel<T><<<(unsigned)dq_grid(a), kThreads, dq::kSmem, s>>>(a, mtiles, band_q, o128, k64, v64);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (ks_grid(a) > 0) {
-    bwd_dk_d256_kernel<T><<<(unsigned)ks_grid(a), kThreads, dkk::kSmem, s>>>(a, q64, o64, v128);
+    bwd_dk_d256_kernel<T><<<(unsigned)ks_grid(a), kThreads, dkk::kSmem, s>>>(a, ntiles, band_k, q64, o64, v128);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_dv_d256_kernel<T><<<(unsigned)ks_grid(a), kThreads, dvk::kSmem, s>>>(a, q64, o64);
+    bwd_dv_d256_kernel<T><<<(unsigned)ks_grid(a), kThreads, dvk::kSmem, s>>>(a, ntiles, band_k, q64, o64);
   }
   return cudaGetLastError();
 }
