@@ -40,7 +40,8 @@
  *     accumulation, P and dS rounded to the same 16-bit type for the tensor cores, outputs
  *     rounded once to nearest-even; the CANN doc lists both BFLOAT16 and FLOAT16 for
  *     q / k / v) or ATTN_SINK_FP32 (fp32 everywhere, no tensor cores).
- *   - Supported head dims: head_dim_qk in {64, 128}; head_dim_v in {32, 64, 128}.
+ *   - Supported head dims: head_dim_qk in {64, 128} with head_dim_v in {32, 64, 128}, and
+ *     head_dim_qk = head_dim_v = 256 (the CANN flash_attn doc lists 64, 128 and 256).
  *   - Ownership: the caller allocates every buffer (inputs, outputs, workspace).  The
  *     library never allocates, frees or synchronises; every pointer except `params`
  *     is a device pointer and must be 16-byte aligned.  Calls are asynchronous on
@@ -87,8 +88,8 @@ typedef struct {
   int max_seqlen_k;     /* >= every sequence's key length                              */
   int num_heads_q;      /* Hq > 0                                                      */
   int num_heads_kv;     /* Hkv > 0, Hq % Hkv == 0                                      */
-  int head_dim_qk;      /* 64 or 128                                                   */
-  int head_dim_v;       /* 32, 64 or 128                                               */
+  int head_dim_qk;      /* 64 or 128; or 256 with head_dim_v = 256                     */
+  int head_dim_v;       /* 32, 64 or 128; or 256 with head_dim_qk = 256                */
   float softmax_scale;  /* multiplies QK^T; finite.  The slime wrapper's default is
                            1/sqrt(head_dim_qk); here the caller passes it explicitly   */
   int causal;           /* nonzero: bottom-right causal                                */
