@@ -188,7 +188,18 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
     unsigned char* base = smem + (st % kStages) * STAGE_BYTES;
     const uint32_t k_s = smem_u32(base), v_s = smem_u32(base + kStageKeys * DK * 2);
     const long long t0 = c_lo + (long long)st * kStageKeys;
-    if constexpr (!PAGED) {
+    if constexpr (!PAGED && KCH == VCH && DK <= 128) {
+      // K and V rows of a key coincide: one address per copy pair
+      constexpr int NR = kStageKeys * KCH / (kWarps * 32);
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        const int idx = tid + k * kWarps * 32, r = idx / KCH, ch = idx % KCH;
+        const bool ok = t0 + r < c_hi;
+        const long long base = ((k0 + t0 + r) * a.hkv + g) * DK + ch * 8;
+        cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, ok ? kp + base : kp, ok);
+        cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, ok ? vp + base : vp, ok);
+      }
+    } else if constexpr (!PAGED) {
       for (int idx = tid; idx < kStageKeys * KCH; idx += kWarps * 32) {
         const int r = idx / KCH, ch = idx % KCH;
         const bool ok = t0 + r < c_hi;
@@ -200,6 +211,22 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
         const bool ok = t0 + r < c_hi;
         const T* src = ok ? vp + ((k0 + t0 + r) * a.hkv + g) * DV + ch * 8 : vp;
         cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, src, ok);
+      }
+    } else if constexpr (KCH == VCH && DK <= 128) {
+      // K and V rows of a key coincide: every row this thread copies is read from shared
+      // memory first, all loads before the first copy, then K and V are issued from them
+      constexpr int NR = kStageKeys * KCH / (kWarps * 32);
+      const long long* rows = s_row + (st % kStages) * kStageKeys;
+      long long rw[NR];
+#pragma unroll
+      for (int k = 0; k < NR; ++k) rw[k] = rows[(tid + k * kWarps * 32) / KCH];
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        const int idx = tid + k * kWarps * 32, r = idx / KCH, ch = idx % KCH;
+        const bool ok = rw[k] >= 0;
+        const long long base = (rw[k] * a.hkv + g) * DK + ch * 8;
+        cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, ok ? kp + base : kp, ok);
+        cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, ok ? vp + base : vp, ok);
       }
     } else {
       const long long* rows = s_row + (st % kStages) * kStageKeys;
