@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
     unsigned char* base = smem + (st % kStages) * STAGE_BYTES;
     const uint32_t k_s = smem_u32(base), v_s = smem_u32(base + kStageKeys * DK * 2);
     const long long t0 = c_lo + (long long)st * kStageKeys;
-    if constexpr (!PAGED && KCH == VCH && DK <= 128) {
+    if constexpr (!PAGED && KCH == VCH) {
       // K and V rows of a key coincide: one address per copy pair
       constexpr int NR = kStageKeys * KCH / (kWarps * 32);
 #pragma unroll
