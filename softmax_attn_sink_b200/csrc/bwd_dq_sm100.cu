@@ -13,15 +13,22 @@
 // numbers in the same order.
 //
 // Per key tile j (128 keys):
-//   MMA thread:   S = Q K_j^T -> S columns, dP = dout V_j^T -> dP columns (SS, K-major),
-//                 then, once the compute warps wrote dS, dQ += dS K_j (A = dS from TMEM,
-//                 B = K_j read MN-major from the same shared-memory tile).
+//   MMA thread:   S_j = Q K_j^T (SS, K-major) into S buffer j % 2, dP = dout V_j^T into
+//                 the dP columns, and, once the compute warps wrote dS_j over S_j,
+//                 dQ += dS_j K_j (A = dS from TMEM, B = K_j read MN-major from the same
+//                 shared-memory tile).  Issue order: S(0), dP(0), then per tile
+//                 S(j+1), [dS(j) written], dP(j+1), dQ(j): S(j+1) runs while the compute
+//                 warps work on tile j, and they start on tile j+1 as soon as dP(j+1) is
+//                 done, while dQ(j) runs.  K tiles go through a 3-stage ring (2 with
+//                 dropout, whose keep-byte ring takes the room), V tiles through 2 stages.
 //   compute warps (thread = query row, TMEM lane): two 64-key halves; P = 2^{S scale log2e
 //                 - lse_tot log2e} (masked scores are -inf, so P = 0), dS = P (dP - D),
 //                 rounded to the input type and written over the S columns of its half.
-// TMEM columns: S [0,128) dP [128,256) dQ [256,256+DK).  dS of tile j sits in S's columns
-// until dQ(j) has read it; S(j+1) is issued after dQ(j) by the same thread, and MMAs from
-// one thread execute in issue order.  Every mbarrier wait is bounded; a timeout sets the
+// TMEM columns: S buffer 0 [0,128), dP [128,256), dQ [256,256+DK), S buffer 1 [384,512).
+// dS(j) sits in S buffer j % 2 until dQ(j) has read it; S(j+2) into the same buffer is
+// issued after dQ(j) by the same thread, and MMAs from one thread execute in issue order.
+// dP(j+1) overwrites dP(j) after the compute warps have signalled dS(j), so after their
+// last read of it.  Every mbarrier wait is bounded; a timeout sets the
 // status word and the CTA drains and frees its TMEM instead of hanging.
 #include <cuda.h>
 
@@ -45,7 +52,8 @@ constexpr int kThreadsDrop = 384;
 constexpr int kRegsLowD = 136, kRegsHighD = 232;
 static_assert(128 * (2 * kRegsLowD + kRegsHighD) <= kThreadsDrop * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+constexpr uint32_t kColP = 128, kColQ = 256;
+__host__ __device__ constexpr uint32_t col_S(int b) { return b ? 384u : 0u; }
 
 template <int DK, int DV, bool DROP>
 struct DqLayout {
@@ -53,18 +61,19 @@ struct DqLayout {
   static constexpr int kHalf = 128 * 128;              // one 128-row x 64-column box
   static constexpr int kQBytes = KH * kHalf, kOBytes = VH * kHalf;
   static constexpr int kKBytes = KH * kHalf, kVBytes = VH * kHalf;
+  static constexpr int KS = DROP ? 2 : 3;              // K ring depth
   static constexpr int kOffQ = 0;
   static constexpr int kOffO = kOffQ + kQBytes;
-  static constexpr int kOffK = kOffO + kOBytes;        // K ring, 2 stages
-  static constexpr int kOffV = kOffK + 2 * kKBytes;    // V ring, 2 stages
+  static constexpr int kOffK = kOffO + kOBytes;        // K ring, KS stages
+  static constexpr int kOffV = kOffK + KS * kKBytes;   // V ring, 2 stages
   // dropout keep bytes, 2 stages x 128 rows x 128 keys; row r's 16-byte block u sits at
   // slot u ^ (r % 8), so that the compute warps' 16-byte row reads hit distinct banks
   static constexpr int kZStage = 128 * 128;
   static constexpr int kOffZ = kOffV + 2 * kVBytes;
   static constexpr int kOffBar = kOffZ + (DROP ? 2 * kZStage : 0);
-  // qd_full, kv_full[2], kv_empty[2], sdp_full, ds_full, dq_done, drain (+ rng_full[2],
-  // rng_empty[2] with dropout)
-  static constexpr int kNumBars = DROP ? 13 : 9;
+  // qd_full, k_full[3], k_empty[3], v_full[2], v_empty[2], sdp_full, ds_full, dq_done, drain
+  // (+ rng_full[2], rng_empty[2] with dropout)
+  static constexpr int kNumBars = DROP ? 19 : 15;
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   // + slack to align the base to 1 KB; at least 116 KB so two CTAs never share an SM (each
   // holds all 512 TMEM columns)
@@ -74,14 +83,16 @@ struct DqLayout {
 struct DqBars {
   uint32_t base;
   __device__ __forceinline__ uint32_t qd_full() const { return base; }
-  __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 8u * (1 + s); }
-  __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8u * (3 + s); }
-  __device__ __forceinline__ uint32_t sdp_full() const { return base + 8u * 5; }
-  __device__ __forceinline__ uint32_t ds_full() const { return base + 8u * 6; }
-  __device__ __forceinline__ uint32_t dq_done() const { return base + 8u * 7; }
-  __device__ __forceinline__ uint32_t drain() const { return base + 8u * 8; }
-  __device__ __forceinline__ uint32_t rng_full(int s) const { return base + 8u * (9 + s); }
-  __device__ __forceinline__ uint32_t rng_empty(int s) const { return base + 8u * (11 + s); }
+  __device__ __forceinline__ uint32_t k_full(int s) const { return base + 8u * (1 + s); }
+  __device__ __forceinline__ uint32_t k_empty(int s) const { return base + 8u * (4 + s); }
+  __device__ __forceinline__ uint32_t v_full(int s) const { return base + 8u * (7 + s); }
+  __device__ __forceinline__ uint32_t v_empty(int s) const { return base + 8u * (9 + s); }
+  __device__ __forceinline__ uint32_t sdp_full() const { return base + 8u * 11; }
+  __device__ __forceinline__ uint32_t ds_full() const { return base + 8u * 12; }
+  __device__ __forceinline__ uint32_t dq_done() const { return base + 8u * 13; }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * 14; }
+  __device__ __forceinline__ uint32_t rng_full(int s) const { return base + 8u * (15 + s); }
+  __device__ __forceinline__ uint32_t rng_empty(int s) const { return base + 8u * (17 + s); }
 };
 
 // CTA -> (row tile m, sequence b, q head h): the deepest row tiles first (under a causal mask
@@ -129,9 +140,13 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 
   if (threadIdx.x == 0) {
     mbar_init(bar.qd_full(), 1);
+    for (int s = 0; s < L::KS; ++s) {
+      mbar_init(bar.k_full(s), 1);
+      mbar_init(bar.k_empty(s), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar.kv_full(s), 1);
-      mbar_init(bar.kv_empty(s), 1);
+      mbar_init(bar.v_full(s), 1);
+      mbar_init(bar.v_empty(s), 1);
     }
     mbar_init(bar.sdp_full(), 1);
     mbar_init(bar.ds_full(), 4);   // one arrival per compute warp
@@ -166,22 +181,26 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       mbar_arrive_expect_tx(bar.qd_full(), L::kQBytes + L::kOBytes);
       for (int hf = 0; hf < L::KH; ++hf) tma_load_3d(sQ + hf * L::kHalf, &tm_q, bar.qd_full(), hf * 64, h, row);
       for (int hf = 0; hf < L::VH; ++hf) tma_load_3d(sO + hf * L::kHalf, &tm_do, bar.qd_full(), hf * 64, h, row);
-      int issued = 0;
+      int nk = 0, nv = 0;   // tiles whose K / V loads were issued
       for (int j = 0; j < n; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(bar.kv_empty(st), ((j >> 1) & 1) ^ 1, a.status)) break;
+        const int sk_ = j % L::KS, sv_ = j & 1;
         const int krow = (int)(k0 + lo + (long long)j * kBN);
-        mbar_arrive_expect_tx(bar.kv_full(st), L::kKBytes + L::kVBytes);
+        if (!mbar_wait(bar.k_empty(sk_), ((j / L::KS) & 1) ^ 1, a.status)) break;
+        mbar_arrive_expect_tx(bar.k_full(sk_), L::kKBytes);
         for (int hf = 0; hf < L::KH; ++hf)
-          tma_load_3d(sK + st * L::kKBytes + hf * L::kHalf, &tm_k, bar.kv_full(st), hf * 64, g, krow);
+          tma_load_3d(sK + sk_ * L::kKBytes + hf * L::kHalf, &tm_k, bar.k_full(sk_), hf * 64, g, krow);
+        nk = j + 1;
+        if (!mbar_wait(bar.v_empty(sv_), ((j >> 1) & 1) ^ 1, a.status)) break;
+        mbar_arrive_expect_tx(bar.v_full(sv_), L::kVBytes);
         for (int hf = 0; hf < L::VH; ++hf)
-          tma_load_3d(sV + st * L::kVBytes + hf * L::kHalf, &tm_v, bar.kv_full(st), hf * 64, g, krow);
-        issued = j + 1;
+          tma_load_3d(sV + sv_ * L::kVBytes + hf * L::kHalf, &tm_v, bar.v_full(sv_), hf * 64, g, krow);
+        nv = j + 1;
       }
       // make sure no copy is still landing in shared memory when the CTA exits
       mbar_wait(bar.qd_full(), 0, a.status);
-      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
-        mbar_wait(bar.kv_full(j & 1), (j >> 1) & 1, a.status);
+      for (int p = nk - L::KS < 0 ? 0 : nk - L::KS; p < nk; ++p)
+        mbar_wait(bar.k_full(p % L::KS), (p / L::KS) & 1, a.status);
+      for (int p = nv - 2 < 0 ? 0 : nv - 2; p < nv; ++p) mbar_wait(bar.v_full(p & 1), (p >> 1) & 1, a.status);
     }
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
@@ -196,33 +215,51 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       const uint64_t kK = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
       const uint64_t mK = smem_desc(sK, L::kHalf, 1024, kLayoutSwizzle128B);
       const uint64_t kV = smem_desc(sV, 16, 1024, kLayoutSwizzle128B);
-      bool ok = mbar_wait(bar.qd_full(), 0, a.status);
-      for (int j = 0; j < n && ok; ++j) {
-        const int st = j & 1;
-        if (!(ok = mbar_wait(bar.kv_full(st), (j >> 1) & 1, a.status))) break;
+      // S(j) = Q K_j^T into S buffer j % 2; that buffer's dS(j - 2) was read by dQ(j - 2),
+      // issued earlier by this thread
+      auto issue_s = [&](int j) -> bool {
+        const int sk_ = j % L::KS;
+        if (!mbar_wait(bar.k_full(sk_), (j / L::KS) & 1, a.status)) return false;
         tc_fence_after();
-        const uint64_t koff = (uint64_t)((st * L::kKBytes) >> 4), voff = (uint64_t)((st * L::kVBytes) >> 4);
-        // S = Q K^T and dP = dout V^T.  S's columns held dS(j - 1), read by dQ(j - 1), which
-        // this thread issued earlier.
+        const uint64_t koff = (uint64_t)((sk_ * L::kKBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + kColS, kQ + off16, kK + koff + off16, id_s, ks > 0);
+          mma_ss(tmem + col_S(j & 1), kQ + off16, kK + koff + off16, id_s, ks > 0);
         }
+        return true;
+      };
+      // dP(j) = dout V_j^T; then V_j's stage is free and tile j's S and dP are announced
+      auto issue_p = [&](int j) -> bool {
+        const int sv_ = j & 1;
+        if (!mbar_wait(bar.v_full(sv_), (j >> 1) & 1, a.status)) return false;
+        tc_fence_after();
+        const uint64_t voff = (uint64_t)((sv_ * L::kVBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < DV / 16; ++ks) {
           const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
           mma_ss(tmem + kColP, kO + off16, kV + voff + off16, id_s, ks > 0);
         }
+        mma_commit(bar.v_empty(sv_));
         mma_commit(bar.sdp_full());
-        // dQ += dS K, once the compute warps have written dS
+        return true;
+      };
+      bool ok = mbar_wait(bar.qd_full(), 0, a.status);
+      if (ok) ok = issue_s(0) && issue_p(0);
+      for (int j = 0; j < n && ok; ++j) {
+        if (j + 1 < n && !(ok = issue_s(j + 1))) break;   // overlaps the compute warps' tile j
+        // the compute warps have written dS(j) and are done reading dP(j)
         if (!(ok = mbar_wait(bar.ds_full(), j & 1, a.status))) break;
         tc_fence_after();
+        if (j + 1 < n && !(ok = issue_p(j + 1))) break;
+        // dQ += dS(j) K_j, then K_j's stage is free
+        const int sk_ = j % L::KS;
+        const uint64_t koff = (uint64_t)((sk_ * L::kKBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + kColQ, tmem + kColS + kk * 8, mK + koff + (uint64_t)((kk * 2048) >> 4), id_q,
+          mma_ts(tmem + kColQ, tmem + col_S(j & 1) + kk * 8, mK + koff + (uint64_t)((kk * 2048) >> 4), id_q,
                  (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar.kv_empty(st));
+        mma_commit(bar.k_empty(sk_));
       }
       if (ok) mma_commit(bar.dq_done());
       // every MMA must be complete before the TMEM is freed
@@ -263,8 +300,8 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t sv[64], pv[64];
-        tmem_ld32(tmem + lane_off + kColS + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tmem + lane_off + kColS + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tmem + lane_off + col_S(j & 1) + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tmem + lane_off + col_S(j & 1) + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_ld32(tmem + lane_off + kColP + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
         tmem_ld32(tmem + lane_off + kColP + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
         tmem_wait_ld();
@@ -307,7 +344,7 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         }
         // dS of keys [64 hh, 64 hh + 64) over S columns [32 hh, 32 hh + 32): half 0 goes over
         // S columns already read, half 1 over half 0's S columns
-        tmem_st32(tmem + lane_off + kColS + hh * 32, pk);
+        tmem_st32(tmem + lane_off + col_S(j & 1) + hh * 32, pk);
       }
       tmem_wait_st();
       tc_fence_before();
