@@ -436,6 +436,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+
 template <typename Elem, int DV, bool DQ, bool DROP>
 __global__ void __launch_bounds__(kThreadsP, 1)
 bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
@@ -609,7 +610,57 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       mbar_wait(bar.drain(), 0, a.status);
     }
   } else if (warp < 4) {
-    regs_dec<kRegsLow>();   // warps 2-3: no role, but part of the first warpgroup
+    regs_dec<kRegsLow>();   // warps 2-3: dropout keep flags (below), else no role
+    if constexpr (DROP) {
+      // Each half's 64 queries x 128 keys take 512 Philox calls (a call gives the bytes of 16
+      // keys for one query).  Thread rt draws block blk = rt / 8 for queries u + 16 k,
+      // u in {rt % 8, rt % 8 + 8}, k = 0..3, a half ahead of the compute warps, turns them
+      // into drop flags and, once the half's dS staging area is free, writes there the
+      // words [block][key tk][u] (byte k: query u + 16 k), then syncs on named barrier
+      // 3 + half with the compute warps (64 + 128 threads).  Both sides take that barrier
+      // exactly once per half, also after a timed-out wait, so its generations always pair
+      // up; while the compute warps work on a half these warps draw the next one.
+      const int rt = (warp - 2) * 32 + lane, blk = rt >> 3, u0 = rt & 7;
+      const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
+      constexpr int kBlockWords = 16 * 16 + 16;   // + 16 words: blocks 2w, 2w+1 in other banks
+      bool ok = true;
+      for (int t = 0; t < T; ++t) {
+        const int h = head_of(t);
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const long long qa = qbase_of(t) + 64 * hh;
+          uint32_t fw[2][16];   // [u half][4 k + word]
+#pragma unroll
+          for (int uh = 0; uh < 2; ++uh)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint4 w = dropout_bytes(a.drop, (uint32_t)((n0 >> 4) + blk),
+                                            (uint32_t)(q0 + qa + u0 + 8 * uh + 16 * k), (uint32_t)h);
+              fw[uh][4 * k] = drop_flags4(w.x, t4, t4h);
+              fw[uh][4 * k + 1] = drop_flags4(w.y, t4, t4h);
+              fw[uh][4 * k + 2] = drop_flags4(w.z, t4, t4h);
+              fw[uh][4 * k + 3] = drop_flags4(w.w, t4, t4h);
+            }
+          if (ok && t >= 1) ok = __all_sync(0xffffffffu, mbar_wait(bar.ds_free(hh), (t - 1) & 1, a.status));
+          if (ok) {
+            const uint32_t stage = sDS + hh * L::kHalf;
+#pragma unroll
+            for (int uh = 0; uh < 2; ++uh)
+#pragma unroll
+              for (int tk = 0; tk < 16; ++tk) {
+                // flag byte of key tk of query u + 16 k is byte tk % 4 of fw[uh][4 k + tk / 4]
+                const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
+                const uint32_t lo2 = __byte_perm(fw[uh][tk >> 2], fw[uh][4 + (tk >> 2)], sel);
+                const uint32_t hi2 = __byte_perm(fw[uh][8 + (tk >> 2)], fw[uh][12 + (tk >> 2)], sel);
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage + 4u * (blk * kBlockWords + tk * 16 + u0 + 8 * uh)),
+                             "r"(__byte_perm(lo2, hi2, 0x5410))
+                             : "memory");
+              }
+          }
+          named_bar_sync(3 + hh, 192);
+        }
+      }
+    }
   } else if (warp < 8) {
     // ================================ compute warps (thread = key row) ===================
     regs_inc<kRegsHigh>();
@@ -646,47 +697,19 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       for (int hh = 0; hh < 2; ++hh) {
         const uint32_t cS = hh ? kColSb : kColSa, cP = hh ? kColDPb : kColDPa;
         const long long qa = i0 + 64 * hh;
-        // Dropout drop flags of this half, drawn before the waits so that the Philox work
-        // overlaps the tensor pipe: a call gives the bytes of 16 keys for one query, so the 16
-        // threads of a 16-key block share the block's 64 calls (4 each).
-        uint32_t fw[DROP ? 16 : 1];
-        if constexpr (DROP) {
-          const uint32_t kb = (uint32_t)((n0 >> 4) + (r >> 4));
-          const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
-#pragma unroll
-          for (int s4 = 0; s4 < 4; ++s4) {
-            const uint4 w = dropout_bytes(a.drop, kb, (uint32_t)(q0 + qa + (r & 15) + 16 * s4), (uint32_t)h);
-            fw[4 * s4] = drop_flags4(w.x, t4, t4h);
-            fw[4 * s4 + 1] = drop_flags4(w.y, t4, t4h);
-            fw[4 * s4 + 2] = drop_flags4(w.z, t4, t4h);
-            fw[4 * s4 + 3] = drop_flags4(w.w, t4, t4h);
-          }
-        }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar.sdp_full(hh), t & 1, a.status));
         if (ok && t >= 1) ok = __all_sync(0xffffffffu, mbar_wait(bar.ds_free(hh), (t - 1) & 1, a.status));
         if (ok) tc_fence_after();
-        // The flag bytes are swapped through the (now free) dS staging area of this half:
-        // word [block][key t][u] holds, in byte k, the flag byte of query u + 16 k for key t.
-        // Both barriers are passed by every compute warp, also after a timed-out wait
+        // The drop flags of this half, written by warps 2-3 into the (now free) dS staging
+        // area: word [block][key t][u] holds, in byte k, the flag byte of query u + 16 k for
+        // key t.  Both barriers are passed by every compute warp, also after a timed-out wait
         // (ok = false), like the named barriers of the tile loop.
         uint32_t zb[DROP ? 16 : 1];
         if constexpr (DROP) {
           const uint32_t stage = sDS + hh * L::kHalf;
-          const int blk = r >> 4, u = r & 15;
-          constexpr int kBlockWords = 16 * 16 + 16;   // + 16 words: blocks 2w, 2w+1 in other banks
-          if (ok) {
-#pragma unroll
-            for (int tk = 0; tk < 16; ++tk) {
-              // flag byte of key tk of query u + 16 s4 is byte tk % 4 of fw[4 s4 + tk / 4]
-              const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
-              const uint32_t lo2 = __byte_perm(fw[tk >> 2], fw[4 + (tk >> 2)], sel);
-              const uint32_t hi2 = __byte_perm(fw[8 + (tk >> 2)], fw[12 + (tk >> 2)], sel);
-              const uint32_t word = __byte_perm(lo2, hi2, 0x5410);
-              asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage + 4u * (blk * kBlockWords + tk * 16 + u)), "r"(word)
-                           : "memory");
-            }
-          }
-          named_bar_sync(2, 128);
+          const int blk = r >> 4;
+          constexpr int kBlockWords = 16 * 16 + 16;
+          named_bar_sync(3 + hh, 192);   // warps 2-3 have written this half's flags
           if (ok) {
             const uint32_t src = stage + 4u * (blk * kBlockWords + (r & 15) * 16);
 #pragma unroll
