@@ -48,23 +48,22 @@ constexpr int kTile128 = 4 * kBox128;
 __device__ __forceinline__ uint64_t kmaj_off(int ks, int box) { return (uint64_t)(((ks >> 2) * box + (ks & 3) * 32) >> 4); }
 
 // The calling thread's 256-element row into TMEM columns [col, col + 128) of its lane as
-// packed pairs (zeros when !ok), then this warp's arrival on `bar`.
+// packed pairs (zeros when !ok), then this warp's arrival on `bar`.  All 32 loads are issued
+// before the first store (one memory round trip).
 template <typename T>
 __device__ __forceinline__ void stage_row(const T* row, bool ok, uint32_t taddr, uint32_t bar, int lane) {
   const uint4* src = reinterpret_cast<const uint4*>(row);
-#pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
-    uint32_t w[32];
+  uint32_t w[4][32];
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const uint4 x = ok ? src[c * 8 + v] : make_uint4(0u, 0u, 0u, 0u);
-      w[4 * v] = x.x;
-      w[4 * v + 1] = x.y;
-      w[4 * v + 2] = x.z;
-      w[4 * v + 3] = x.w;
-    }
-    tmem_st32(taddr + c * 32, w);
+  for (int v = 0; v < 32; ++v) {
+    const uint4 x = ok ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+    w[v >> 3][4 * (v & 7)] = x.x;
+    w[v >> 3][4 * (v & 7) + 1] = x.y;
+    w[v >> 3][4 * (v & 7) + 2] = x.z;
+    w[v >> 3][4 * (v & 7) + 3] = x.w;
   }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_st32(taddr + c * 32, w[c]);
   tmem_wait_st();
   tc_fence_before();
   __syncwarp();

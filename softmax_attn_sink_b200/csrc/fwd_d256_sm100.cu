@@ -218,23 +218,22 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     const int i = m0 + r;
     const bool row_ok = i < sq;
-    // Q row i into TMEM columns [0, 128) as packed pairs (zeros past the sequence end)
+    // Q row i into TMEM columns [0, 128) as packed pairs (zeros past the sequence end); all
+    // 32 loads of the row are issued before the first store (one memory round trip)
     {
       const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) +
                                                          ((long long)(q0 + (row_ok ? i : 0)) * a.hq + h) * D);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t w[32];
+      uint32_t w[4][32];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const uint4 x = row_ok ? qrow[c * 8 + v] : make_uint4(0u, 0u, 0u, 0u);
-          w[4 * v] = x.x;
-          w[4 * v + 1] = x.y;
-          w[4 * v + 2] = x.z;
-          w[4 * v + 3] = x.w;
-        }
-        tmem_st32(tmem + lane_off + kColQ + c * 32, w);
+      for (int v = 0; v < 32; ++v) {
+        const uint4 x = row_ok ? qrow[v] : make_uint4(0u, 0u, 0u, 0u);
+        w[v >> 3][4 * (v & 7)] = x.x;
+        w[v >> 3][4 * (v & 7) + 1] = x.y;
+        w[v >> 3][4 * (v & 7) + 2] = x.z;
+        w[v >> 3][4 * (v & 7) + 3] = x.w;
       }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st32(tmem + lane_off + kColQ + c * 32, w[c]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

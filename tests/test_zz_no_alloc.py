@@ -45,12 +45,12 @@ def _params(d, q, k, v, max_k):
                            head_dim_v=v.shape[2], softmax_scale=d.softmax_scale, causal=True)
 
 
-@pytest.mark.parametrize("num_splits", [0, 5])
-def test_noalloc_decode_matches_workspace_decode_twice(num_splits):
+@pytest.mark.parametrize("num_splits,dim", [(0, 128), (5, 128), (0, 256)])
+def test_noalloc_decode_matches_workspace_decode_twice(num_splits, dim):
     import torch
     import softmax_attn_sink_b200 as sab
     f = _noalloc_fn()
-    d = W.random_decode(41, [3000, 1, 777, 5000], hq=16, hkv=2, dk=128, dv=128)
+    d = W.random_decode(41, [3000, 1, 777, 5000], hq=16, hkv=2, dk=dim, dv=dim)
     q, k, v, cu, sink = _inputs(d)
     max_k = 5000
     ref_out, ref_lse = sab.attn_sink_decode(q, k, v, cu, max_k, sink, d.softmax_scale, True,
