@@ -30,6 +30,7 @@
 #include <type_traits>
 
 #include "sm100_ptx.cuh"
+#include "tma_map.h"
 
 namespace attn_sink {
 namespace {
@@ -746,36 +747,6 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
 
 // ---- host ------------------------------------------------------------------------------------
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [rows, heads, 256] of 16-bit elements as a 3-D tensor; boxes of `box_rows` rows x 1 head x
-// 64 columns (128 bytes), 128-byte swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap* map, const void* base, int heads, int rows, int box_rows, CUtensorMapDataType dt) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * heads};
-  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 long long dq_grid(const BwdArgs& a) { return (long long)((a.max_sq + dq::kBM - 1) / dq::kBM) * a.batch * a.hq; }
 long long ks_grid(const BwdArgs& a) { return (long long)((a.max_sk + ks::kBN - 1) / ks::kBN) * a.batch * a.hkv; }
 
@@ -791,12 +762,11 @@ int band_of(const BwdArgs& a, long long per_group) {
 
 template <typename T>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
-  constexpr CUtensorMapDataType dt =
-      std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap q64, o64, o128, k64, v64, v128;
-  if (!make_map(&q64, a.q, a.hq, a.total_q, 64, dt) || !make_map(&o64, a.dout, a.hq, a.total_q, 64, dt) ||
-      !make_map(&o128, a.dout, a.hq, a.total_q, 128, dt) || !make_map(&k64, a.k, a.hkv, a.total_k, 64, dt) ||
-      !make_map(&v64, a.v, a.hkv, a.total_k, 64, dt) || !make_map(&v128, a.v, a.hkv, a.total_k, 128, dt))
+  if (!make_map_3d(&q64, a.q, D, a.hq, a.total_q, 64, dt) || !make_map_3d(&o64, a.dout, D, a.hq, a.total_q, 64, dt) ||
+      !make_map_3d(&o128, a.dout, D, a.hq, a.total_q, 128, dt) || !make_map_3d(&k64, a.k, D, a.hkv, a.total_k, 64, dt) ||
+      !make_map_3d(&v64, a.v, D, a.hkv, a.total_k, 64, dt) || !make_map_3d(&v128, a.v, D, a.hkv, a.total_k, 128, dt))
     return cudaErrorInvalidValue;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(bwd_dq_d256_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::kSmem)) ||

@@ -27,6 +27,7 @@
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
+#include "tma_map.h"
 
 namespace attn_sink {
 
@@ -900,39 +901,6 @@ __global__ void dq_convert_hmajor_kernel(const float* __restrict__ acc, T* __res
   reinterpret_cast<uint4*>(dq)[i] = o;
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [rows, heads, d] of 16-bit elements as a 3-D tensor; boxes of 128 rows x 1 head x 64
-// columns, 128B swizzle.
-bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows, CUtensorMapDataType dt) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * heads};
-  const cuuint32_t box[3] = {64, 1, 128};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <typename T> constexpr CUtensorMapDataType tma_dtype();
-template <> constexpr CUtensorMapDataType tma_dtype<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
-template <> constexpr CUtensorMapDataType tma_dtype<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
 template <typename T> constexpr int dtype_code();
 template <> constexpr int dtype_code<__nv_bfloat16>() { return 0; }
 template <> constexpr int dtype_code<__half>() { return 2; }
@@ -942,8 +910,8 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   using L = PLayout<DV>;
   constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, a.q, 128, a.hq, a.total_q, dt) || !make_map(&tk, a.k, 128, a.hkv, a.total_k, dt) ||
-      !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
+  if (!make_map_3d(&tq, a.q, 128, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, 128, a.hkv, a.total_k, 128, dt) ||
+      !make_map_3d(&tv, a.v, DV, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DV, a.hq, a.total_q, 128, dt))
     return cudaErrorInvalidValue;
   const bool dq = a.dq_acc != nullptr;
   cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * 128 * sizeof(float), s) : cudaSuccess;
@@ -970,8 +938,8 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   using L = BLayout<DK, DV>;
   constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
-      !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt) || !make_map(&to, a.dout, DV, a.hq, a.total_q, dt))
+  if (!make_map_3d(&tq, a.q, DK, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, DK, a.hkv, a.total_k, 128, dt) ||
+      !make_map_3d(&tv, a.v, DV, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DV, a.hq, a.total_q, 128, dt))
     return cudaErrorInvalidValue;
   const bool dq = a.dq_acc != nullptr;
   cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * DK * sizeof(float), s) : cudaSuccess;

@@ -27,6 +27,7 @@
 #include <type_traits>
 
 #include "sm100_ptx.cuh"
+#include "tma_map.h"
 
 namespace attn_sink {
 namespace {
@@ -380,36 +381,6 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
 
 // ---- host ----------------------------------------------------------------------------------
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [rows, heads, 256] of 16-bit elements as a 3-D tensor; boxes of 64 rows x 1 head x 64
-// columns (128 bytes), 128-byte swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap* map, const void* base, int heads, int rows, CUtensorMapDataType dt) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * heads};
-  const cuuint32_t box[3] = {64, 1, kBN};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 long long grid_of(const FwdArgs& a) {
   const long long zmax = (a.max_sq + kBM - 1) / kBM;
   return zmax * a.batch * a.hq;
@@ -419,10 +390,9 @@ template <typename T>
 cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   const int zmax = (a.max_sq + kBM - 1) / kBM;
   if (zmax <= 0) return cudaSuccess;
-  constexpr CUtensorMapDataType dt =
-      std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tk, tv;
-  if (!make_map(&tk, a.k, a.hkv, a.total_k, dt) || !make_map(&tv, a.v, a.hkv, a.total_k, dt))
+  if (!make_map_3d(&tk, a.k, D, a.hkv, a.total_k, kBN, dt) || !make_map_3d(&tv, a.v, D, a.hkv, a.total_k, kBN, dt))
     return cudaErrorInvalidValue;
   auto kernel = a.drop.threshold ? fwd_d256_sm100_kernel<T, true> : fwd_d256_sm100_kernel<T, false>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);

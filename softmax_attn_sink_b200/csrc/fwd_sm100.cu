@@ -37,6 +37,7 @@
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
+#include "tma_map.h"
 
 namespace attn_sink {
 namespace {
@@ -732,36 +733,6 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
 
 // ---- host: tensor maps and launch ----------------------------------------------------------
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [rows, heads, d] of 16-bit elements viewed as a 3-D tensor (d innermost); boxes of 128 rows x
-// 1 head x 64 columns (128 bytes), 128-byte swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap* map, const void* base, int d, int heads, int rows, CUtensorMapDataType dt) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * heads};
-  const cuuint32_t box[3] = {64, 1, 128};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Multiprocessors and opt-in shared memory per block of the current device (cached per device).
 struct DeviceShape {
   int sms = 0, smem_optin = 0;
@@ -795,9 +766,6 @@ void schedule_shape(const FwdArgs& a, int& zmax, int& width) {
   width = even ? a.hq / 2 : a.hq;
 }
 
-template <typename T> constexpr CUtensorMapDataType tma_dtype();
-template <> constexpr CUtensorMapDataType tma_dtype<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
-template <> constexpr CUtensorMapDataType tma_dtype<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
 
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
@@ -810,8 +778,8 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv;
   constexpr CUtensorMapDataType dt = tma_dtype<T>();
-  if (!make_map(&tq, a.q, DK, a.hq, a.total_q, dt) || !make_map(&tk, a.k, DK, a.hkv, a.total_k, dt) ||
-      !make_map(&tv, a.v, DV, a.hkv, a.total_k, dt))
+  if (!make_map_3d(&tq, a.q, DK, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, DK, a.hkv, a.total_k, 128, dt) ||
+      !make_map_3d(&tv, a.v, DV, a.hkv, a.total_k, 128, dt))
     return cudaErrorInvalidValue;
   // Persistent launch (one CTA per SM walking the item list) when the item table fits in
   // shared memory; otherwise one CTA per item of the dense (level, sequence, unit pair) grid.
