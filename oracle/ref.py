@@ -355,22 +355,28 @@ def merge_partials(parts, sink_h: float) -> Tuple[np.ndarray, float]:
 # --- sampled checks at full size ------------------------------------------------------
 
 def fwd_rows(q, k, v, cu_seqlens_q, cu_seqlens_k, sink, softmax_scale: float, causal: bool,
-             window_left: int, window_right: int, b: int, h: int, rows: Sequence[int]):
+             window_left: int, window_right: int, b: int, h: int, rows: Sequence[int], dropout=None):
     """out [len(rows), dv] and lse [len(rows)] for chosen query rows (sequence-local
-    indices) of sequence b, q head h; identical arithmetic to ``fwd``."""
+    indices) of sequence b, q head h; identical arithmetic to ``fwd`` (dropout included:
+    the keep decisions of exactly those packed rows)."""
     q0, q1 = _seq_ranges(cu_seqlens_q, b)
     k0, k1 = _seq_ranges(cu_seqlens_k, b)
     hq, hkv = q.shape[1], k.shape[1]
     g = h // (hq // hkv)
     rows = np.asarray(rows, dtype=np.int64)
     full = allowed_mask(q1 - q0, k1 - k0, causal, window_left, window_right)
+    drop = None
+    if dropout is not None:
+        p, seed, offset = dropout
+        t = dropout_threshold(p)
+        drop = dropout_keep(seed, offset, t, q0 + rows, h, k1 - k0) * (256.0 / t)
     r = attend_head(_f64(q[q0 + rows, h]), _f64(k[k0:k1, g]), _f64(v[k0:k1, g]),
-                    _sink_of(sink, h), softmax_scale, full[rows])
+                    _sink_of(sink, h), softmax_scale, full[rows], drop)
     return r["out"], r["lse"]
 
 
 def bwd_sequence_group(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, sink, softmax_scale: float,
-                       causal: bool, window_left: int, window_right: int, b: int, g: int):
+                       causal: bool, window_left: int, window_right: int, b: int, g: int, dropout=None):
     """Backward restricted to sequence b and kv head g (all q heads of its group).
 
     Returns dq [sq, G, dk] for those q heads, dk [sk, dk] and dv [sk, dv] of kv head g,
@@ -387,7 +393,7 @@ def bwd_sequence_group(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, sink, softmax_
     for hh in range(group):
         h = g * group + hh
         r = bwd_head(q[q0:q1, h], k[k0:k1, g], v[k0:k1, g], dout[q0:q1, h], _sink_of(sink, h),
-                     softmax_scale, mask)
+                     softmax_scale, mask, _drop_weights(dropout, q0, q1, h, k1 - k0))
         dq[:, hh] = r["dq"]
         dk += r["dk"]
         dv += r["dv"]

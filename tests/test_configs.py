@@ -90,6 +90,39 @@ def test_config3_training_fwd_bwd_sampled():
     check_grad(to_np(ds)[g:g + 1], np.array([total]), "bf16", "dsink")
 
 
+def test_config3_training_with_dropout_sampled():
+    """The training workload with dropout p = 0.1 at full size: sampled forward rows and one
+    whole (sequence, head) of the backward (dsink with dropout is checked on the small cases
+    of test_dropout.py: its oracle needs every row's keep bytes of the head)."""
+    p = W.config3()
+    drop = (0.1, 0x5EED5EED1234ABCD, 3)
+    td = torch.bfloat16
+    q, k, v, do = dev(p.q, td), dev(p.k, td), dev(p.v, td), dev(p.dout, td)
+    cu = dev(p.cu_seqlens_q)
+    sink = dev(p.sink)
+    out, lse = sab.attn_sink_fwd(q, k, v, cu, cu, 8192, 8192, sink, p.softmax_scale, True, dropout=drop)
+    dq, dk, dv, ds = sab.attn_sink_bwd(q, k, v, out, do, lse, cu, cu, 8192, 8192, sink,
+                                       p.softmax_scale, True, dropout=drop)
+    torch.cuda.synchronize()
+    o, l = to_np(out), to_np(lse)
+    a = (p.cu_seqlens_q, p.cu_seqlens_k, p.sink, p.softmax_scale, True, -1, -1)
+    s = 256.0 / ref.dropout_threshold(drop[0])
+    rng = np.random.default_rng(102)
+    for b in (0, 3):
+        for h in (2, 11):
+            rows = _sample_rows(8192, rng)
+            ro, rl = ref.fwd_rows(p.q, p.k, p.v, *a, b=b, h=h, rows=rows, dropout=drop)
+            idx = np.asarray(rows) + 8192 * b
+            check_out(o[idx, h] / s, ro / s, "bf16", f"out[b={b},h={h}]")
+            check_lse(l[h, idx], rl, "bf16", f"lse[b={b},h={h}]")
+    b, g = 2, 9
+    gq, gk, gv, gs = ref.bwd_sequence_group(p.q, p.k, p.v, p.dout, *a, b=b, g=g, dropout=drop)
+    sl = slice(8192 * b, 8192 * (b + 1))
+    check_grad(to_np(dq[sl, g]), gq[:, 0], "bf16", "dq")
+    check_grad(to_np(dk[sl, g]), gk, "bf16", "dk")
+    check_grad(to_np(dv[sl, g]), gv, "bf16", "dv")
+
+
 @pytest.mark.parametrize("n", [1.0, 0.5, 3.0])
 def test_config4_softmax_n_window(n):
     p = W.config4(n)

@@ -536,6 +536,26 @@ def test_p14_threshold_rounds_halves_up_from_the_float_p():
     assert ref.dropout_threshold(p) == 230
 
 
+def test_p14_sampled_helpers_follow_fwd_and_bwd_with_dropout():
+    """fwd_rows and bwd_sequence_group with dropout reproduce the rows and the (sequence, kv
+    head) slice of fwd / bwd with the same dropout (the helpers used on full-size problems)."""
+    p = W.random_problem(77, [40, 57], [50, 57], 4, 2, 8, 6, True, 20, 0, with_dout=True)
+    a = (p.cu_seqlens_q, p.cu_seqlens_k, p.sink, p.softmax_scale, True, 20, 0)
+    drop = (0.3, 12345, 6)
+    ro, rl = ref.fwd(p.q, p.k, p.v, *a, dropout=drop)
+    rows = [0, 3, 17, 56]
+    o, l = ref.fwd_rows(p.q, p.k, p.v, *a, b=1, h=3, rows=rows, dropout=drop)
+    assert np.allclose(o, ro[40 + np.asarray(rows), 3], rtol=0, atol=1e-14)
+    assert np.allclose(l, rl[3, 40 + np.asarray(rows)], rtol=0, atol=1e-14)
+    dq, dk, dv, ds = ref.bwd(p.q, p.k, p.v, p.dout, *a, dropout=drop)
+    gq, gk, gv, gs = ref.bwd_sequence_group(p.q, p.k, p.v, p.dout, *a, b=1, g=1, dropout=drop)
+    assert np.allclose(gq, dq[40:97, 2:4], atol=1e-13)
+    assert np.allclose(gk, dk[50:107, 1], atol=1e-13) and np.allclose(gv, dv[50:107, 1], atol=1e-13)
+    # dsink of a head sums its sequences: the slice's part plus sequence 0's
+    g0 = ref.bwd_sequence_group(p.q, p.k, p.v, p.dout, *a, b=0, g=1, dropout=drop)[3]
+    assert np.allclose(gs + g0, ds[2:4], atol=1e-13)
+
+
 def test_p14_no_dropout_is_identity():
     """p = 0 (T = 256) gives exactly the forward and backward without dropout."""
     p = W.random_problem(140, [9, 5], [11, 5], 4, 2, 8, 6, True, dtype="fp32", with_dout=True)
