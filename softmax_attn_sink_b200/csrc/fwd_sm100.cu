@@ -696,24 +696,34 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       const long long grow = (long long)q0 + i;   // packed row of this thread's query
       T* out = static_cast<T*>(a.out);
       uint4* orow = reinterpret_cast<uint4*>(out + (grow * a.hq + h) * DV);
+      // The O row in as few TMEM round trips as the registers allow (this is on the unit's
+      // path to its next item): all of it at once, or 32 columns at a time with dropout,
+      // whose flag words take the room.
+      constexpr int kChunks = DV / 32, kPer = DROP ? 1 : kChunks;
 #pragma unroll
-      for (int c = 0; c < DV / 32; ++c) {
-        uint32_t o[32];
+      for (int c0 = 0; c0 < kChunks; c0 += kPer) {
+        uint32_t o[kPer][32];
         if (have_o) {
-          tmem_ld32(tO + c * 32, o);
+#pragma unroll
+          for (int c = 0; c < kPer; ++c) tmem_ld32(tO + (c0 + c) * 32, o[c]);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
+          for (int c = 0; c < kPer; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[c][e] = 0u;
         }
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack2<T>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        if (row_ok) {
+        for (int c = 0; c < kPer; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            orow[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack2<T>(__uint_as_float(o[c][2 * e]) * inv, __uint_as_float(o[c][2 * e + 1]) * inv);
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              orow[(c0 + c) * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
       }
       if (row_ok && a.lse)
