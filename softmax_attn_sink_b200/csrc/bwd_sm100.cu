@@ -400,8 +400,7 @@ constexpr int kRegsLow = 136, kRegsHigh = 184;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreadsP * 168, "register split");
 
 template <int DV>
-struct PLayout {
-  static constexpr int DK = 128;
+struct PLayout {   // head dim 128: K and Q tiles are two 64-column boxes
   static constexpr int VH = DV / 64;
   static constexpr int kHalf = 128 * 128;
   static constexpr int kKBytes = 2 * kHalf, kVBytes = VH * kHalf;

@@ -2,7 +2,6 @@
 times.  Small configs are compared element by element; large ones on sampled rows
 (and, for the backward, one whole (sequence, head) plus the full dsink of one head),
 each sample computed by the oracle one by one."""
-import math
 
 import numpy as np
 import pytest

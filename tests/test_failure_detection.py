@@ -3,7 +3,6 @@ time limit and report a timeout through a per-device status word instead of hang
 diagnostics entry point makes one such wait run out on purpose (a barrier nothing
 completes); the host reads the timeout, and the same context then still computes correct
 results."""
-import numpy as np
 import pytest
 
 import workloads as W

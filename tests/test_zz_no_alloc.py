@@ -9,7 +9,6 @@ second call reuses the array the first one left behind).  The file name sorts la
 that a run stopping at the first failure has already run every other test."""
 import ctypes
 
-import numpy as np
 import pytest
 
 import workloads as W
