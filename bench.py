@@ -431,6 +431,12 @@ def bench_fwd_d256(args, world, peaks, peak_kind):
                                                           True, dq=dq, dk=dk, dv=dv, dsink=dsink),
                                 3, 1, world, flush)
     ba = bflops / (statistics.mean(b_per) * 1e-3) / 1e12
+    # the same backward with dropout p = 0.1 (the forward's keep bytes redrawn)
+    sab.attn_sink_fwd(q, k, v, cu, cu, mx, mx, sink, 1.0 / 16.0, True, out=out, lse=lse, dropout=DROPOUT)
+    bd_per, bd_total = time_steps(lambda: sab.attn_sink_bwd(q, k, v, out, do, lse, cu, cu, mx, mx, sink, 1.0 / 16.0,
+                                                            True, dq=dq, dk=dk, dv=dv, dsink=dsink, dropout=DROPOUT),
+                                  3, 1, world, flush)
+    bda = bflops / (statistics.mean(bd_per) * 1e-3) / 1e12
     # decode: 16 sequences of the decode workload's lengths, 32 q / 4 kv heads at d = 256
     dl = W.config5_meta().cu_seqlens_k
     dlens = np.diff(dl)[:16]
@@ -459,7 +465,11 @@ def bench_fwd_d256(args, world, peaks, peak_kind):
                     "ms_per_step": round(b_total / 3, 3), "flops": bflops, "steps": 3,
                     "roofline": {"bound": "tensor", "achieved": round(ba, 2), "peak": pk, "unit": "TFLOP/s",
                                  "frac": round(ba / pk, 4), "traffic": None,
-                                 "kernels": "preprocess + CUDA-core dK/dV + CUDA-core dQ"}},
+                                 "kernels": "preprocess + tcgen05 dQ + dK + dV"}},
+            "bwd_dropout": {"value": round(bflops * world / (bd_total / 3 * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                            "ms_per_step": round(bd_total / 3, 3), "flops": bflops, "steps": 3, "dropout": [DROPOUT[0]],
+                            "roofline": {"bound": "tensor", "achieved": round(bda, 2), "peak": pk, "unit": "TFLOP/s",
+                                         "frac": round(bda / pk, 4), "traffic": None}},
             "decode": {"workload": "decode16_gqa32x4_d256_L8k-32k", "value": round(dbytes * world / (d_total / steps * 1e-3) / 1e9, 1),
                        "unit": "GB/s", "ms_per_step": round(d_total / steps, 4), "bytes_per_step": dbytes,
                        "roofline": {"bound": "hbm", "achieved": round(da, 1), "peak": pb, "unit": "GB/s",

@@ -126,7 +126,7 @@ struct Bars {
 };
 }  // namespace dq
 
-template <typename T>
+template <typename T, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_d256_kernel(const BwdArgs a, int mtiles, int band, const __grid_constant__ CUtensorMap tm_o,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -154,7 +154,9 @@ bwd_dq_d256_kernel(const BwdArgs a, int mtiles, int band, const __grid_constant_
   long long l1, h1, l2, h2;
   row_key_range(m0, sq, sk, a.left, a.right, l1, h1);
   row_key_range(m0 + nrows - 1, sq, sk, a.left, a.right, l2, h2);
-  const int lo = (int)l1, hi = (int)(h2 < l1 ? l1 : h2);
+  int lo = (int)l1;
+  const int hi = (int)(h2 < l1 ? l1 : h2);
+  if (DROP && hi > lo) lo &= ~15;   // dropout draws keep bytes for 16-key blocks
   const int n = hi > lo ? (hi - lo + kBN - 1) / kBN : 0;
 
   const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -265,8 +267,23 @@ bwd_dq_d256_kernel(const BwdArgs a, int mtiles, int band, const __grid_constant_
       Dr = a.D[idx];
     }
     const float scale2 = a.scale * kLog2e;
+    const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
+      // dropout: drop flags of this row's 64 keys of the tile (4 Philox calls, drawn before
+      // the wait so that they overlap the tensor pipe); dS = P (Z dP - D)
+      uint32_t fl[DROP ? 16 : 1];
+      if constexpr (DROP) {
+        const uint32_t kb0 = (uint32_t)(lo + j * kBN) >> 4;
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+          const uint4 w = dropout_bytes(a.drop, kb0 + gq, (uint32_t)(q0 + i), (uint32_t)h);
+          fl[4 * gq] = drop_flags4(w.x, t4, t4h);
+          fl[4 * gq + 1] = drop_flags4(w.y, t4, t4h);
+          fl[4 * gq + 2] = drop_flags4(w.z, t4, t4h);
+          fl[4 * gq + 3] = drop_flags4(w.w, t4, t4h);
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(bar.sdp_full(), j & 1, a.status))) { ok = false; break; }
       tc_fence_after();
       const int klo = rlo - j * kBN, khi = rhi - j * kBN;   // visible columns [klo, khi)
@@ -283,7 +300,16 @@ bwd_dq_d256_kernel(const BwdArgs a, int mtiles, int band, const __grid_constant_
           const float s0 = (c0 >= klo && c0 < khi) ? __uint_as_float(sv[2 * e]) : kNegInf;
           const float s1 = (c0 + 1 >= klo && c0 + 1 < khi) ? __uint_as_float(sv[2 * e + 1]) : kNegInf;
           const float p0 = ex2(fmaf(s0, scale2, neg_lt)), p1 = ex2(fmaf(s1, scale2, neg_lt));
-          pk[e] = pack2<T>(p0 * (__uint_as_float(pv[2 * e]) - Dr), p1 * (__uint_as_float(pv[2 * e + 1]) - Dr));
+          if constexpr (DROP) {
+            // keys c0, c0 + 1: bytes 0-1 (e even) or 2-3 (e odd) of flag word c0 / 4
+            const uint32_t w = fl[c0 >> 2];
+            const uint32_t d0 = (e & 1) ? prmt_sign<0xAAAA>(w) : prmt_sign<0x8888>(w);
+            const uint32_t d1 = (e & 1) ? prmt_sign<0xBBBB>(w) : prmt_sign<0x9999>(w);
+            pk[e] = pack2<T>(p0 * fmaf(__uint_as_float(pv[2 * e] & ~d0), a.drop.scale, -Dr),
+                             p1 * fmaf(__uint_as_float(pv[2 * e + 1] & ~d1), a.drop.scale, -Dr));
+          } else {
+            pk[e] = pack2<T>(p0 * (__uint_as_float(pv[2 * e]) - Dr), p1 * (__uint_as_float(pv[2 * e + 1]) - Dr));
+          }
         }
         // dS of keys [32 c, 32 c + 32) over S columns [16 c, 16 c + 16), already read
         tmem_st16(tmem + lane_off + kColS + c * 16, pk);
@@ -348,6 +374,60 @@ __device__ __forceinline__ bool tile_of(const BwdArgs& a, int ntiles, int band, 
   t.T = t.n_m * (a.hq / a.hkv);
   return true;
 }
+// Dropout in the key-stationary kernels: a compute thread owns a key, but a Philox call gives
+// the keep bytes of 16 keys for one query.  Warps 2-3 draw the 512 calls of a 64-query x
+// 128-key tile (thread rt: key block rt / 8, queries u + 16 k for u in {rt % 8, rt % 8 + 8},
+// k = 0..3), turn them into drop flags (bit 7 of a byte set = dropped) and write them
+// transposed into a two-stage buffer: word [block][key tk][u] holds, in byte k, the flag of
+// query u + 16 k for key 16 block + tk.  Producer and compute warps meet on named barrier
+// 3 + t % 2 once per tile (64 + 128 threads); the producer passes the barrier of tile t - 1
+// only after the compute warps are done with tile t - 2, whose stage tile t reuses.
+constexpr int kZBlockWords = 16 * 16 + 16;   // + 16 words: blocks 2w, 2w+1 in other banks
+constexpr int kZBytes = 4 * 8 * kZBlockWords;
+__device__ __forceinline__ void draw_flags(const BwdArgs& a, uint32_t zbuf, int rt, int n0, long long row0, int h) {
+  const int blk = rt >> 3, u0 = rt & 7;
+  const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
+  uint32_t fw[2][16];   // [u half][4 k + word]
+#pragma unroll
+  for (int uh = 0; uh < 2; ++uh)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 w = dropout_bytes(a.drop, (uint32_t)((n0 >> 4) + blk), (uint32_t)(row0 + u0 + 8 * uh + 16 * k),
+                                    (uint32_t)h);
+      fw[uh][4 * k] = drop_flags4(w.x, t4, t4h);
+      fw[uh][4 * k + 1] = drop_flags4(w.y, t4, t4h);
+      fw[uh][4 * k + 2] = drop_flags4(w.z, t4, t4h);
+      fw[uh][4 * k + 3] = drop_flags4(w.w, t4, t4h);
+    }
+#pragma unroll
+  for (int uh = 0; uh < 2; ++uh)
+#pragma unroll
+    for (int tk = 0; tk < 16; ++tk) {
+      // flag byte of key tk of query u + 16 k is byte tk % 4 of fw[uh][4 k + tk / 4]
+      const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
+      const uint32_t lo2 = __byte_perm(fw[uh][tk >> 2], fw[uh][4 + (tk >> 2)], sel);
+      const uint32_t hi2 = __byte_perm(fw[uh][8 + (tk >> 2)], fw[uh][12 + (tk >> 2)], sel);
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(zbuf + 4u * (blk * kZBlockWords + tk * 16 + u0 + 8 * uh)),
+                   "r"(__byte_perm(lo2, hi2, 0x5410))
+                   : "memory");
+    }
+}
+
+// The 16 flag words of key r of a tile (word u: queries u + 16 k in byte k).
+__device__ __forceinline__ void read_flags(uint32_t zbuf, int r, uint32_t (&zb)[16]) {
+  const uint32_t src = zbuf + 4u * ((r >> 4) * kZBlockWords + (r & 15) * 16);
+#pragma unroll
+  for (int v4 = 0; v4 < 4; ++v4)
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(zb[4 * v4]), "=r"(zb[4 * v4 + 1]), "=r"(zb[4 * v4 + 2]), "=r"(zb[4 * v4 + 3])
+                 : "r"(src + 16u * v4)
+                 : "memory");
+}
+
+// Drop mask (all ones if dropped) of query q (0..63) of the tile from the key's flag words.
+__device__ __forceinline__ uint32_t drop_mask(const uint32_t (&zb)[16], int q) {
+  return prmt_sign_r(zb[q & 15], (8u | (uint32_t)(q >> 4)) * 0x1111u);
+}
 }  // namespace ks
 
 // ---- dV --------------------------------------------------------------------------------------
@@ -356,7 +436,8 @@ constexpr int kStages = 3;
 constexpr int kOffQ = 0;                           // Q ring
 constexpr int kOffO = kOffQ + kStages * kTile64;   // dout ring
 constexpr int kOffLT = kOffO + kStages * kTile64;  // -lse_tot log2e of the tile's queries [2][64]
-constexpr int kOffBar = kOffLT + 2 * 64 * 4;
+constexpr int kOffZ = kOffLT + 2 * 64 * 4;         // dropout flags, 2 stages
+constexpr int kOffBar = kOffZ + 2 * ks::kZBytes;
 constexpr int kNumBars = 1 + 2 * kStages + 6;      // k_full, qd_full[S], qd_empty[S], s_full[2], p_full[2], dv_done, drain
 constexpr int kOffSlot = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffSlot + 16 + 1024;
@@ -374,7 +455,7 @@ struct Bars {
 };
 }  // namespace dvk
 
-template <typename T>
+template <typename T, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_o) {
@@ -391,6 +472,7 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
   unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
   const uint32_t sQ = base_u32 + kOffQ, sO = base_u32 + kOffO;
   float* s_nlt = reinterpret_cast<float*>(smem + kOffLT);
+  const uint32_t sZ = base_u32 + kOffZ;
   const Bars bar{base_u32 + kOffBar};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -473,6 +555,13 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
       mma_commit(bar.drain());
       mbar_wait(bar.drain(), 0, a.status);
     }
+  } else if (DROP && warp < 4) {
+    // warps 2-3: the dropout flags of every tile, a tile ahead of the compute warps
+    const int rt = (warp - 2) * 32 + lane;
+    for (int t = 0; t < T_; ++t) {
+      ks::draw_flags(a, sZ + (t & 1) * ks::kZBytes, rt, tl.n0, (long long)tl.q0 + qbase_of(t), head_of(t));
+      named_bar_sync(3 + (t & 1), 192);
+    }
   } else if (warp >= 4) {
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
@@ -499,11 +588,14 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
       named_bar_sync(1, 128);   // buffer t & 1 was last read in tile t - 2
       if (t + 1 < T_) pf = fetch(t + 1);
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar.s_full(t & 1), (t >> 1) & 1, a.status));
-      if (!ok) continue;   // keep passing the named barrier with the other warps
+      if constexpr (DROP) named_bar_sync(3 + (t & 1), 192);   // this tile's flags are written
+      if (!ok) continue;   // keep passing the named barriers with the other warps
       tc_fence_after();
       const int c_lo = jlo - qbase_of(t), c_hi = jhi - qbase_of(t);   // visible columns
       const uint32_t tS = tmem + lane_off + col_S(t & 1);
       const float* nl = s_nlt + (t & 1) * kBM;
+      uint32_t zb[DROP ? 16 : 1];
+      if constexpr (DROP) ks::read_flags(sZ + (t & 1) * ks::kZBytes, r, zb);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
@@ -516,7 +608,12 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
           const float2 n2 = *reinterpret_cast<const float2*>(nl + c0);
           const float s0 = (c0 >= c_lo && c0 < c_hi) ? __uint_as_float(sv[2 * e]) : kNegInf;
           const float s1 = (c0 + 1 >= c_lo && c0 + 1 < c_hi) ? __uint_as_float(sv[2 * e + 1]) : kNegInf;
-          pk[e] = pack2<T>(ex2(fmaf(s0, scale2, n2.x)), ex2(fmaf(s1, scale2, n2.y)));
+          float p0 = ex2(fmaf(s0, scale2, n2.x)), p1 = ex2(fmaf(s1, scale2, n2.y));
+          if constexpr (DROP) {   // dV takes the kept probabilities (256 / T is applied to dV)
+            p0 = __uint_as_float(__float_as_uint(p0) & ~ks::drop_mask(zb, c0));
+            p1 = __uint_as_float(__float_as_uint(p1) & ~ks::drop_mask(zb, c0 + 1));
+          }
+          pk[e] = pack2<T>(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);   // P^T over S^T columns already read
       }
@@ -529,7 +626,7 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
     if (have) have = __all_sync(0xffffffffu, mbar_wait(bar.dv_done(), 0, a.status));
     tc_fence_after();
     if (ok)
-      store_row<T>(tmem + lane_off + kColDV, have, 1.f,
+      store_row<T>(tmem + lane_off + kColDV, have, DROP ? a.drop.scale : 1.f,
                    static_cast<T*>(a.grad_v) + ((long long)(tl.k0 + j) * a.hkv + tl.g) * D, key_ok);
   }
   tc_fence_before();
@@ -548,7 +645,8 @@ constexpr int kOffV = 0;                           // V, 4 boxes of 128 rows
 constexpr int kOffQ = kOffV + kTile128;            // Q ring
 constexpr int kOffO = kOffQ + kStages * kTile64;   // dout ring
 constexpr int kOffLT = kOffO + kStages * kTile64;  // -lse_tot log2e [2][64], D [2][64]
-constexpr int kOffBar = kOffLT + 4 * 64 * 4;
+constexpr int kOffZ = kOffLT + 4 * 64 * 4;         // dropout flags, 2 stages
+constexpr int kOffBar = kOffZ + 2 * ks::kZBytes;
 constexpr int kNumBars = 2 + 2 * kStages + 4;      // k_full, v_full, qd_full[S], qd_empty[S], sdp_full, ds_full, dk_done, drain
 constexpr int kOffSlot = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffSlot + 16 + 1024;
@@ -566,7 +664,7 @@ struct Bars {
 };
 }  // namespace dkk
 
-template <typename T>
+template <typename T, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_v) {
@@ -584,6 +682,7 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
   const uint32_t sV = base_u32 + kOffV, sQ = base_u32 + kOffQ, sO = base_u32 + kOffO;
   float* s_nlt = reinterpret_cast<float*>(smem + kOffLT);
   float* s_D = s_nlt + 2 * kBM;
+  const uint32_t sZ = base_u32 + kOffZ;
   const Bars bar{base_u32 + kOffBar};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -667,6 +766,13 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
       mma_commit(bar.drain());
       mbar_wait(bar.drain(), 0, a.status);
     }
+  } else if (DROP && warp < 4) {
+    // warps 2-3: the dropout flags of every tile, a tile ahead of the compute warps
+    const int rt = (warp - 2) * 32 + lane;
+    for (int t = 0; t < T_; ++t) {
+      ks::draw_flags(a, sZ + (t & 1) * ks::kZBytes, rt, tl.n0, (long long)tl.q0 + qbase_of(t), head_of(t));
+      named_bar_sync(3 + (t & 1), 192);
+    }
   } else if (warp >= 4) {
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
@@ -700,11 +806,14 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
       named_bar_sync(1, 128);   // buffer t & 1 was last read in tile t - 2
       if (t + 1 < T_) fetch(t + 1);
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar.sdp_full(), t & 1, a.status));
-      if (!ok) continue;   // keep passing the named barrier with the other warps
+      if constexpr (DROP) named_bar_sync(3 + (t & 1), 192);   // this tile's flags are written
+      if (!ok) continue;   // keep passing the named barriers with the other warps
       tc_fence_after();
       const int c_lo = jlo - qbase_of(t), c_hi = jhi - qbase_of(t);
       const float* nl = s_nlt + (t & 1) * kBM;
       const float* dd = s_D + (t & 1) * kBM;
+      uint32_t zb[DROP ? 16 : 1];
+      if constexpr (DROP) ks::read_flags(sZ + (t & 1) * ks::kZBytes, r, zb);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], pv[32];
@@ -720,7 +829,13 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
           const float s0 = (c0 >= c_lo && c0 < c_hi) ? __uint_as_float(sv[2 * e]) : kNegInf;
           const float s1 = (c0 + 1 >= c_lo && c0 + 1 < c_hi) ? __uint_as_float(sv[2 * e + 1]) : kNegInf;
           const float p0 = ex2(fmaf(s0, scale2, n2.x)), p1 = ex2(fmaf(s1, scale2, n2.y));
-          pk[e] = pack2<T>(p0 * (__uint_as_float(pv[2 * e]) - d2.x), p1 * (__uint_as_float(pv[2 * e + 1]) - d2.y));
+          if constexpr (DROP) {   // dS = P (Z dP - D)
+            const uint32_t m0 = ks::drop_mask(zb, c0), m1 = ks::drop_mask(zb, c0 + 1);
+            pk[e] = pack2<T>(p0 * fmaf(__uint_as_float(pv[2 * e] & ~m0), a.drop.scale, -d2.x),
+                             p1 * fmaf(__uint_as_float(pv[2 * e + 1] & ~m1), a.drop.scale, -d2.y));
+          } else {
+            pk[e] = pack2<T>(p0 * (__uint_as_float(pv[2 * e]) - d2.x), p1 * (__uint_as_float(pv[2 * e + 1]) - d2.y));
+          }
         }
         tmem_st16(tmem + lane_off + kColS + c * 16, pk);   // dS^T over S^T columns already read
       }
@@ -769,9 +884,13 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
       !make_map_3d(&v64, a.v, D, a.hkv, a.total_k, 64, dt) || !make_map_3d(&v128, a.v, D, a.hkv, a.total_k, 128, dt))
     return cudaErrorInvalidValue;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(bwd_dq_d256_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::kSmem)) ||
-      (e = cudaFuncSetAttribute(bwd_dv_d256_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dvk::kSmem)) ||
-      (e = cudaFuncSetAttribute(bwd_dk_d256_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dkk::kSmem)))
+  const bool drop = a.drop.threshold != 0;
+  auto kq = drop ? bwd_dq_d256_kernel<T, true> : bwd_dq_d256_kernel<T, false>;
+  auto kv = drop ? bwd_dv_d256_kernel<T, true> : bwd_dv_d256_kernel<T, false>;
+  auto kk = drop ? bwd_dk_d256_kernel<T, true> : bwd_dk_d256_kernel<T, false>;
+  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::kSmem)) ||
+      (e = cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, dvk::kSmem)) ||
+      (e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, dkk::kSmem)))
     return e;
   const int mtiles = (a.max_sq + dq::kBM - 1) / dq::kBM, ntiles = (a.max_sk + ks::kBN - 1) / ks::kBN;
   const int group = a.hq / a.hkv;
@@ -779,13 +898,13 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   const int band_q = band_of(a, (long long)(a.max_sk > 0 ? a.max_sk : 1) * 2 * D * 2);
   const int band_k = band_of(a, (long long)(a.max_sq > 0 ? a.max_sq : 1) * group * 2 * D * 2);
   if (mtiles > 0) {
-    bwd_dq_d256_kernel<T><<<(unsigned)dq_grid(a), kThreads, dq::kSmem, s>>>(a, mtiles, band_q, o128, k64, v64);
+    kq<<<(unsigned)dq_grid(a), kThreads, dq::kSmem, s>>>(a, mtiles, band_q, o128, k64, v64);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (ks_grid(a) > 0) {
-    bwd_dk_d256_kernel<T><<<(unsigned)ks_grid(a), kThreads, dkk::kSmem, s>>>(a, ntiles, band_k, q64, o64, v128);
+    kk<<<(unsigned)ks_grid(a), kThreads, dkk::kSmem, s>>>(a, ntiles, band_k, q64, o64, v128);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_dv_d256_kernel<T><<<(unsigned)ks_grid(a), kThreads, dvk::kSmem, s>>>(a, ntiles, band_k, q64, o64);
+    kv<<<(unsigned)ks_grid(a), kThreads, dvk::kSmem, s>>>(a, ntiles, band_k, q64, o64);
   }
   return cudaGetLastError();
 }
@@ -794,7 +913,7 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
 
 bool bwd_d256_sm100_supported(const BwdArgs& a, int dtype) {
   if (dtype != 0 && dtype != 2) return false;
-  if (a.dk != D || a.dv != D || a.drop.threshold) return false;
+  if (a.dk != D || a.dv != D) return false;
   if (dq_grid(a) > 0x7fffffffLL || ks_grid(a) > 0x7fffffffLL) return false;   // 1-D grids
   return encode_fn() != nullptr;
 }

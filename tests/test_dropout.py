@@ -83,10 +83,19 @@ BWD_CASES = [
 ]
 
 
+BWD_CASES += [
+    # head dim 256 (dk = dv = 256): the dQ / dK / dV kernels with dropout
+    ("d256_causal_gqa_p10", [1, 129, 0, 257], [1, 129, 0, 257], 4, 2, 256, True, -1, -1, "normal",
+     "bf16", 0.1),
+    ("d256_fp16_window_sq_ne_sk_p30", [200, 5], [230, 90], 2, 1, 256, True, 70, 0, "normal", "fp16", 0.3),
+]
+
+
 @pytest.mark.parametrize("case", BWD_CASES, ids=[c[0] for c in BWD_CASES])
 def test_bwd_dropout_matches_oracle(case):
     name, lq, lk, hq, hkv, dv, causal, wl, wr, sink, dtype, pdrop = case
-    p = W.random_problem(_seed(name) + 5, lq, lk, hq, hkv, 128, dv, causal, wl, wr, sink, dtype,
+    dk = 256 if dv == 256 else 128
+    p = W.random_problem(_seed(name) + 5, lq, lk, hq, hkv, dk, dv, causal, wl, wr, sink, dtype,
                          with_dout=True)
     drop = (pdrop, BIG_SEED ^ _seed(name), 3 + _seed(name))
     out, lse, dq, dk, dv_, ds = run_bwd(p, dropout=drop)
@@ -114,10 +123,10 @@ def _visible_pairs(p):
 
 
 def _structured(lens_q, lens_k, hq, hkv, causal, wl, wr, dtype, for_bwd, d=128):
-    """q = 0 (every visible key equally likely), sink = -inf.  Forward: v one-hot on key
-    position mod 128, so out[i, h, j % 128] = P Z for the one visible key j there.  Backward:
-    k one-hot on key position, v = 1, dout one-hot on query position, so dv[j, :, i % 128]
-    collects P Z of row i and dq[i, h, j % 128] = scale dS_ij."""
+    """q = 0 (every visible key equally likely), sink = -inf, head dim d.  Forward: v one-hot
+    on key position mod d, so out[i, h, j % d] = P Z for the one visible key j there.
+    Backward: k one-hot on key position, v = 1, dout one-hot on query position, so
+    dv[j, :, i % d] collects P Z of row i and dq[i, h, j % d] = scale dS_ij."""
     cu_q, cu_k = W.cu_from_lengths(lens_q), W.cu_from_lengths(lens_k)
     tq, tk = int(cu_q[-1]), int(cu_k[-1])
     q = np.zeros((tq, hq, d), np.float32)
@@ -175,22 +184,23 @@ def test_fwd_dropout_keep_mask_is_exact(case, d):
     assert bad.size == 0, f"{len(bad)} keep decisions differ; first (row, head, col) {bad[:5].tolist()}"
 
 
-@pytest.mark.parametrize("case", MASK_CASES[:2] + [
-    ("causal_fp16_dv_p30", [333, 129], [333, 140], 4, 2, True, 90, 0, "fp16", 0.3)],
-    ids=[c[0] for c in MASK_CASES[:2]] + ["causal_fp16_dv_p30"])
-def test_bwd_dropout_keep_mask_is_exact(case):
+@pytest.mark.parametrize("case,d", [(c, 128) for c in MASK_CASES[:2]] + [
+    (("causal_fp16_dv_p30", [333, 129], [333, 140], 4, 2, True, 90, 0, "fp16", 0.3), 128),
+    (("d256_two_sided_gqa_p20", [300, 517], [300, 517], 4, 2, False, 120, 120, "bf16", 0.2), 256)],
+    ids=[c[0] for c in MASK_CASES[:2]] + ["causal_fp16_dv_p30", "d256_two_sided_gqa_p20"])
+def test_bwd_dropout_keep_mask_is_exact(case, d):
     """dv carries the keep mask bit for bit; dq, the difference of kept and dropped terms,
     is checked element-wise within a tenth of the gap between the two."""
     name, lq, lk, hq, hkv, causal, wl, wr, dtype, pdrop = case
-    p = _structured(lq, lk, hq, hkv, causal, wl, wr, dtype, for_bwd=True)
+    p = _structured(lq, lk, hq, hkv, causal, wl, wr, dtype, for_bwd=True, d=d)
     drop = (pdrop, BIG_SEED ^ (_seed(name) << 40), 5)
     t = ref.dropout_threshold(pdrop)
     grp = hq // hkv
-    want_dv = np.zeros((int(p.cu_seqlens_k[-1]), hkv, 128), bool)
+    want_dv = np.zeros((int(p.cu_seqlens_k[-1]), hkv, d), bool)
     gap = np.zeros((int(p.cu_seqlens_q[-1]), hq, 1))
     for b, q0, q1, k0, k1, vis in _visible_pairs(p):
-        rows = np.arange(q1 - q0) % 128
-        for j in range(k1 - k0):   # a key is seen by at most 128 consecutive rows
+        rows = np.arange(q1 - q0) % d
+        for j in range(k1 - k0):   # a key is seen by at most d consecutive rows
             assert len(set(rows[vis[:, j]])) == int(vis[:, j].sum())
         n = np.maximum(vis.sum(axis=1), 1)
         for h in range(hq):
