@@ -147,8 +147,8 @@ int attn_sink_bwd(const attn_sink_params* params, const void* q, const void* k, 
 
 /*
  * Forward and backward with dropout (see attn_sink_dropout); otherwise the arguments of
- * attn_sink_fwd / attn_sink_bwd.  Tensor-core paths only: bf16 or fp16, and for the
- * backward head_dim_qk == 128 with head_dim_v in {64, 128}, or 256 / 256 (ATTN_SINK_ERR_UNSUPPORTED
+ * attn_sink_fwd / attn_sink_bwd.  Tensor-core paths only: bf16 or fp16 with head_dim_qk and
+ * head_dim_v in {64, 128}, or 256 / 256 (ATTN_SINK_ERR_UNSUPPORTED
  * otherwise; ATTN_SINK_ERR_INVALID_ARG for a NULL dropout or p out of range).  The backward
  * takes the deterministic path (bit-identical results from run to run) and the workspace
  * attn_sink_bwd_workspace_size() gives.

@@ -221,7 +221,7 @@ int run_bwd(const attn_sink_params* p, const void* q, const void* k, const void*
   // deterministic: dK / dV on the key-stationary tensor-core kernel without its dQ part,
   // then dQ query-stationary; the CUDA-core path has no atomics to begin with
   const bool tc = bwd_sm100_supported(a, dt) && bwd_dq_sm100_supported(a, dt);
-  if (a.drop.threshold && !(tc && a.dk == 128)) return ATTN_SINK_ERR_UNSUPPORTED;   // dropout: d = 128 kernels
+  if (a.drop.threshold && !tc) return ATTN_SINK_ERR_UNSUPPORTED;   // dropout: tensor-core kernels only
   if (tc) {
     cudaError_t e = launch_bwd_sm100(a, dt, s);
     if (e == cudaSuccess) e = launch_bwd_dq_sm100(a, dt, s);

@@ -68,13 +68,23 @@ inline int bwd_band_groups(const BwdArgs& a) {
 
 using namespace sm100;
 
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 constexpr int kBN = 128;  // keys per CTA
 constexpr int kBM = 128;  // queries per inner tile
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 0, kColDV = 128, kColR0 = 256, kColR1 = 384;
 
-template <int DK, int DV>
+// Dropout flags of a 128-query x 128-key tile, transposed for the compute threads (one key
+// each): word [block][key tk][w][u] holds, in byte m, the drop flag of query u + 16 (4 w + m);
+// + 16 words per block so that blocks 2x and 2x + 1 start in different banks.
+constexpr int kFlagBlockWords = 16 * 32 + 16;
+constexpr int kFlagBytes = 4 * 8 * kFlagBlockWords;
+
+template <int DK, int DV, bool DROP = false>
 struct BLayout {
   static constexpr int KH = DK / 64, VH = DV / 64;
   static constexpr int kHalf = 128 * 128;                  // 128 rows x 128 bytes
@@ -86,7 +96,8 @@ struct BLayout {
   static constexpr int kOffQ = kOffV + kVBytes;            // 2 stages
   static constexpr int kOffO = kOffQ + 2 * kQBytes;        // 2 stages (dout)
   static constexpr int kOffDS = kOffO + 2 * kOBytes;
-  static constexpr int kOffBar = kOffDS + kDSBytes;
+  static constexpr int kOffZ = kOffDS + kDSBytes;          // dropout flags, 2 stages
+  static constexpr int kOffBar = kOffZ + (DROP ? 2 * kFlagBytes : 0);
   static constexpr int kNumBars = 12;
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffSlot + 16 + 1024;
@@ -106,11 +117,12 @@ struct BBars {
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * 11; }
 };
 
-template <typename Elem, int DK, int DV, bool DQ>
+template <typename Elem, int DK, int DV, bool DQ, bool DROP = false>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do) {
-  using L = BLayout<DK, DV>;
+  static_assert(!(DQ && DROP), "dropout runs with the dQ pass of the deterministic backward");
+  using L = BLayout<DK, DV, DROP>;
   extern __shared__ unsigned char smem_raw[];
 
   // ---- work unit: key tile nt of (sequence b, kv head g) ---------------------------------
@@ -132,7 +144,7 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
   const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
   const uint32_t sK = base_u32 + L::kOffK, sV = base_u32 + L::kOffV, sQ = base_u32 + L::kOffQ,
-                 sO = base_u32 + L::kOffO, sDS = base_u32 + L::kOffDS;
+                 sO = base_u32 + L::kOffO, sDS = base_u32 + L::kOffDS, sZ = base_u32 + L::kOffZ;
   const BBars bar{base_u32 + L::kOffBar};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -260,20 +272,42 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
     for (int t = 0; t < T; ++t) {
       const int h = head_of(t);
       const long long i0 = qbase_of(t);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar.sdp_full(), t & 1, a.status))) { ok = false; break; }
-      if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar.ds_free(), (t - 1) & 1, a.status))) {
-        ok = false;
-        break;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar.sdp_full(), t & 1, a.status));
+      if (ok && t >= 1) ok = __all_sync(0xffffffffu, mbar_wait(bar.ds_free(), (t - 1) & 1, a.status));
+      // with dropout the flag producers (warps 6-9) meet these warps on a named barrier once
+      // per tile, so after a timed-out wait these warps keep passing it instead of leaving
+      if constexpr (DROP) named_bar_sync(3 + (t & 1), 256);
+      if (!ok) {
+        if constexpr (DROP) continue;
+        else break;
       }
       tc_fence_after();
       const float* lt_row = a.lse_tot + (long long)h * a.total_q + q0;
       const float* D_row = a.D + (long long)h * a.total_q + q0;
+      // dropout: this key's flags for the tile's 128 queries, words [w][u] (query u + 16 (4 w + m)
+      // in byte m)
+      uint32_t zb[DROP ? 32 : 1];
+      if constexpr (DROP) {
+        const uint32_t src = sZ + (t & 1) * kFlagBytes + 4u * ((r >> 4) * kFlagBlockWords + (r & 15) * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 8; ++v4)
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(zb[4 * v4]), "=r"(zb[4 * v4 + 1]), "=r"(zb[4 * v4 + 2]), "=r"(zb[4 * v4 + 3])
+                       : "r"(src + 16u * v4)
+                       : "memory");
+      }
 #pragma unroll 1
       for (int c = 0; c < kBM / 32; ++c) {
         uint32_t sv[32], dpv[32];
         tmem_ld32(tmem + lane_off + kColR0 + c * 32, sv);
         tmem_ld32(tmem + lane_off + kColR1 + c * 32, dpv);
         tmem_wait_ld();
+        // queries 32 c + e: word (c / 2) * 16 + e % 16, byte 2 (c % 2) + e / 16
+        uint32_t zh[DROP ? 16 : 1];
+        if constexpr (DROP) {
+#pragma unroll
+          for (int w = 0; w < 16; ++w) zh[w] = (c >> 1) ? zb[16 + w] : zb[w];
+        }
         uint32_t pk[16], dk_[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -289,7 +323,15 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
             if (vis) {
               const float lt = __ldg(lt_row + qi);
               p = ex2(fmaf(__uint_as_float(sv[e + u]), scale2, -lt * kLog2e));
-              ds = p * (__uint_as_float(dpv[e + u]) - __ldg(D_row + qi));
+              if constexpr (DROP) {
+                // dV takes the kept probabilities (256 / T is applied to dV), dS = P (Z dP - D)
+                const uint32_t byte = (uint32_t)(2 * (c & 1) + ((e + u) >> 4));
+                const uint32_t m = prmt_sign_r(zh[(e + u) & 15], (8u | byte) * 0x1111u);
+                ds = p * fmaf(__uint_as_float(dpv[e + u] & ~m), a.drop.scale, -__ldg(D_row + qi));
+                p = __uint_as_float(__float_as_uint(p) & ~m);
+              } else {
+                ds = p * (__uint_as_float(dpv[e + u]) - __ldg(D_row + qi));
+              }
             }
             pp[u] = p;
             dd[u] = ds;
@@ -322,7 +364,7 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
     for (int pass = 0; pass < 2; ++pass) {
       const int ncol = pass == 0 ? DK : DV;
       const uint32_t col = pass == 0 ? kColDK : kColDV;
-      const float mul = pass == 0 ? a.scale : 1.f;
+      const float mul = pass == 0 ? a.scale : (DROP ? a.drop.scale : 1.f);
       uint4* dst = reinterpret_cast<uint4*>(pass == 0 ? dkp : dvp);
       for (int c = 0; c < ncol / 32; ++c) {
         uint32_t v[32];
@@ -342,6 +384,41 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
           for (int u = 0; u < 4; ++u) dst[c * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
+    }
+  } else if (DROP) {
+    // ================================ dropout flags (warps 6-9) ============================
+    // Thread rt draws key block rt / 16 for queries u0 + 16 m (u0 = rt % 16, m = 0..7) of
+    // tile t: 8 Philox calls, a tile ahead of the compute warps, written transposed into
+    // stage t % 2; the compute warps are done with tile t - 2 (the stage's previous use)
+    // once this thread has passed the barrier of tile t - 1.
+    const int rt = (warp - 6) * 32 + lane, blk = rt >> 4, u0 = rt & 15;
+    const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
+    for (int t = 0; t < T; ++t) {
+      uint32_t fw[8][4];   // [m][word]
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const uint4 w = dropout_bytes(a.drop, (uint32_t)((n0 >> 4) + blk), (uint32_t)(q0 + qbase_of(t) + u0 + 16 * m),
+                                      (uint32_t)head_of(t));
+        fw[m][0] = drop_flags4(w.x, t4, t4h);
+        fw[m][1] = drop_flags4(w.y, t4, t4h);
+        fw[m][2] = drop_flags4(w.z, t4, t4h);
+        fw[m][3] = drop_flags4(w.w, t4, t4h);
+      }
+      const uint32_t stage = sZ + (t & 1) * kFlagBytes;
+#pragma unroll
+      for (int tk = 0; tk < 16; ++tk) {
+        const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          // bytes m = 0..3 of this word: queries u0 + 16 (4 w + m), key tk
+          const uint32_t lo2 = __byte_perm(fw[4 * w][tk >> 2], fw[4 * w + 1][tk >> 2], sel);
+          const uint32_t hi2 = __byte_perm(fw[4 * w + 2][tk >> 2], fw[4 * w + 3][tk >> 2], sel);
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage + 4u * (blk * kFlagBlockWords + tk * 32 + w * 16 + u0)),
+                       "r"(__byte_perm(lo2, hi2, 0x5410))
+                       : "memory");
+        }
+      }
+      named_bar_sync(3 + (t & 1), 256);
     }
   } else {
     // ================================ dQ warps (thread = query row) =======================
@@ -432,9 +509,6 @@ struct PBars {
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * 17; }
 };
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 
 template <typename Elem, int DV, bool DQ, bool DROP>
@@ -934,7 +1008,6 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
 
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
-  using L = BLayout<DK, DV>;
   constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tq, tk, tv, to;
   if (!make_map_3d(&tq, a.q, DK, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, DK, a.hkv, a.total_k, 128, dt) ||
@@ -944,13 +1017,16 @@ cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * DK * sizeof(float), s) : cudaSuccess;
   if (e != cudaSuccess) return e;
   if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
-  auto kernel = dq ? bwd_sm100_kernel<T, DK, DV, true> : bwd_sm100_kernel<T, DK, DV, false>;
-  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) != cudaSuccess)
+  const bool drop = !dq && a.drop.threshold != 0;
+  auto kernel = dq ? bwd_sm100_kernel<T, DK, DV, true>
+                   : (drop ? bwd_sm100_kernel<T, DK, DV, false, true> : bwd_sm100_kernel<T, DK, DV, false>);
+  const int smem = drop ? BLayout<DK, DV, true>::kSmem : BLayout<DK, DV>::kSmem;
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
     return e;
   BwdArgs ab = a;
   ab.band_groups = bwd_band_groups(a);
   const long long ctas = (long long)a.hkv * a.batch * ((a.max_sk + kBN - 1) / kBN);
-  kernel<<<(unsigned)ctas, kThreads, L::kSmem, s>>>(ab, tq, tk, tv, to);
+  kernel<<<(unsigned)ctas, kThreads, smem, s>>>(ab, tq, tk, tv, to);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (!dq) return cudaSuccess;
   const long long n8 = (long long)a.total_q * a.hq * DK / 8;

@@ -88,13 +88,21 @@ BWD_CASES += [
     ("d256_causal_gqa_p10", [1, 129, 0, 257], [1, 129, 0, 257], 4, 2, 256, True, -1, -1, "normal",
      "bf16", 0.1),
     ("d256_fp16_window_sq_ne_sk_p30", [200, 5], [230, 90], 2, 1, 256, True, 70, 0, "normal", "fp16", 0.3),
+    # head dim 64 (the dv field reads "64x<dv>"): the d = 64 dK/dV kernel with dropout
+    ("dk64_dv64_causal_gqa_p20", [1, 129, 0, 257], [1, 129, 0, 257], 4, 2, "64x64", True, -1, -1,
+     "normal", "bf16", 0.2),
+    ("dk64_dv128_fp16_window_p10", [300, 70], [333, 90], 4, 1, "64x128", True, 100, 0, "uniform", "fp16",
+     0.1),
 ]
 
 
 @pytest.mark.parametrize("case", BWD_CASES, ids=[c[0] for c in BWD_CASES])
 def test_bwd_dropout_matches_oracle(case):
     name, lq, lk, hq, hkv, dv, causal, wl, wr, sink, dtype, pdrop = case
-    dk = 256 if dv == 256 else 128
+    if isinstance(dv, str):
+        dk, dv = (int(x) for x in dv.split("x"))
+    else:
+        dk = 256 if dv == 256 else 128
     p = W.random_problem(_seed(name) + 5, lq, lk, hq, hkv, dk, dv, causal, wl, wr, sink, dtype,
                          with_dout=True)
     drop = (pdrop, BIG_SEED ^ _seed(name), 3 + _seed(name))
@@ -186,8 +194,9 @@ def test_fwd_dropout_keep_mask_is_exact(case, d):
 
 @pytest.mark.parametrize("case,d", [(c, 128) for c in MASK_CASES[:2]] + [
     (("causal_fp16_dv_p30", [333, 129], [333, 140], 4, 2, True, 90, 0, "fp16", 0.3), 128),
-    (("d256_two_sided_gqa_p20", [300, 517], [300, 517], 4, 2, False, 120, 120, "bf16", 0.2), 256)],
-    ids=[c[0] for c in MASK_CASES[:2]] + ["causal_fp16_dv_p30", "d256_two_sided_gqa_p20"])
+    (("d256_two_sided_gqa_p20", [300, 517], [300, 517], 4, 2, False, 120, 120, "bf16", 0.2), 256),
+    (("d64_causal_gqa_p25", [300, 200], [300, 200], 4, 2, True, 63, 0, "bf16", 0.25), 64)],
+    ids=[c[0] for c in MASK_CASES[:2]] + ["causal_fp16_dv_p30", "d256_two_sided_gqa_p20", "d64_causal_gqa_p25"])
 def test_bwd_dropout_keep_mask_is_exact(case, d):
     """dv carries the keep mask bit for bit; dq, the difference of kept and dropped terms,
     is checked element-wise within a tenth of the gap between the two."""
