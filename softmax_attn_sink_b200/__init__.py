@@ -200,7 +200,7 @@ def attn_sink_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_se
     """Sink-attention forward on packed THD tensors.  Returns (out, lse).  dropout, when
     given, is (p, seed, offset) (tensor-core path; see attn_sink_dropout).
 
-    q [T_q, Hq, dk], k [T_k, Hkv, dk], v [T_k, Hkv, dv] (bf16 or fp32, CUDA, contiguous);
+    q [T_q, Hq, dk], k [T_k, Hkv, dk], v [T_k, Hkv, dv] (bf16, fp16 or fp32, CUDA, contiguous);
     cu_seqlens_q / cu_seqlens_k int32 [B + 1]; sink fp32 [Hq] or None (= -inf);
     softmax_scale defaults to 1/sqrt(dk); window_size (left, right), -1 = unbounded;
     causal is bottom-right aligned.  lse [Hq, T_q] fp32 excludes the sink.
@@ -383,8 +383,10 @@ def selftest_wait_timeout(stream=None) -> None:
 
 class SinkAttention:
     """Autograd wrapper: ``SinkAttention.apply(q, k, v, sink, cu_q, cu_k, max_q, max_k,
-    scale, causal, window_left, window_right)`` -> out, with gradients for q, k, v and the
-    sink (the learnable offset of slime's learnable_softmax_flash_attn_varlen)."""
+    scale, causal, window_left, window_right[, dropout[, deterministic]])`` -> out, with
+    gradients for q, k, v and the sink (the learnable offset of slime's
+    learnable_softmax_flash_attn_varlen).  dropout is None or (p, seed, offset); the backward
+    redraws the forward's keep decisions from it."""
 
     _fn = None
 
@@ -395,21 +397,23 @@ class SinkAttention:
 
             class _F(torch.autograd.Function):
                 @staticmethod
-                def forward(ctx, q, k, v, sink, cu_q, cu_k, max_q, max_k, scale, causal, wl, wr):
+                def forward(ctx, q, k, v, sink, cu_q, cu_k, max_q, max_k, scale, causal, wl, wr,
+                            dropout=None, deterministic=False):
                     out, lse = attn_sink_fwd(q, k, v, cu_q, cu_k, max_q, max_k, sink, scale,
-                                             causal, (wl, wr))
+                                             causal, (wl, wr), dropout=dropout)
                     ctx.save_for_backward(q, k, v, sink, cu_q, cu_k, out, lse)
-                    ctx.cfg = (max_q, max_k, scale, causal, wl, wr)
+                    ctx.cfg = (max_q, max_k, scale, causal, wl, wr, dropout, deterministic)
                     return out
 
                 @staticmethod
                 def backward(ctx, dout):
                     q, k, v, sink, cu_q, cu_k, out, lse = ctx.saved_tensors
-                    max_q, max_k, scale, causal, wl, wr = ctx.cfg
+                    max_q, max_k, scale, causal, wl, wr, dropout, deterministic = ctx.cfg
                     dq, dk, dv, ds = attn_sink_bwd(q, k, v, out, dout.contiguous(), lse, cu_q,
                                                    cu_k, max_q, max_k, sink, scale, causal,
-                                                   (wl, wr))
-                    return dq, dk, dv, ds, None, None, None, None, None, None, None, None
+                                                   (wl, wr), deterministic=deterministic,
+                                                   dropout=dropout)
+                    return (dq, dk, dv, ds) + (None,) * 10
 
             cls._fn = _F
         return cls._fn.apply(*args)
