@@ -374,60 +374,10 @@ __device__ __forceinline__ bool tile_of(const BwdArgs& a, int ntiles, int band, 
   t.T = t.n_m * (a.hq / a.hkv);
   return true;
 }
-// Dropout in the key-stationary kernels: a compute thread owns a key, but a Philox call gives
-// the keep bytes of 16 keys for one query.  Warps 2-3 draw the 512 calls of a 64-query x
-// 128-key tile (thread rt: key block rt / 8, queries u + 16 k for u in {rt % 8, rt % 8 + 8},
-// k = 0..3), turn them into drop flags (bit 7 of a byte set = dropped) and write them
-// transposed into a two-stage buffer: word [block][key tk][u] holds, in byte k, the flag of
-// query u + 16 k for key 16 block + tk.  Producer and compute warps meet on named barrier
-// 3 + t % 2 once per tile (64 + 128 threads); the producer passes the barrier of tile t - 1
-// only after the compute warps are done with tile t - 2, whose stage tile t reuses.
-constexpr int kZBlockWords = 16 * 16 + 16;   // + 16 words: blocks 2w, 2w+1 in other banks
-constexpr int kZBytes = 4 * 8 * kZBlockWords;
-__device__ __forceinline__ void draw_flags(const BwdArgs& a, uint32_t zbuf, int rt, int n0, long long row0, int h) {
-  const int blk = rt >> 3, u0 = rt & 7;
-  const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
-  uint32_t fw[2][16];   // [u half][4 k + word]
-#pragma unroll
-  for (int uh = 0; uh < 2; ++uh)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 w = dropout_bytes(a.drop, (uint32_t)((n0 >> 4) + blk), (uint32_t)(row0 + u0 + 8 * uh + 16 * k),
-                                    (uint32_t)h);
-      fw[uh][4 * k] = drop_flags4(w.x, t4, t4h);
-      fw[uh][4 * k + 1] = drop_flags4(w.y, t4, t4h);
-      fw[uh][4 * k + 2] = drop_flags4(w.z, t4, t4h);
-      fw[uh][4 * k + 3] = drop_flags4(w.w, t4, t4h);
-    }
-#pragma unroll
-  for (int uh = 0; uh < 2; ++uh)
-#pragma unroll
-    for (int tk = 0; tk < 16; ++tk) {
-      // flag byte of key tk of query u + 16 k is byte tk % 4 of fw[uh][4 k + tk / 4]
-      const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
-      const uint32_t lo2 = __byte_perm(fw[uh][tk >> 2], fw[uh][4 + (tk >> 2)], sel);
-      const uint32_t hi2 = __byte_perm(fw[uh][8 + (tk >> 2)], fw[uh][12 + (tk >> 2)], sel);
-      asm volatile("st.shared.u32 [%0], %1;" ::"r"(zbuf + 4u * (blk * kZBlockWords + tk * 16 + u0 + 8 * uh)),
-                   "r"(__byte_perm(lo2, hi2, 0x5410))
-                   : "memory");
-    }
-}
-
-// The 16 flag words of key r of a tile (word u: queries u + 16 k in byte k).
-__device__ __forceinline__ void read_flags(uint32_t zbuf, int r, uint32_t (&zb)[16]) {
-  const uint32_t src = zbuf + 4u * ((r >> 4) * kZBlockWords + (r & 15) * 16);
-#pragma unroll
-  for (int v4 = 0; v4 < 4; ++v4)
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(zb[4 * v4]), "=r"(zb[4 * v4 + 1]), "=r"(zb[4 * v4 + 2]), "=r"(zb[4 * v4 + 3])
-                 : "r"(src + 16u * v4)
-                 : "memory");
-}
-
-// Drop mask (all ones if dropped) of query q (0..63) of the tile from the key's flag words.
-__device__ __forceinline__ uint32_t drop_mask(const uint32_t (&zb)[16], int q) {
-  return prmt_sign_r(zb[q & 15], (8u | (uint32_t)(q >> 4)) * 0x1111u);
-}
+// Dropout in the key-stationary kernels: warps 2-3 draw each 64-query tile's flags
+// (draw_flags64) into stage t % 2 of a two-stage buffer, and they meet the compute warps on named
+// barrier 3 + t % 2 once per tile (64 + 128 threads).  The producer passes the barrier of tile
+// t - 1 only after the compute warps are done with tile t - 2, whose stage tile t reuses.
 }  // namespace ks
 
 // ---- dV --------------------------------------------------------------------------------------
@@ -437,7 +387,7 @@ constexpr int kOffQ = 0;                           // Q ring
 constexpr int kOffO = kOffQ + kStages * kTile64;   // dout ring
 constexpr int kOffLT = kOffO + kStages * kTile64;  // -lse_tot log2e of the tile's queries [2][64]
 constexpr int kOffZ = kOffLT + 2 * 64 * 4;         // dropout flags, 2 stages
-constexpr int kOffBar = kOffZ + 2 * ks::kZBytes;
+constexpr int kOffBar = kOffZ + 2 * kFlagBytes64;
 constexpr int kNumBars = 1 + 2 * kStages + 6;      // k_full, qd_full[S], qd_empty[S], s_full[2], p_full[2], dv_done, drain
 constexpr int kOffSlot = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffSlot + 16 + 1024;
@@ -559,7 +509,7 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
     // warps 2-3: the dropout flags of every tile, a tile ahead of the compute warps
     const int rt = (warp - 2) * 32 + lane;
     for (int t = 0; t < T_; ++t) {
-      ks::draw_flags(a, sZ + (t & 1) * ks::kZBytes, rt, tl.n0, (long long)tl.q0 + qbase_of(t), head_of(t));
+      draw_flags64(a.drop, sZ + (t & 1) * kFlagBytes64, rt, tl.n0 >> 4, (long long)tl.q0 + qbase_of(t), head_of(t));
       named_bar_sync(3 + (t & 1), 192);
     }
   } else if (warp >= 4) {
@@ -595,7 +545,7 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
       const uint32_t tS = tmem + lane_off + col_S(t & 1);
       const float* nl = s_nlt + (t & 1) * kBM;
       uint32_t zb[DROP ? 16 : 1];
-      if constexpr (DROP) ks::read_flags(sZ + (t & 1) * ks::kZBytes, r, zb);
+      if constexpr (DROP) read_flags64(sZ + (t & 1) * kFlagBytes64, r, zb);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
@@ -610,8 +560,8 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
           const float s1 = (c0 + 1 >= c_lo && c0 + 1 < c_hi) ? __uint_as_float(sv[2 * e + 1]) : kNegInf;
           float p0 = ex2(fmaf(s0, scale2, n2.x)), p1 = ex2(fmaf(s1, scale2, n2.y));
           if constexpr (DROP) {   // dV takes the kept probabilities (256 / T is applied to dV)
-            p0 = __uint_as_float(__float_as_uint(p0) & ~ks::drop_mask(zb, c0));
-            p1 = __uint_as_float(__float_as_uint(p1) & ~ks::drop_mask(zb, c0 + 1));
+            p0 = __uint_as_float(__float_as_uint(p0) & ~flag_mask64(zb, c0));
+            p1 = __uint_as_float(__float_as_uint(p1) & ~flag_mask64(zb, c0 + 1));
           }
           pk[e] = pack2<T>(p0, p1);
         }
@@ -646,7 +596,7 @@ constexpr int kOffQ = kOffV + kTile128;            // Q ring
 constexpr int kOffO = kOffQ + kStages * kTile64;   // dout ring
 constexpr int kOffLT = kOffO + kStages * kTile64;  // -lse_tot log2e [2][64], D [2][64]
 constexpr int kOffZ = kOffLT + 4 * 64 * 4;         // dropout flags, 2 stages
-constexpr int kOffBar = kOffZ + 2 * ks::kZBytes;
+constexpr int kOffBar = kOffZ + 2 * kFlagBytes64;
 constexpr int kNumBars = 2 + 2 * kStages + 4;      // k_full, v_full, qd_full[S], qd_empty[S], sdp_full, ds_full, dk_done, drain
 constexpr int kOffSlot = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffSlot + 16 + 1024;
@@ -770,7 +720,7 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
     // warps 2-3: the dropout flags of every tile, a tile ahead of the compute warps
     const int rt = (warp - 2) * 32 + lane;
     for (int t = 0; t < T_; ++t) {
-      ks::draw_flags(a, sZ + (t & 1) * ks::kZBytes, rt, tl.n0, (long long)tl.q0 + qbase_of(t), head_of(t));
+      draw_flags64(a.drop, sZ + (t & 1) * kFlagBytes64, rt, tl.n0 >> 4, (long long)tl.q0 + qbase_of(t), head_of(t));
       named_bar_sync(3 + (t & 1), 192);
     }
   } else if (warp >= 4) {
@@ -813,7 +763,7 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
       const float* nl = s_nlt + (t & 1) * kBM;
       const float* dd = s_D + (t & 1) * kBM;
       uint32_t zb[DROP ? 16 : 1];
-      if constexpr (DROP) ks::read_flags(sZ + (t & 1) * ks::kZBytes, r, zb);
+      if constexpr (DROP) read_flags64(sZ + (t & 1) * kFlagBytes64, r, zb);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], pv[32];
@@ -830,7 +780,7 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
           const float s1 = (c0 + 1 >= c_lo && c0 + 1 < c_hi) ? __uint_as_float(sv[2 * e + 1]) : kNegInf;
           const float p0 = ex2(fmaf(s0, scale2, n2.x)), p1 = ex2(fmaf(s1, scale2, n2.y));
           if constexpr (DROP) {   // dS = P (Z dP - D)
-            const uint32_t m0 = ks::drop_mask(zb, c0), m1 = ks::drop_mask(zb, c0 + 1);
+            const uint32_t m0 = flag_mask64(zb, c0), m1 = flag_mask64(zb, c0 + 1);
             pk[e] = pack2<T>(p0 * fmaf(__uint_as_float(pv[2 * e] & ~m0), a.drop.scale, -d2.x),
                              p1 * fmaf(__uint_as_float(pv[2 * e + 1] & ~m1), a.drop.scale, -d2.y));
           } else {

@@ -694,43 +694,16 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       // 3 + half with the compute warps (64 + 128 threads).  Both sides take that barrier
       // exactly once per half, also after a timed-out wait, so its generations always pair
       // up; while the compute warps work on a half these warps draw the next one.
-      const int rt = (warp - 2) * 32 + lane, blk = rt >> 3, u0 = rt & 7;
-      const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
-      constexpr int kBlockWords = 16 * 16 + 16;   // + 16 words: blocks 2w, 2w+1 in other banks
+      const int rt = (warp - 2) * 32 + lane;
       bool ok = true;
       for (int t = 0; t < T; ++t) {
         const int h = head_of(t);
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
-          const long long qa = qbase_of(t) + 64 * hh;
-          uint32_t fw[2][16];   // [u half][4 k + word]
-#pragma unroll
-          for (int uh = 0; uh < 2; ++uh)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint4 w = dropout_bytes(a.drop, (uint32_t)((n0 >> 4) + blk),
-                                            (uint32_t)(q0 + qa + u0 + 8 * uh + 16 * k), (uint32_t)h);
-              fw[uh][4 * k] = drop_flags4(w.x, t4, t4h);
-              fw[uh][4 * k + 1] = drop_flags4(w.y, t4, t4h);
-              fw[uh][4 * k + 2] = drop_flags4(w.z, t4, t4h);
-              fw[uh][4 * k + 3] = drop_flags4(w.w, t4, t4h);
-            }
+          uint32_t fw[2][16];
+          draw_flag_words64(a.drop, rt, n0 >> 4, q0 + qbase_of(t) + 64 * hh, h, fw);
           if (ok && t >= 1) ok = __all_sync(0xffffffffu, mbar_wait(bar.ds_free(hh), (t - 1) & 1, a.status));
-          if (ok) {
-            const uint32_t stage = sDS + hh * L::kHalf;
-#pragma unroll
-            for (int uh = 0; uh < 2; ++uh)
-#pragma unroll
-              for (int tk = 0; tk < 16; ++tk) {
-                // flag byte of key tk of query u + 16 k is byte tk % 4 of fw[uh][4 k + tk / 4]
-                const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
-                const uint32_t lo2 = __byte_perm(fw[uh][tk >> 2], fw[uh][4 + (tk >> 2)], sel);
-                const uint32_t hi2 = __byte_perm(fw[uh][8 + (tk >> 2)], fw[uh][12 + (tk >> 2)], sel);
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage + 4u * (blk * kBlockWords + tk * 16 + u0 + 8 * uh)),
-                             "r"(__byte_perm(lo2, hi2, 0x5410))
-                             : "memory");
-              }
-          }
+          if (ok) store_flag_words64(sDS + hh * L::kHalf, rt, fw);
           named_bar_sync(3 + hh, 192);
         }
       }
@@ -780,19 +753,8 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         // (ok = false), like the named barriers of the tile loop.
         uint32_t zb[DROP ? 16 : 1];
         if constexpr (DROP) {
-          const uint32_t stage = sDS + hh * L::kHalf;
-          const int blk = r >> 4;
-          constexpr int kBlockWords = 16 * 16 + 16;
           named_bar_sync(3 + hh, 192);   // warps 2-3 have written this half's flags
-          if (ok) {
-            const uint32_t src = stage + 4u * (blk * kBlockWords + (r & 15) * 16);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(zb[4 * v4]), "=r"(zb[4 * v4 + 1]), "=r"(zb[4 * v4 + 2]), "=r"(zb[4 * v4 + 3])
-                           : "r"(src + 16u * v4)
-                           : "memory");
-          }
+          if (ok) read_flags64(sDS + hh * L::kHalf, r, zb);
           named_bar_sync(2, 128);   // every thread has its bytes before dS overwrites the area
         }
         if (!ok) continue;

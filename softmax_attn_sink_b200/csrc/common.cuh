@@ -86,6 +86,73 @@ __device__ __forceinline__ uint32_t prmt_sign_r(uint32_t a, uint32_t sel) {
   return r;
 }
 
+// Drop flags for a kernel whose compute thread owns a key (a Philox call covers 16 keys of one
+// query).  For a tile of 64 queries x 128 keys, 64 producer threads draw the 512 calls (thread
+// rt: key block rt / 8, queries u + 16 k for u in {rt % 8, rt % 8 + 8}, k = 0..3) and store
+// the flags transposed: word [block][key tk][u] holds, in byte k, the flag of query u + 16 k
+// for key 16 block + tk; + 16 words per block put blocks 2w and 2w + 1 in other banks.
+constexpr int kFlagWords64 = 16 * 16 + 16;
+constexpr int kFlagBytes64 = 4 * 8 * kFlagWords64;
+
+// rt's share of the tile whose first key block is key_block0 and first packed row row0, as
+// flag words in registers (fw[uh][4 k + word]: queries rt % 8 + 8 uh + 16 k).
+__device__ __forceinline__ void draw_flag_words64(const Dropout& d, int rt, long long key_block0, long long row0,
+                                                  int h, uint32_t (&fw)[2][16]) {
+  const int blk = rt >> 3, u0 = rt & 7;
+  const uint32_t t4 = (d.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
+#pragma unroll
+  for (int uh = 0; uh < 2; ++uh)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 w = dropout_bytes(d, (uint32_t)(key_block0 + blk), (uint32_t)(row0 + u0 + 8 * uh + 16 * k),
+                                    (uint32_t)h);
+      fw[uh][4 * k] = drop_flags4(w.x, t4, t4h);
+      fw[uh][4 * k + 1] = drop_flags4(w.y, t4, t4h);
+      fw[uh][4 * k + 2] = drop_flags4(w.z, t4, t4h);
+      fw[uh][4 * k + 3] = drop_flags4(w.w, t4, t4h);
+    }
+}
+
+// Stores rt's flag words transposed into the tile's buffer at zbuf.
+__device__ __forceinline__ void store_flag_words64(uint32_t zbuf, int rt, const uint32_t (&fw)[2][16]) {
+  const int blk = rt >> 3, u0 = rt & 7;
+#pragma unroll
+  for (int uh = 0; uh < 2; ++uh)
+#pragma unroll
+    for (int tk = 0; tk < 16; ++tk) {
+      // flag byte of key tk of query u + 16 k is byte tk % 4 of fw[uh][4 k + tk / 4]
+      const uint32_t sel = (uint32_t)(tk & 3) | ((uint32_t)(4 + (tk & 3)) << 4);
+      const uint32_t lo2 = __byte_perm(fw[uh][tk >> 2], fw[uh][4 + (tk >> 2)], sel);
+      const uint32_t hi2 = __byte_perm(fw[uh][8 + (tk >> 2)], fw[uh][12 + (tk >> 2)], sel);
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(zbuf + 4u * (blk * kFlagWords64 + tk * 16 + u0 + 8 * uh)),
+                   "r"(__byte_perm(lo2, hi2, 0x5410))
+                   : "memory");
+    }
+}
+
+__device__ __forceinline__ void draw_flags64(const Dropout& d, uint32_t zbuf, int rt, long long key_block0,
+                                             long long row0, int h) {
+  uint32_t fw[2][16];
+  draw_flag_words64(d, rt, key_block0, row0, h, fw);
+  store_flag_words64(zbuf, rt, fw);
+}
+
+// The 16 flag words of key r of the tile (word u: queries u + 16 k in byte k).
+__device__ __forceinline__ void read_flags64(uint32_t zbuf, int r, uint32_t (&zb)[16]) {
+  const uint32_t src = zbuf + 4u * ((r >> 4) * kFlagWords64 + (r & 15) * 16);
+#pragma unroll
+  for (int v4 = 0; v4 < 4; ++v4)
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(zb[4 * v4]), "=r"(zb[4 * v4 + 1]), "=r"(zb[4 * v4 + 2]), "=r"(zb[4 * v4 + 3])
+                 : "r"(src + 16u * v4)
+                 : "memory");
+}
+
+// All-ones mask if query q (0..63) of the tile is dropped for this key, else 0.
+__device__ __forceinline__ uint32_t flag_mask64(const uint32_t (&zb)[16], int q) {
+  return prmt_sign_r(zb[q & 15], (8u | (uint32_t)(q >> 4)) * 0x1111u);
+}
+
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
