@@ -77,10 +77,15 @@ struct Layout {
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffItems = (kOffTmemSlot + 16 + 127) / 128 * 128;  // ItemDesc[kItemSlots]
   static constexpr int kOffTable = kOffItems + kItemSlots * 128;           // item list of a persistent launch
-  // bytes for a table of `table_ints` ints, + slack to align the base to 1 KB; at least 116 KB
-  // so that two CTAs never share an SM (each CTA holds all 512 TMEM columns)
-  static constexpr long long smem_bytes(long long table_ints) {
-    return (kOffTable + 4 * table_ints + 1024) > 118784 ? (kOffTable + 4 * table_ints + 1024) : 118784;
+  // Output staging after the table: 32 rows x 64 columns (128 B) per softmax warp.
+  static constexpr int kStageBytes = 32 * 128;
+  static constexpr long long stage_offset(long long table_ints) { return (kOffTable + 4 * table_ints + 127) / 128 * 128; }
+  // bytes for a table of `table_ints` ints (and the staging area), + slack to align the base
+  // to 1 KB; at least 116 KB so that two CTAs never share an SM (each CTA holds all 512 TMEM
+  // columns)
+  static constexpr long long smem_bytes(long long table_ints, bool staged) {
+    const long long b = (staged ? stage_offset(table_ints) + 8LL * kStageBytes : kOffTable + 4 * table_ints) + 1024;
+    return b > 118784 ? b : 118784;
   }
 };
 
@@ -114,6 +119,7 @@ struct Sched {
   int zmax;        // levels of the longest sequence (bounded by max_seqlen_q)
   int width;       // unit pairs per (sequence, level)
   int persistent;  // 1: the grid's CTAs walk the numbered list; 0: CTA i runs item i of the dense grid
+  int stage_off;   // byte offset of the output staging area from the aligned base; 0: none
 };
 
 // Levels of sequence b: its row tiles (two q heads per item) or row-tile pairs (one head per item).
@@ -417,12 +423,20 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       constexpr uint32_t idesc_pv = idesc_of<T>(kBM, DV, 0, 1);
       // Shared-memory descriptors, built once: an address offset is an addition to the start
       // field (addresses stay below 2^18 bytes, so the 14-bit field never carries).
-      const uint64_t dQ0 = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
-      const uint64_t dQ1 = dQ0 + (uint64_t)(L::kQBytes >> 4);
-      const uint64_t dK0 = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
-      const uint64_t dV0 = smem_desc(sV, L::kHalfBytes, 1024, kLayoutSwizzle128B);
+      // All three share the high word (1024-byte stride, SW128), kept once in desc_hi.
+      const uint64_t dQ0_ = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
+      const uint32_t desc_hi = (uint32_t)(dQ0_ >> 32);
+      const uint32_t dQ0 = (uint32_t)dQ0_, dQ1 = dQ0 + (uint32_t)(L::kQBytes >> 4);
+      const uint32_t dK0 = (uint32_t)smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
+      const uint32_t dV0 = (uint32_t)smem_desc(sV, L::kHalfBytes, 1024, kLayoutSwizzle128B);
       int kv = 0, qn = 0;
       int pcA = 0, pcB = 0;  // P tiles taken so far per unit (p_full phases)
+      // Look-ahead across items: on an item's last tile the MMA thread peeks at the next item
+      // (without releasing its ring slot, so the descriptor stays in place) and issues each
+      // unit's QK of its tile 0 right after that unit's last PV; a unit's next S then does
+      // not wait for the other unit's last softmax.  That Q was loaded once every QK of the
+      // item had read Q; its K is the ring's next tile.
+      bool qk0_issued = false;
       for (int r = 0;; ++r) {
         const int slot = r % kItemSlots;
         if (!mbar_wait(bar.item_full(slot), (r / kItemSlots) & 1, a.status)) break;
@@ -432,9 +446,11 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         mbar_arrive(bar.item_empty(slot));
         if (kind == 0) break;
         if (n == 0) continue;
-        if (!mbar_wait(bar.q_full(), qn & 1, a.status)) break;
-        ++qn;
-        bool ok = true;
+        if (!qk0_issued) {
+          if (!mbar_wait(bar.q_full(), qn & 1, a.status)) break;
+          ++qn;
+        }
+        bool ok = true, nx_qk = false;
         int k_waited = -1;  // last tile of this item whose K load was waited for
         auto wait_k = [&](int j) -> bool {
           if (k_waited >= j) return true;
@@ -443,19 +459,19 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           k_waited = j;
           return true;
         };
-        // S_u(j) = Q_u K_j^T.  S_u is overwritten while P_u (inside S_u) was read by the
-        // previous PV_u: MMAs issued by one thread execute in issue order, so that read is
-        // done before this write.
+        // S_u(j) = Q_u K_j^T (j = n: tile 0 of the next item, whose K is ring tile kv + n).
+        // S_u is overwritten while P_u (inside S_u) was read by the previous PV_u: MMAs issued
+        // by one thread execute in issue order, so that read is done before this write.
         auto issue_qk = [&](int u, int j) -> bool {
           if (!wait_k(j)) return false;
           tc_fence_after();
           const int st = (kv + j) % kStages;
-          const uint64_t dq = u ? dQ1 : dQ0, dk = dK0 + (uint64_t)(st * (L::kKBytes >> 4));
+          const uint32_t dq = u ? dQ1 : dQ0, dk = dK0 + (uint32_t)(st * (L::kKBytes >> 4));
           const uint32_t dS = tmem + col_S(u);
 #pragma unroll
           for (int ks = 0; ks < DK / 16; ++ks) {
             const uint32_t off16 = ((ks >> 2) * L::kHalfBytes + (ks & 3) * 32) >> 4;
-            mma_ss(dS, dq + off16, dk + off16, idesc_qk, ks > 0);
+            mma_ss_lo(dS, dq + off16, dk + off16, desc_hi, idesc_qk, ks > 0);
           }
           mma_commit(bar.s_full(u));
           return true;
@@ -467,30 +483,51 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           tc_fence_after();
           const int st = (kv + j) % kStages;
           const bool first = j == (u ? jB0 : jA0);
-          const uint64_t dv = dV0 + (uint64_t)(st * (L::kVBytes >> 4));
+          const uint32_t dv = dV0 + (uint32_t)(st * (L::kVBytes >> 4));
           const uint32_t dO = tmem + col_O(u), aP = tmem + col_S(u);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(dO, aP + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (!first || kk > 0) ? 1u : 0u);
+            mma_ts_lo(dO, aP + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), desc_hi, idesc_pv, (!first || kk > 0) ? 1u : 0u);
           mma_commit(bar.pv_done(u));
           return true;
         };
         auto active = [&](int u, int j) { return u ? (j >= jB0 && j < jB1) : (j >= jA0 && j < jA1); };
-        for (int u = 0; u < 2 && ok; ++u)
-          if (active(u, 0)) ok = issue_qk(u, 0);
+        if (!qk0_issued)
+          for (int u = 0; u < 2 && ok; ++u)
+            if (active(u, 0)) ok = issue_qk(u, 0);
         if (!ok) break;
+        qk0_issued = false;
         if (n == 1) mma_commit(bar.q_empty());  // every QK of the item is issued
         mma_commit(bar.k_empty(kv % kStages));
+        // V(j) is waited for one step ahead (while the previous QKs are still queued), so a
+        // unit's P arrival finds this thread already waiting for it.
+        if (!(ok = mbar_wait(bar.v_full(kv % kStages), (kv / kStages) & 1, a.status))) break;
         for (int j = 0; j < n && ok; ++j) {
           const int p = kv + j, st = p % kStages;
-          if (!(ok = mbar_wait(bar.v_full(st), (p / kStages) & 1, a.status))) break;
           for (int u = 0; u < 2 && ok; ++u) {
             if (active(u, j)) ok = issue_pv(u, j);
-            if (ok && j + 1 < n && active(u, j + 1)) ok = issue_qk(u, j + 1);
+            if (!ok) break;
+            if (u == 1) {
+              mma_commit(bar.v_empty(st));   // both PVs of tile j are issued
+              if (j + 1 < n && !(ok = mbar_wait(bar.v_full((p + 1) % kStages), ((p + 1) / kStages) & 1, a.status)))
+                break;
+            }
+            if (j + 1 < n) {
+              if (active(u, j + 1)) ok = issue_qk(u, j + 1);
+            } else {
+              const int ns = (r + 1) % kItemSlots;
+              if (u == 0) {
+                if (!(ok = mbar_wait(bar.item_full(ns), ((r + 1) / kItemSlots) & 1, a.status))) break;
+                nx_qk = items[ns].kind != 0 && items[ns].n_tiles > 0;
+                // the next item's Q (loaded once this item's QKs completed)
+                if (nx_qk && !(ok = mbar_wait(bar.q_full(), qn & 1, a.status))) break;
+                qn += nx_qk ? 1 : 0;
+              }
+              if (nx_qk && items[ns].j0[u] == 0 && items[ns].j1[u] > 0) ok = issue_qk(u, n);
+            }
           }
           if (!ok) break;
           if (j + 2 == n) mma_commit(bar.q_empty());  // the last QKs are issued
-          mma_commit(bar.v_empty(st));
           if (j + 1 < n) {
             // a tile no unit needs still has to be consumed for the producer's accounting
             if (!(ok = wait_k(j + 1))) break;
@@ -501,6 +538,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         kv += n;
         pcA += jA1 - jA0;
         pcB += jB1 - jB0;
+        qk0_issued = nx_qk;
       }
       // every MMA must be complete before the TMEM is freed
       mma_commit(bar.drain());
@@ -552,6 +590,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     const uint32_t tS = tmem + lane_off + col_S(u), tO = tmem + lane_off + col_O(u);
     const float scale2 = a.scale * kLog2e;
+    const uint32_t stg = sc.stage_off ? base_u32 + (uint32_t)sc.stage_off + (uint32_t)(warp - 4) * L::kStageBytes : 0u;
     int sc_u = 0;  // S tiles of this unit taken so far (s_full / pv_done phases)
     for (int it = 0;; ++it) {
       const int slot = it % kItemSlots;
@@ -696,6 +735,8 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       const long long grow = (long long)q0 + i;   // packed row of this thread's query
       T* out = static_cast<T*>(a.out);
       uint4* orow = reinterpret_cast<uint4*>(out + (grow * a.hq + h) * DV);
+      // Rows of this warp (queries i - lane ..) that exist, for the staged stores.
+      const int nrow = sq - (i - lane);
       // The O row in as few TMEM round trips as the registers allow (this is on the unit's
       // path to its next item): all of it at once, or 32 columns at a time with dropout,
       // whose flag words take the room.
@@ -719,10 +760,30 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = pack2<T>(__uint_as_float(o[c][2 * e]) * inv, __uint_as_float(o[c][2 * e + 1]) * inv);
-          if (row_ok) {
+          const int cc = c0 + c;   // 32-column chunk
+          if (stg) {
+            // Staged: the warp's 32 rows x 64 columns go through shared memory (16-byte
+            // chunk k of row r at chunk k ^ (r % 8): no bank conflicts either way), and each
+            // store then writes 4 rows x 128 contiguous bytes instead of 32 rows x 16 bytes.
 #pragma unroll
             for (int v = 0; v < 4; ++v)
-              orow[(c0 + c) * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              st_shared_v4(stg + lane * 128 + ((((cc & 1) * 4 + v) ^ (lane & 7)) << 4), pk[4 * v], pk[4 * v + 1],
+                           pk[4 * v + 2], pk[4 * v + 3]);
+            if (cc & 1) {
+              __syncwarp();
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int rr = 4 * k + (lane >> 3), ch = lane & 7;
+                const uint4 w = ld_shared_v4(stg + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                if (rr < nrow)
+                  *reinterpret_cast<uint4*>(out + ((grow - lane + rr) * a.hq + h) * DV + (cc >> 1) * 64 + ch * 8) = w;
+              }
+              __syncwarp();
+            }
+          } else if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              orow[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
         }
       }
@@ -794,9 +855,22 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   // Persistent launch (one CTA per SM walking the item list) when the item table fits in
   // shared memory; otherwise one CTA per item of the dense (level, sequence, unit pair) grid.
   const long long items_ub = (long long)zmax * a.batch * width;
-  const long long smem_p = L::smem_bytes(3LL * zmax + a.batch);
-  Sched sc{zmax, width, smem_p <= dev.smem_optin ? 1 : 0};
-  const long long smem = sc.persistent ? smem_p : L::smem_bytes(0);
+  // The output staging area goes in when it fits beside the table (else rows are stored
+  // directly from registers).
+  const long long tbl = 3LL * zmax + a.batch;
+  Sched sc{zmax, width, 1, 0};
+  long long smem;
+  if (L::smem_bytes(tbl, true) <= dev.smem_optin) {
+    sc.stage_off = (int)L::stage_offset(tbl);
+    smem = L::smem_bytes(tbl, true);
+  } else if (L::smem_bytes(tbl, false) <= dev.smem_optin) {
+    smem = L::smem_bytes(tbl, false);
+  } else {
+    sc.persistent = 0;
+    const bool st = L::smem_bytes(0, true) <= dev.smem_optin;
+    sc.stage_off = st ? (int)L::stage_offset(0) : 0;
+    smem = L::smem_bytes(0, st);
+  }
   const long long grid = sc.persistent ? (items_ub < dev.sms ? items_ub : dev.sms) : items_ub;
   auto kernel = a.drop.threshold ? fwd_sm100_kernel<T, DK, DV, true> : fwd_sm100_kernel<T, DK, DV, false>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

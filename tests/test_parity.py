@@ -31,6 +31,9 @@ def _oracle_fwd(p):
 _LENS_A = [int(n) for n in np.random.default_rng(11).integers(0, 700, size=40)] + [0, 1]
 _LENS_B = [int(n) for n in np.random.default_rng(12).integers(1, 900, size=30)]
 _LENS_C = [int(n) for n in np.random.default_rng(13).integers(0, 5, size=9000)]
+# 600 short sequences: the item table leaves no room for the forward's output staging area,
+# so the persistent forward stores rows directly from registers.
+_LENS_D = [int(n) for n in np.random.default_rng(43).integers(0, 300, size=600)]
 
 FWD_CASES = [
     # name, lens_q, lens_k, hq, hkv, dk, dv, causal, wl, wr, sink, dtype
@@ -68,6 +71,7 @@ FWD_CASES = [
     # 9000 sequences: the item table would not fit in shared memory, so the forward runs one
     # CTA per item of the dense grid instead.
     ("grid_mode_many_sequences", _LENS_C, _LENS_C, 2, 1, 128, 128, True, -1, -1, "normal", "bf16"),
+    ("persistent_unstaged", _LENS_D, _LENS_D, 4, 2, 128, 128, True, -1, -1, "normal", "bf16"),
     # head dim 256: the one-unit tensor-core forward (Q in TMEM, 64-key tiles), its fp16
     # variant, and the CUDA-core kernel for fp32
     ("d256_causal_gqa", [1, 63, 64, 65, 0, 300, 700], [1, 63, 64, 65, 0, 300, 700], 8, 2, 256, 256,
