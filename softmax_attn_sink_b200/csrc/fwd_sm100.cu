@@ -592,6 +592,69 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
     const float scale2 = a.scale * kLog2e;
     const uint32_t stg = sc.stage_off ? base_u32 + (uint32_t)sc.stage_off + (uint32_t)(warp - 4) * L::kStageBytes : 0u;
     int sc_u = 0;  // S tiles of this unit taken so far (s_full / pv_done phases)
+    constexpr int kChunks = DV / 32;
+    // Epilogue of an item: out = O / (l + 2^{sink2 - m}),  lse = (m + log2 l) ln 2.  Without
+    // dropout it is deferred to the unit's next item: after that item's first softmax the
+    // warps read O (its first S being ready means every earlier PV of the unit is complete),
+    // then announce P, and scale and store the old O while the next PV and QK run.
+    constexpr bool kDefer = !DROP;
+    bool pend = false;                        // an item's O waits in TMEM for its epilogue
+    int e_h = 0, e_nrow = 0;                  // its head, rows of this warp that exist
+    long long e_grow = 0;                     // packed row of this thread's query
+    bool e_row = false;
+    float e_inv = 0.f, e_lse = 0.f;
+    T* const out = static_cast<T*>(a.out);
+    // scale, convert and store 32 output columns (chunk cc) of the item in e_*
+    auto emit = [&](const uint32_t (&o)[32], int cc) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        pk[e] = pack2<T>(__uint_as_float(o[2 * e]) * e_inv, __uint_as_float(o[2 * e + 1]) * e_inv);
+      if (stg) {
+        // Staged: the warp's 32 rows x 64 columns go through shared memory (16-byte chunk k
+        // of row r at chunk k ^ (r % 8): no bank conflicts either way), and each store then
+        // writes 4 rows x 128 contiguous bytes instead of 32 rows x 16 bytes.
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          st_shared_v4(stg + lane * 128 + ((((cc & 1) * 4 + v) ^ (lane & 7)) << 4), pk[4 * v], pk[4 * v + 1],
+                       pk[4 * v + 2], pk[4 * v + 3]);
+        if (cc & 1) {
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rr = 4 * k + (lane >> 3), ch = lane & 7;
+            const uint4 w = ld_shared_v4(stg + rr * 128 + ((ch ^ (rr & 7)) << 4));
+            if (rr < e_nrow)
+              *reinterpret_cast<uint4*>(out + ((e_grow - lane + rr) * a.hq + e_h) * DV + (cc >> 1) * 64 + ch * 8) = w;
+          }
+          __syncwarp();
+        }
+      } else if (e_row) {
+        uint4* orow = reinterpret_cast<uint4*>(out + (e_grow * a.hq + e_h) * DV);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          orow[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
+    };
+    auto emit_lse = [&]() {
+      if (e_row && a.lse) a.lse[(long long)e_h * a.total_q + e_grow] = e_lse;
+    };
+    // The pending epilogue, when the next item does not take its deferred path: wait for the
+    // unit's last PV (the sc_u-th pv_done phase), then read O and store it.
+    auto flush = [&]() -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (sc_u - 1) & 1, a.status))) return false;
+      tc_fence_after();
+      uint32_t o[kChunks][32];
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) tmem_ld32(tO + c * 32, o[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) emit(o[c], c);
+      emit_lse();
+      tc_fence_before();
+      pend = false;
+      return true;
+    };
     for (int it = 0;; ++it) {
       const int slot = it % kItemSlots;
       if (!__all_sync(0xffffffffu, mbar_wait(bar.item_full(slot), (it / kItemSlots) & 1, a.status))) break;
@@ -600,6 +663,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       const int q0 = d.q0, sq = d.sq, sk = d.sk, klo0 = d.lo, i = d.m0[u] + r;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar.item_empty(slot));
+      if (kDefer && pend && (kind == 0 || !valid || j1 == j0) && !flush()) break;
       if (kind == 0) break;
       if (!valid) continue;
       const bool row_ok = i < sq;
@@ -712,35 +776,52 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           }
         }
         tmem_wait_st();
+        if (kDefer && pend) {
+          // the previous item's O, before this announcement lets PV(j0) overwrite it
+          uint32_t o[kChunks][32];
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) tmem_ld32(tO + c * 32, o[c]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar.p_full(u));
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) emit(o[c], c);
+          emit_lse();
+          pend = false;
+          continue;
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar.p_full(u));
       }
       if (!ok) break;
 
-      // ---- epilogue: out = O / (l + 2^{sink2 - m}),  lse = (m + log2 l) ln 2 ---------------
-      // The next item's first PV_u overwrites O_u only after this unit's next P arrival,
-      // which these warps make after the reads below.
+      // ---- epilogue (see emit): record this item's output state -------------------------
       const bool have_o = j1 > j0;
+      sc_u += j1 - j0;
+      {
+        const float sink2 = a.sink ? a.sink[h] * kLog2e : kNegInf;
+        const float e_sink = (sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m);
+        const float den = l + e_sink;
+        // with dropout, O summed the kept probabilities unscaled: the 256 / T factor goes here
+        e_inv = den > 0.f ? (DROP ? a.drop.scale : 1.f) / den : 0.f;
+        e_lse = l > 0.f ? (m + __log2f(l)) * kLn2 : kNegInf;
+        e_h = h;
+        e_grow = (long long)q0 + i;
+        e_row = row_ok;
+        e_nrow = sq - (i - lane);   // rows of this warp (queries i - lane ..) that exist
+      }
+      if (kDefer && have_o) {
+        pend = true;
+        continue;
+      }
       if (have_o) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (ph + j1 - 1) & 1, a.status))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (sc_u - 1) & 1, a.status))) break;
         tc_fence_after();
       }
-      sc_u += j1 - j0;
-      const float sink2 = a.sink ? a.sink[h] * kLog2e : kNegInf;
-      const float e_sink = (sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m);
-      const float den = l + e_sink;
-      // with dropout, O summed the kept probabilities unscaled: the 256 / T factor goes here
-      const float inv = den > 0.f ? (DROP ? a.drop.scale : 1.f) / den : 0.f;
-      const long long grow = (long long)q0 + i;   // packed row of this thread's query
-      T* out = static_cast<T*>(a.out);
-      uint4* orow = reinterpret_cast<uint4*>(out + (grow * a.hq + h) * DV);
-      // Rows of this warp (queries i - lane ..) that exist, for the staged stores.
-      const int nrow = sq - (i - lane);
-      // The O row in as few TMEM round trips as the registers allow (this is on the unit's
-      // path to its next item): all of it at once, or 32 columns at a time with dropout,
-      // whose flag words take the room.
-      constexpr int kChunks = DV / 32, kPer = DROP ? 1 : kChunks;
+      // O 32 columns at a time with dropout (whose flag words take the room), else at once
+      constexpr int kPer = DROP ? 1 : kChunks;
 #pragma unroll
       for (int c0 = 0; c0 < kChunks; c0 += kPer) {
         uint32_t o[kPer][32];
@@ -755,40 +836,9 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
             for (int e = 0; e < 32; ++e) o[c][e] = 0u;
         }
 #pragma unroll
-        for (int c = 0; c < kPer; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack2<T>(__uint_as_float(o[c][2 * e]) * inv, __uint_as_float(o[c][2 * e + 1]) * inv);
-          const int cc = c0 + c;   // 32-column chunk
-          if (stg) {
-            // Staged: the warp's 32 rows x 64 columns go through shared memory (16-byte
-            // chunk k of row r at chunk k ^ (r % 8): no bank conflicts either way), and each
-            // store then writes 4 rows x 128 contiguous bytes instead of 32 rows x 16 bytes.
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              st_shared_v4(stg + lane * 128 + ((((cc & 1) * 4 + v) ^ (lane & 7)) << 4), pk[4 * v], pk[4 * v + 1],
-                           pk[4 * v + 2], pk[4 * v + 3]);
-            if (cc & 1) {
-              __syncwarp();
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int rr = 4 * k + (lane >> 3), ch = lane & 7;
-                const uint4 w = ld_shared_v4(stg + rr * 128 + ((ch ^ (rr & 7)) << 4));
-                if (rr < nrow)
-                  *reinterpret_cast<uint4*>(out + ((grow - lane + rr) * a.hq + h) * DV + (cc >> 1) * 64 + ch * 8) = w;
-              }
-              __syncwarp();
-            }
-          } else if (row_ok) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              orow[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          }
-        }
+        for (int c = 0; c < kPer; ++c) emit(o[c], c0 + c);
       }
-      if (row_ok && a.lse)
-        a.lse[(long long)h * a.total_q + grow] = l > 0.f ? (m + __log2f(l)) * kLn2 : kNegInf;
+      emit_lse();
       tc_fence_before();
     }
   }
