@@ -18,8 +18,11 @@
 //               Q), then K and V tiles into a 2-stage ring.
 //   warp 1      TMEM allocation and the MMA issuer (one thread), in the order
 //                 PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1)
-//               so the tensor core works for one unit while the other unit's softmax runs.
-//               QK: S_U = Q_U K^T (A, B from shared memory); PV: O_U += P_U V (P from TMEM).
+//               so the tensor core works for one unit while the other unit's softmax runs;
+//               on an item's last tile the QKs of the next item's first tile follow the
+//               PVs directly.  QK: S_U = Q_U K^T (A, B from shared memory); PV: O_U += P_U V
+//               (P from TMEM).  An MMA issue returns only once the tensor core takes it, so
+//               the thread waits for the next tile's V while earlier MMAs are still queued.
 //   warp 2      the scheduler: builds the item list, then decodes the CTA's items one by one
 //               into a 2-slot shared-memory ring that the other roles read (warp 3 idles).
 //   warps 4-7   softmax and epilogue of unit A, warps 8-11 of unit B: thread t owns query row
@@ -27,7 +30,9 @@
 //               in post-scale units); the running sum counts keys only and e^{sink-m} joins
 //               the denominator in the epilogue, so the vanilla lse is m + log sum.  O is
 //               rescaled lazily, only when a row's max grows by more than 2^8 (exact: O and
-//               the sum share the stale reference).
+//               the sum share the stale reference).  An item's epilogue runs after the
+//               unit's next first softmax has read O out of TMEM (without dropout), and its
+//               rows go out through a per-warp shared-memory stage as whole row segments.
 // TMEM columns: S_A [0,128) O_A [128,256) S_B [256,384) O_B [384,512); P_U (bf16) is written
 // over the first 64 columns of S_U once S_U has been read; the next QK_U into S_U is issued
 // after the PV_U that reads it, and MMAs from one thread execute in issue order.  Because a
