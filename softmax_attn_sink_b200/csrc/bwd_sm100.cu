@@ -462,9 +462,8 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
 //
 // Same gradient as above.  Each 128-query tile is processed as two halves a/b so that the
 // tensor pipe works on one half while the compute warps work on the other:
-//   MMA order per tile t:  [wait compute_a] dQ^T_a dV_a dK_a  [wait compute_b]
-//                          S_a(t+1) dP_a(t+1)  dQ^T_b dV_b dK_b  S_b(t+1) dP_b(t+1)
-//   (dQ^T of a half first, so its dQ warps read it while dV and dK run)
+//   MMA order per tile t:  [wait compute_a] dV_a dK_a dQ^T_a  [wait compute_b]
+//                          S_a(t+1) dP_a(t+1)  dV_b dK_b dQ^T_b  S_b(t+1) dP_b(t+1)
 // dQ is produced transposed, dQ^T = K^T dS^T (M = head dim), so a dQ warp thread owns one
 // head-dim index and each warp-wide reduction covers 128 contiguous bytes of a dQ row.
 // TMEM: dK [0,128) dV [128,256) S_a [256,320) dP_a [320,384) S_b [384,448) dP_b [448,512);
@@ -651,14 +650,6 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         const uint64_t qoff = (uint64_t)((st * L::kQBytes) >> 4), ooff = (uint64_t)((st * L::kOBytes) >> 4);
         const uint64_t dsoff = (uint64_t)((hh * L::kHalf) >> 4);
         const uint32_t cS = tmem + (hh ? kColSb : kColSa), cP = tmem + (hh ? kColDPb : kColDPa);
-        // dQ^T first: the dQ warps read it while dV and dK run, so the next dP (into the same
-        // columns) finds them done
-        if (DQ) {
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ss(cP, mK + (uint64_t)((kk * 2048) >> 4), mDS + dsoff + (uint64_t)((kk * 2048) >> 4), id_dq, kk > 0);
-          mma_commit(bar.dq_full(hh));
-        }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tmem + kColDV, cS + kk * 8, mO + ooff + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_dv,
@@ -668,6 +659,12 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem + kColDK, kDS + dsoff + (uint64_t)((kk * 32) >> 4),
                  mQ + qoff + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_dk, (t > 0 || hh > 0 || kk > 0));
+        if (DQ) {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ss(cP, mK + (uint64_t)((kk * 2048) >> 4), mDS + dsoff + (uint64_t)((kk * 2048) >> 4), id_dq, kk > 0);
+          mma_commit(bar.dq_full(hh));
+        }
         mma_commit(bar.ds_free(hh));
       };
       bool ok = mbar_wait(bar.kv_full(), 0, a.status);
