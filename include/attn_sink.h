@@ -231,13 +231,17 @@ int attn_sink_decode_paged(const attn_sink_params* params, const void* q, const 
  * attn_sink_decode, minus the workspace: the chunk partials live in a fixed 16 MiB
  * device array inside the library, present on every GPU that loads the library until the
  * process exits.  No cudaMalloc, cudaFree or other allocating routine is called.
- *   - num_splits == 0 picks the automatic split count, lowered until the partials fit in
- *     16 MiB; an explicit num_splits whose partials need more than 16 MiB, or a problem
- *     that does not fit even with one split, returns ATTN_SINK_ERR_WORKSPACE before any
- *     launch.
- *   - The first call on each device looks up the array's device address (a
- *     cudaGetSymbolAddress with that device current) and caches it; make that first call
- *     before capturing any stream.
+ *   - num_splits == 0 picks the automatic split count of attn_sink_decode_num_splits(),
+ *     or, when its partials need more than 16 MiB, the largest smaller count whose
+ *     partials fit; an explicit num_splits whose partials need more than 16 MiB, or a
+ *     problem that does not fit even with one split, returns ATTN_SINK_ERR_WORKSPACE
+ *     before any launch.
+ *   - Each call made outside stream capture looks up the array's device address
+ *     (cudaGetSymbolAddress with the device current), so the address stays right after a
+ *     cudaDeviceReset or in another context of the device.  A call made while `stream`
+ *     is being captured reuses the address of the device's last uncaptured call; make at
+ *     least one uncaptured call on a device before capturing (otherwise
+ *     ATTN_SINK_ERR_CUDA).
  *   - All calls share the one array and it keeps the last call's contents.  Nothing in
  *     it has to start at zero (each call writes every slot it later reads), but calls
  *     whose kernels overlap on the GPU race on it: order them on one stream.

@@ -20,6 +20,8 @@
 // previous call's leftovers are never read.
 #include <stdint.h>
 
+#include <atomic>
+
 #include "attn_sink.h"
 
 namespace {
@@ -30,22 +32,37 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices];
+// Last address looked up per device, for calls made while the stream is being captured.
+std::atomic<void*> g_scratch_addr[kMaxDevices];
 
-// Device address of g_decode_scratch on the current device.  The array's name in host
-// code is only a host-side stand-in for the symbol, never a device address, so the
-// address is looked up once per device (with that device current) and cached.
-int scratch_address(void** out) {
+// Device address of g_decode_scratch in the current device's context, for a call on
+// `stream`.  The array's name in host code is only a host-side stand-in for the symbol,
+// never a device address, so the address comes from cudaGetSymbolAddress with the device
+// current.  It is looked up afresh on every call made outside stream capture: the module
+// holding the array is loaded per context, so after cudaDeviceReset (or in another context
+// of the same device) the array may sit elsewhere, and a cached address would then point
+// at memory this context does not own.  While `stream` is being captured no lookup is
+// made (it could load a module in the middle of a capture); the address recorded by the
+// device's last uncaptured call is used, and a capture that comes before any uncaptured
+// call on the device is refused.  The per-device record is atomic, so first calls from
+// several host threads at once do not race.
+int scratch_address(cudaStream_t stream, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_SINK_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return ATTN_SINK_ERR_UNSUPPORTED;
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr) return ATTN_SINK_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return ATTN_SINK_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone) {
+    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) return ATTN_SINK_ERR_CUDA;  // no uncaptured call on this device yet
+    *out = p;
+    return ATTN_SINK_OK;
   }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr) return ATTN_SINK_ERR_CUDA;
+  g_scratch_addr[dev].store(p, std::memory_order_release);
+  *out = p;
   return ATTN_SINK_OK;
 }
 
@@ -61,18 +78,23 @@ extern "C" int attn_sink_decode_noalloc(const attn_sink_params* params, const vo
   if (splits == 0) {
     splits = attn_sink_decode_num_splits(params);
     if (splits < 0) return ATTN_SINK_ERR_INVALID_ARG;  // params rejected
-    // shrink the automatic split count until the partials fit the fixed array
-    while (splits > 1 && attn_sink_decode_workspace_size(params, splits) > kNoAllocScratchBytes) {
-      const size_t need = attn_sink_decode_workspace_size(params, splits);
-      int next = (int)((double)splits * (double)kNoAllocScratchBytes / (double)need);
-      splits = next < splits ? (next > 0 ? next : 1) : splits - 1;
+    // the automatic count, or the largest count below it whose partials fit the fixed
+    // array (the workspace size grows with the split count)
+    if (attn_sink_decode_workspace_size(params, splits) > kNoAllocScratchBytes) {
+      int lo = 1, hi = splits;  // invariant: hi does not fit; the answer is in [1, hi)
+      while (hi - lo > 1) {
+        const int mid = lo + (hi - lo) / 2;
+        if (attn_sink_decode_workspace_size(params, mid) <= kNoAllocScratchBytes) lo = mid;
+        else hi = mid;
+      }
+      splits = lo;
     }
   }
   const size_t need = attn_sink_decode_workspace_size(params, splits);
   if (need == SIZE_MAX) return ATTN_SINK_ERR_INVALID_ARG;
   if (need > kNoAllocScratchBytes) return ATTN_SINK_ERR_WORKSPACE;  // beyond the fixed maximum
   void* scratch = nullptr;
-  const int st = scratch_address(&scratch);
+  const int st = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
   if (st != ATTN_SINK_OK) return st;
   return attn_sink_decode(params, q, k, v, cu_seqlens_k, sink, splits, out, lse, scratch,
                           kNoAllocScratchBytes, stream);

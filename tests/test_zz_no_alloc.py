@@ -5,14 +5,17 @@ fixed 16 MiB array inside the library instead of a caller workspace.
 
 Called through the C ABI with ctypes.  Its results must match attn_sink_decode's on the
 same inputs, within the bf16 tolerances the other tests use, on two calls in a row (the
-second call reuses the array the first one left behind).  The file name sorts last so
-that a run stopping at the first failure has already run every other test."""
+second call reuses the array the first one left behind), and the oracle's decode.  The
+file name sorts last so that a run stopping at the first failure has already run every
+other test."""
 import ctypes
 
+import numpy as np
 import pytest
 
 import workloads as W
 from _check import check_lse, check_out, to_np
+from oracle import ref
 
 pytestmark = pytest.mark.gpu
 
@@ -44,6 +47,13 @@ def _params(d, q, k, v, max_k):
                            head_dim_v=v.shape[2], softmax_scale=d.softmax_scale, causal=True)
 
 
+def _call(f, p, q, k, v, cu, sink, num_splits, out, lse):
+    import torch
+    return f(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), cu.data_ptr(),
+             sink.data_ptr(), num_splits, out.data_ptr(), None if lse is None else lse.data_ptr(),
+             torch.cuda.current_stream().cuda_stream)
+
+
 @pytest.mark.parametrize("num_splits,dim", [(0, 128), (5, 128), (0, 256)])
 def test_noalloc_decode_matches_workspace_decode_twice(num_splits, dim):
     import torch
@@ -54,29 +64,88 @@ def test_noalloc_decode_matches_workspace_decode_twice(num_splits, dim):
     max_k = 5000
     ref_out, ref_lse = sab.attn_sink_decode(q, k, v, cu, max_k, sink, d.softmax_scale, True,
                                             (-1, -1), num_splits)
+    ro, rl = ref.decode(d.q, d.k, d.v, d.cu_seqlens_k, d.sink, d.softmax_scale)
     p = _params(d, q, k, v, max_k)
-    stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):
         out = torch.full_like(ref_out, float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
-        st = f(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), cu.data_ptr(),
-               sink.data_ptr(), num_splits, out.data_ptr(), lse.data_ptr(), stream)
+        st = _call(f, p, q, k, v, cu, sink, num_splits, out, lse)
         assert st == 0, sab.lib().attn_sink_status_string(st)
         torch.cuda.synchronize()
         check_out(to_np(out), to_np(ref_out), "bf16", f"out (call {call + 1})")
         check_lse(to_np(lse), to_np(ref_lse), "bf16", f"lse (call {call + 1})")
+        # and against the oracle directly
+        check_out(to_np(out), ro, "bf16", f"out vs oracle (call {call + 1})")
+        check_lse(to_np(lse), rl, "bf16", f"lse vs oracle (call {call + 1})")
+
+
+# 64 sequences x 64 q heads: with one 2048-key sequence the automatic count is 8 splits of
+# 256 keys, whose partials (4096 rows x 8 splits x 520 bytes) need just over 16 MiB.
+_BIG_LENS = [2048] + [int(n) for n in np.random.default_rng(44).integers(1, 400, size=63)]
+
+
+def _largest_fitting(lib, p, upto):
+    best = 0
+    for s in range(1, upto + 1):
+        if lib.attn_sink_decode_workspace_size(ctypes.byref(p), s) <= SCRATCH_BYTES:
+            best = s
+    return best
+
+
+def test_noalloc_decode_lowers_the_automatic_split_count_to_fit():
+    import torch
+    import softmax_attn_sink_b200 as sab
+    L = sab.lib()
+    f = _noalloc_fn()
+    d = W.random_decode(43, _BIG_LENS, hq=64, hkv=8, dk=128, dv=128)
+    q, k, v, cu, sink = _inputs(d)
+    p = _params(d, q, k, v, 2048)
+    auto = L.attn_sink_decode_num_splits(ctypes.byref(p))
+    assert L.attn_sink_decode_workspace_size(ctypes.byref(p), auto) > SCRATCH_BYTES
+    fit = _largest_fitting(L, p, auto)
+    assert 1 <= fit < auto
+    ref_out, ref_lse = sab.attn_sink_decode(q, k, v, cu, 2048, sink, d.softmax_scale, True,
+                                            (-1, -1), fit)
+    for call in range(2):
+        out = torch.full_like(ref_out, float("nan"))
+        lse = torch.full_like(ref_lse, float("nan"))
+        st = _call(f, p, q, k, v, cu, sink, 0, out, lse)
+        assert st == 0, L.attn_sink_status_string(st)
+        torch.cuda.synchronize()
+        # the same kernels with the same split count: the same bits
+        assert torch.equal(out, ref_out), f"out differs from attn_sink_decode (call {call + 1})"
+        assert torch.equal(lse, ref_lse), f"lse differs from attn_sink_decode (call {call + 1})"
+    o, l = to_np(out), to_np(lse)
+    for b in (0, 1, 63):
+        k0, k1 = int(d.cu_seqlens_k[b]), int(d.cu_seqlens_k[b + 1])
+        for g in (0, 5):
+            heads = list(range(g * 8, g * 8 + 8))
+            ro, rl = ref.decode(d.q[b:b + 1, heads], d.k[k0:k1, g:g + 1], d.v[k0:k1, g:g + 1],
+                                np.array([0, k1 - k0]), d.sink[heads], d.softmax_scale)
+            check_out(o[b, heads], ro[0], "bf16", f"out[b={b},g={g}] vs oracle")
+            check_lse(l[heads, b], rl[:, 0], "bf16", f"lse[b={b},g={g}] vs oracle")
 
 
 def test_noalloc_decode_rejects_partials_beyond_the_fixed_array():
     import torch
     import softmax_attn_sink_b200 as sab
+    L = sab.lib()
     f = _noalloc_fn()
-    d = W.random_decode(42, [64, 64], hq=16, hkv=2, dk=128, dv=128)
+    d = W.random_decode(43, _BIG_LENS, hq=64, hkv=8, dk=128, dv=128)
     q, k, v, cu, sink = _inputs(d)
-    p = _params(d, q, k, v, 64)
-    per_split = 2 * 16 * (128 + 2) * 4
-    too_many = SCRATCH_BYTES // per_split + 8
-    out = torch.empty(2, 16, 128, dtype=torch.bfloat16, device="cuda")
-    st = f(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), cu.data_ptr(),
-           sink.data_ptr(), too_many, out.data_ptr(), None, torch.cuda.current_stream().cuda_stream)
+    p = _params(d, q, k, v, 2048)
+    # the smallest explicit count whose partials (by the library's own sizing) exceed 16 MiB
+    first_over = next(s for s in range(1, 4096)
+                      if L.attn_sink_decode_workspace_size(ctypes.byref(p), s) > SCRATCH_BYTES)
+    out = torch.full((64, 64, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((64, 64), float("nan"), dtype=torch.float32, device="cuda")
+    st = _call(f, p, q, k, v, cu, sink, first_over, out, lse)
     assert st == 3  # ATTN_SINK_ERR_WORKSPACE, returned before any launch
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all() and torch.isnan(lse).all(), "a rejected call wrote its outputs"
+    st = _call(f, p, q, k, v, cu, sink, first_over - 1, out, lse)
+    assert st == 0, L.attn_sink_status_string(st)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = sab.attn_sink_decode(q, k, v, cu, 2048, sink, d.softmax_scale, True,
+                                            (-1, -1), first_over - 1)
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
