@@ -1,6 +1,6 @@
 """The five workload configurations at full size, in the launch configuration bench.py
 times.  Small configs are compared element by element; large ones on sampled rows
-(and, for the backward, one whole (sequence, head) plus the full dsink of one head),
+(and, for the backward, whole (sequence, head) groups plus every dsink value),
 each sample computed by the oracle one by one."""
 
 import numpy as np
@@ -9,6 +9,7 @@ import pytest
 import workloads as W
 from oracle import ref
 from _check import check_grad, check_lse, check_out, to_np
+from _oracle_pool import dsink_term, group_bwd, pool_map
 
 pytestmark = pytest.mark.gpu
 
@@ -71,22 +72,30 @@ def test_config3_training_fwd_bwd_sampled():
             idx = np.asarray(rows) + 8192 * b
             check_out(o[idx, h], ro, "bf16", f"out[b={b},h={h}]")
             check_lse(l[h, idx], rl, "bf16", f"lse[b={b},h={h}]")
-    # one whole (sequence, head) of the backward
-    b, g = 1, 5
-    gq, gk, gv, gs = ref.bwd_sequence_group(p.q, p.k, p.v, p.dout, *a, b=b, g=g)
-    sl = slice(8192 * b, 8192 * (b + 1))
-    check_grad(to_np(dq[sl, g]), gq[:, 0], "bf16", "dq")
-    check_grad(to_np(dk[sl, g]), gk, "bf16", "dk")
-    check_grad(to_np(dv[sl, g]), gv, "bf16", "dv")
-    # dsink of head g sums over all four sequences
-    total = gs[0]
-    for bb in (0, 2, 3):
-        q0, q1 = 8192 * bb, 8192 * (bb + 1)
-        r = ref.attend_head(p.q[q0:q1, g], p.k[q0:q1, g], p.v[q0:q1, g], float(p.sink[g]),
-                            p.softmax_scale, ref.allowed_mask(8192, 8192, True))
-        D = (r["out"] * p.dout[q0:q1, g].astype(np.float64)).sum(1)
-        total += -float((r["p_sink"] * D).sum())
-    check_grad(to_np(ds)[g:g + 1], np.array([total]), "bf16", "dsink")
+    # The backward runs the (sequence, kv head) groups in bands of 8 (four sequences x 16
+    # heads = 64 groups; each band is one sequence's heads 0-7 or 8-15): dq / dk / dv of
+    # every band's first group, and all 16 dsink values, each a sum over the four sequences.
+    firsts = [(b, g) for b in range(4) for g in (0, 8)]
+    sl = lambda b: slice(8192 * b, 8192 * (b + 1))  # noqa: E731
+    gitems = [(p.q[sl(b), g:g + 1], p.k[sl(b), g:g + 1], p.v[sl(b), g:g + 1], p.dout[sl(b), g:g + 1],
+               p.sink[g:g + 1], p.softmax_scale, True, -1, -1) for b, g in firsts]
+    ditems = [(p.q[sl(b), h], p.k[sl(b), h], p.v[sl(b), h], p.dout[sl(b), h], float(p.sink[h]),
+               p.softmax_scale, True, -1, -1) for b in range(4) for h in range(16) if (b, h) not in firsts]
+    dkeys = [(b, h) for b in range(4) for h in range(16) if (b, h) not in firsts]
+    gres = pool_map(group_bwd, gitems)
+    dres = pool_map(dsink_term, ditems)
+    gdq, gdk, gdv = to_np(dq), to_np(dk), to_np(dv)
+    total = np.zeros(16)
+    for (b, g), (rq, rk, rv, rs) in zip(firsts, gres):
+        check_grad(gdq[sl(b), g], rq[:, 0], "bf16", f"dq[b={b},h={g}]")
+        check_grad(gdk[sl(b), g], rk, "bf16", f"dk[b={b},g={g}]")
+        check_grad(gdv[sl(b), g], rv, "bf16", f"dv[b={b},g={g}]")
+        total[g] += rs[0]
+    for (b, h), t in zip(dkeys, dres):
+        total[h] += t
+    print("dsink gpu   ", np.array2string(to_np(ds), precision=5, max_line_width=200))
+    print("dsink oracle", np.array2string(total, precision=5, max_line_width=200))
+    check_grad(to_np(ds), total, "bf16", "dsink")
 
 
 def test_config3_training_with_dropout_sampled():
