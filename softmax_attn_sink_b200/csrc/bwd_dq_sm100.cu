@@ -411,12 +411,14 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 
 // ---- host -----------------------------------------------------------------------------------
 
-template <typename Elem, int DK, int DV>
+// DVO <= DV: the width of v and dout in memory; with DVO = 32 their tiles are 64-column boxes
+// whose columns 32-63 the copies fill with zeros, which leaves dP = dout V^T exact.
+template <typename Elem, int DK, int DV, int DVO = DV>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   constexpr CUtensorMapDataType dt = tma_dtype<Elem>();
   CUtensorMap tq, tk, tv, to;
   if (!make_map_3d(&tq, a.q, DK, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, DK, a.hkv, a.total_k, 128, dt) ||
-      !make_map_3d(&tv, a.v, DV, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DV, a.hq, a.total_q, 128, dt))
+      !make_map_3d(&tv, a.v, DVO, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DVO, a.hq, a.total_q, 128, dt))
     return cudaErrorInvalidValue;
   const bool drop = a.drop.threshold != 0;
   auto kernel = drop ? bwd_dq_sm100_kernel<Elem, DK, DV, true> : bwd_dq_sm100_kernel<Elem, DK, DV, false>;
@@ -434,6 +436,8 @@ cudaError_t launch_dims(const BwdArgs& a, cudaStream_t s) {
   if (a.dk == 128 && a.dv == 64) return launch_typed<Elem, 128, 64>(a, s);
   if (a.dk == 64 && a.dv == 64) return launch_typed<Elem, 64, 64>(a, s);
   if (a.dk == 64 && a.dv == 128) return launch_typed<Elem, 64, 128>(a, s);
+  if (a.dk == 128 && a.dv == 32) return launch_typed<Elem, 128, 64, 32>(a, s);
+  if (a.dk == 64 && a.dv == 32) return launch_typed<Elem, 64, 64, 32>(a, s);
   return cudaErrorInvalidValue;
 }
 
@@ -441,7 +445,7 @@ cudaError_t launch_dims(const BwdArgs& a, cudaStream_t s) {
 
 bool bwd_dq_sm100_supported(const BwdArgs& a, int dtype) {
   if (dtype != 0 && dtype != 2) return false;
-  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
+  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 32 || a.dv == 64 || a.dv == 128))) return false;
   if ((long long)((a.max_sq + kBM - 1) / kBM) * a.batch * a.hq > 0x7fffffffLL) return false;  // 1-D grid
   return encode_fn() != nullptr;
 }

@@ -117,7 +117,10 @@ struct BBars {
   __device__ __forceinline__ uint32_t drain() const { return base + 8u * 11; }
 };
 
-template <typename Elem, int DK, int DV, bool DQ, bool DROP = false>
+// DVO <= DV is the width of v, dout and dv in memory (DV that of the tiles and products):
+// with DVO = 32 the V and dout tiles are 64-column boxes over 32-column tensors, whose
+// columns 32-63 the copies fill with zeros, so dP is exact and dV's columns 32-63 stay zero.
+template <typename Elem, int DK, int DV, bool DQ, bool DROP = false, int DVO = DV>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do) {
@@ -359,10 +362,10 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
     const bool have = __all_sync(0xffffffffu, ok && T > 0 && mbar_wait(bar.ds_free(), (T - 1) & 1, a.status));
     tc_fence_after();
     Elem* dkp = static_cast<Elem*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
-    Elem* dvp = static_cast<Elem*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
+    Elem* dvp = static_cast<Elem*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DVO;
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
-      const int ncol = pass == 0 ? DK : DV;
+      const int ncol = pass == 0 ? DK : DVO;
       const uint32_t col = pass == 0 ? kColDK : kColDV;
       const float mul = pass == 0 ? a.scale : (DROP ? a.drop.scale : 1.f);
       uint4* dst = reinterpret_cast<uint4*>(pass == 0 ? dkp : dvp);
@@ -511,7 +514,7 @@ struct PBars {
 
 
 
-template <typename Elem, int DV, bool DQ, bool DROP>
+template <typename Elem, int DV, bool DQ, bool DROP, int DVO = DV>
 __global__ void __launch_bounds__(kThreadsP, 1)
 bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -833,10 +836,10 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     const bool have = __all_sync(0xffffffffu, ok && T > 0 && mbar_wait(bar.ds_free(1), (T - 1) & 1, a.status));
     tc_fence_after();
     Elem* dkp = static_cast<Elem*>(a.grad_k) + ((k0 + j) * a.hkv + g) * DK;
-    Elem* dvp = static_cast<Elem*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DV;
+    Elem* dvp = static_cast<Elem*>(a.grad_v) + ((k0 + j) * a.hkv + g) * DVO;
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
-      const int ncol = pass == 0 ? DK : DV;
+      const int ncol = pass == 0 ? DK : DVO;
       const uint32_t col = pass == 0 ? kColDK : kColDV;
       const float mul = pass == 0 ? a.scale : (DROP ? a.drop.scale : 1.f);
       uint4* dst = reinterpret_cast<uint4*>(pass == 0 ? dkp : dvp);
@@ -940,20 +943,21 @@ template <typename T> constexpr int dtype_code();
 template <> constexpr int dtype_code<__nv_bfloat16>() { return 0; }
 template <> constexpr int dtype_code<__half>() { return 2; }
 
-template <typename T, int DV>
+template <typename T, int DV, int DVO = DV>
 cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   using L = PLayout<DV>;
   constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tq, tk, tv, to;
   if (!make_map_3d(&tq, a.q, 128, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, 128, a.hkv, a.total_k, 128, dt) ||
-      !make_map_3d(&tv, a.v, DV, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DV, a.hq, a.total_q, 128, dt))
+      !make_map_3d(&tv, a.v, DVO, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DVO, a.hq, a.total_q, 128, dt))
     return cudaErrorInvalidValue;
   const bool dq = a.dq_acc != nullptr;
   cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * 128 * sizeof(float), s) : cudaSuccess;
   if (e != cudaSuccess) return e;
   if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
-  auto kernel = dq ? bwd_sm100_d128_kernel<T, DV, true, false>
-                  : (a.drop.threshold ? bwd_sm100_d128_kernel<T, DV, false, true> : bwd_sm100_d128_kernel<T, DV, false, false>);
+  auto kernel = dq ? bwd_sm100_d128_kernel<T, DV, true, false, DVO>
+                  : (a.drop.threshold ? bwd_sm100_d128_kernel<T, DV, false, true, DVO>
+                                      : bwd_sm100_d128_kernel<T, DV, false, false, DVO>);
   if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) != cudaSuccess)
     return e;
   BwdArgs ab = a;
@@ -968,20 +972,20 @@ cudaError_t launch_d128(const BwdArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, int DVO = DV>
 cudaError_t launch_typed(const BwdArgs& a, cudaStream_t s) {
   constexpr CUtensorMapDataType dt = tma_dtype<T>();
   CUtensorMap tq, tk, tv, to;
   if (!make_map_3d(&tq, a.q, DK, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, DK, a.hkv, a.total_k, 128, dt) ||
-      !make_map_3d(&tv, a.v, DV, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DV, a.hq, a.total_q, 128, dt))
+      !make_map_3d(&tv, a.v, DVO, a.hkv, a.total_k, 128, dt) || !make_map_3d(&to, a.dout, DVO, a.hq, a.total_q, 128, dt))
     return cudaErrorInvalidValue;
   const bool dq = a.dq_acc != nullptr;
   cudaError_t e = dq ? cudaMemsetAsync(a.dq_acc, 0, (size_t)a.total_q * a.hq * DK * sizeof(float), s) : cudaSuccess;
   if (e != cudaSuccess) return e;
   if ((e = launch_bwd_preprocess(a, dtype_code<T>(), s)) != cudaSuccess) return e;
   const bool drop = !dq && a.drop.threshold != 0;
-  auto kernel = dq ? bwd_sm100_kernel<T, DK, DV, true>
-                   : (drop ? bwd_sm100_kernel<T, DK, DV, false, true> : bwd_sm100_kernel<T, DK, DV, false>);
+  auto kernel = dq ? bwd_sm100_kernel<T, DK, DV, true, false, DVO>
+                   : (drop ? bwd_sm100_kernel<T, DK, DV, false, true, DVO> : bwd_sm100_kernel<T, DK, DV, false, false, DVO>);
   const int smem = drop ? BLayout<DK, DV, true>::kSmem : BLayout<DK, DV>::kSmem;
   if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
     return e;
@@ -1002,6 +1006,9 @@ cudaError_t launch_dims(const BwdArgs& a, cudaStream_t s) {
   if (a.dk == 128 && a.dv == 64) return launch_d128<T, 64>(a, s);
   if (a.dk == 64 && a.dv == 64) return launch_typed<T, 64, 64>(a, s);
   if (a.dk == 64 && a.dv == 128) return launch_typed<T, 64, 128>(a, s);
+  // dv = 32: 64-wide V / dout tiles over zero-filled columns
+  if (a.dk == 128 && a.dv == 32) return launch_d128<T, 64, 32>(a, s);
+  if (a.dk == 64 && a.dv == 32) return launch_typed<T, 64, 64, 32>(a, s);
   return cudaErrorInvalidValue;
 }
 
@@ -1009,7 +1016,7 @@ cudaError_t launch_dims(const BwdArgs& a, cudaStream_t s) {
 
 bool bwd_sm100_supported(const BwdArgs& a, int dtype) {
   if (dtype != 0 && dtype != 2) return false;
-  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
+  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 32 || a.dv == 64 || a.dv == 128))) return false;
   if ((long long)a.batch * a.hkv * ((a.max_sk + kBN - 1) / kBN) > 0x7fffffffLL) return false;  // 1-D grid
   return encode_fn() != nullptr;
 }

@@ -314,7 +314,11 @@ struct ItemDesc {
 };
 static_assert(sizeof(ItemDesc) == 128, "item slot size");
 
-template <typename T, int DK, int DV, bool DROP>
+// DV is the width of the PV product and of V's shared-memory tile (64 or 128); DVO <= DV is
+// the width of v and out in memory.  With DVO = 32, V is loaded as a 64-column box over a
+// 32-column tensor, whose columns 32-63 the copy fills with zeros, so O's columns 32-63 stay
+// zero and only the first 32 are stored.
+template <typename T, int DK, int DV, int DVO, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -595,9 +599,10 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     const uint32_t tS = tmem + lane_off + col_S(u), tO = tmem + lane_off + col_O(u);
     const float scale2 = a.scale * kLog2e;
-    const uint32_t stg = sc.stage_off ? base_u32 + (uint32_t)sc.stage_off + (uint32_t)(warp - 4) * L::kStageBytes : 0u;
+    // the staged store moves 64-column (128-byte) row segments
+    const uint32_t stg = (DVO % 64 == 0 && sc.stage_off) ? base_u32 + (uint32_t)sc.stage_off + (uint32_t)(warp - 4) * L::kStageBytes : 0u;
     int sc_u = 0;  // S tiles of this unit taken so far (s_full / pv_done phases)
-    constexpr int kChunks = DV / 32;
+    constexpr int kChunks = DVO / 32;
     // Epilogue of an item: out = O / (l + 2^{sink2 - m}),  lse = (m + log2 l) ln 2.  Without
     // dropout it is deferred to the unit's next item: after that item's first softmax the
     // warps read O (its first S being ready means every earlier PV of the unit is complete),
@@ -630,12 +635,12 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
             const int rr = 4 * k + (lane >> 3), ch = lane & 7;
             const uint4 w = ld_shared_v4(stg + rr * 128 + ((ch ^ (rr & 7)) << 4));
             if (rr < e_nrow)
-              *reinterpret_cast<uint4*>(out + ((e_grow - lane + rr) * a.hq + e_h) * DV + (cc >> 1) * 64 + ch * 8) = w;
+              *reinterpret_cast<uint4*>(out + ((e_grow - lane + rr) * a.hq + e_h) * DVO + (cc >> 1) * 64 + ch * 8) = w;
           }
           __syncwarp();
         }
       } else if (e_row) {
-        uint4* orow = reinterpret_cast<uint4*>(out + (e_grow * a.hq + e_h) * DV);
+        uint4* orow = reinterpret_cast<uint4*>(out + (e_grow * a.hq + e_h) * DVO);
 #pragma unroll
         for (int v = 0; v < 4; ++v)
           orow[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
@@ -771,7 +776,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           }
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < DV / 32; ++c) {
+          for (int c = 0; c < DVO / 32; ++c) {
             uint32_t o[32];
             tmem_ld32(tO + c * 32, o);
             tmem_wait_ld();
@@ -893,7 +898,7 @@ void schedule_shape(const FwdArgs& a, int& zmax, int& width) {
 }
 
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, int DVO = DV>
 cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   using L = Layout<DK, DV>;
   int zmax, width;
@@ -905,7 +910,7 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   constexpr CUtensorMapDataType dt = tma_dtype<T>();
   if (!make_map_3d(&tq, a.q, DK, a.hq, a.total_q, 128, dt) || !make_map_3d(&tk, a.k, DK, a.hkv, a.total_k, 128, dt) ||
-      !make_map_3d(&tv, a.v, DV, a.hkv, a.total_k, 128, dt))
+      !make_map_3d(&tv, a.v, DVO, a.hkv, a.total_k, 128, dt))
     return cudaErrorInvalidValue;
   // Persistent launch (one CTA per SM walking the item list) when the item table fits in
   // shared memory; otherwise one CTA per item of the dense (level, sequence, unit pair) grid.
@@ -915,19 +920,20 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   const long long tbl = 3LL * zmax + a.batch;
   Sched sc{zmax, width, 1, 0};
   long long smem;
-  if (L::smem_bytes(tbl, true) <= dev.smem_optin) {
+  constexpr bool kStageable = DVO % 64 == 0;
+  if (kStageable && L::smem_bytes(tbl, true) <= dev.smem_optin) {
     sc.stage_off = (int)L::stage_offset(tbl);
     smem = L::smem_bytes(tbl, true);
   } else if (L::smem_bytes(tbl, false) <= dev.smem_optin) {
     smem = L::smem_bytes(tbl, false);
   } else {
     sc.persistent = 0;
-    const bool st = L::smem_bytes(0, true) <= dev.smem_optin;
+    const bool st = kStageable && L::smem_bytes(0, true) <= dev.smem_optin;
     sc.stage_off = st ? (int)L::stage_offset(0) : 0;
     smem = L::smem_bytes(0, st);
   }
   const long long grid = sc.persistent ? (items_ub < dev.sms ? items_ub : dev.sms) : items_ub;
-  auto kernel = a.drop.threshold ? fwd_sm100_kernel<T, DK, DV, true> : fwd_sm100_kernel<T, DK, DV, false>;
+  auto kernel = a.drop.threshold ? fwd_sm100_kernel<T, DK, DV, DVO, true> : fwd_sm100_kernel<T, DK, DV, DVO, false>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kernel<<<(unsigned)grid, kThreads, (size_t)smem, s>>>(a, sc, tq, tk, tv);
@@ -938,7 +944,7 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
 
 bool fwd_sm100_supported(const FwdArgs& a, int dtype) {
   if ((dtype != 0 && dtype != 2) || a.cu_q == nullptr) return false;
-  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return false;
+  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 32 || a.dv == 64 || a.dv == 128))) return false;
   int zmax, width;
   schedule_shape(a, zmax, width);
   if ((long long)zmax * a.batch * width > 0x7fffffffLL) return false;  // item numbers are 32-bit
@@ -952,6 +958,9 @@ cudaError_t launch_dims(const FwdArgs& a, cudaStream_t s) {
   if (a.dk == 128 && a.dv == 64) return launch_typed<T, 128, 64>(a, s);
   if (a.dk == 64 && a.dv == 64) return launch_typed<T, 64, 64>(a, s);
   if (a.dk == 64 && a.dv == 128) return launch_typed<T, 64, 128>(a, s);
+  // dv = 32: a 64-wide PV over zero-filled V columns
+  if (a.dk == 64 && a.dv == 32) return launch_typed<T, 64, 64, 32>(a, s);
+  if (a.dk == 128 && a.dv == 32) return launch_typed<T, 128, 64, 32>(a, s);
   return cudaErrorInvalidValue;
 }
 }  // namespace

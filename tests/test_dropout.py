@@ -50,6 +50,7 @@ FWD_CASES = [
     ("persistent_many_items_p15", _LENS_P, _LENS_P, 6, 2, 128, 128, True, -1, -1, "normal", "bf16",
      0.15),
     ("grid_mode_p10", _LENS_G, _LENS_G, 2, 1, 128, 128, True, -1, -1, "normal", "bf16", 0.1),
+    ("dk64_dv32_window_p10", [300, 129], [333, 200], 2, 1, 64, 32, True, 100, 0, "normal", "bf16", 0.1),
     ("d256_causal_gqa_p20", [300, 129, 0, 257], [300, 129, 0, 257], 4, 2, 256, 256, True, -1, -1,
      "normal", "bf16", 0.2),
     ("d256_fp16_window_p10", [200, 65], [230, 90], 2, 1, 256, 256, True, 70, 0, "normal", "fp16", 0.1),
@@ -89,6 +90,9 @@ BWD_CASES += [
     # head dim 64 (the dv field reads "64x<dv>"): the d = 64 dK/dV kernel with dropout
     ("dk64_dv64_causal_gqa_p20", [1, 129, 0, 257], [1, 129, 0, 257], 4, 2, "64x64", True, -1, -1,
      "normal", "bf16", 0.2),
+    ("dk64_dv32_causal_p20", [1, 129, 0, 257], [1, 129, 0, 257], 4, 2, "64x32", True, -1, -1,
+     "normal", "bf16", 0.2),
+    ("dk128_dv32_window_p10", [300, 70], [333, 90], 2, 1, "128x32", True, 100, 0, "normal", "bf16", 0.1),
     ("dk64_dv128_fp16_window_p10", [300, 70], [333, 90], 4, 1, "64x128", True, 100, 0, "uniform", "fp16",
      0.1),
 ]

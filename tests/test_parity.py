@@ -67,7 +67,12 @@ FWD_CASES = [
     ("fp16_causal_gqa", _LENS_B[:8], _LENS_B[:8], 8, 2, 128, 128, True, -1, -1, "normal", "fp16"),
     ("fp16_odd_group_window", [300, 129], [333, 200], 3, 1, 128, 64, True, 100, 0, "normal", "fp16"),
     ("fp16_dk64", [257, 64], [257, 64], 4, 2, 64, 64, False, -1, -1, "uniform", "fp16"),
-    ("fp16_dv32_simt", [190], [190], 2, 1, 128, 32, True, -1, -1, "normal", "fp16"),
+    # dv = 32 on the tensor cores: 64-wide PV over zero-filled V columns, 32 columns stored
+    ("fp16_dv32", [190], [190], 2, 1, 128, 32, True, -1, -1, "normal", "fp16"),
+    ("dk64_dv32_varlen_gqa", [1, 127, 0, 129, 333], [1, 127, 0, 129, 340], 8, 2, 64, 32, True, -1, -1,
+     "normal", "bf16"),
+    ("dk64_dv32_odd_group_persistent", _LENS_A, _LENS_A, 3, 1, 64, 32, True, 200, 0, "uniform", "bf16"),
+    ("dk128_dv32_sq_ne_sk", [5, 100, 200, 7], [2, 300, 150, 0], 4, 2, 128, 32, True, -1, -1, "normal", "bf16"),
     # 9000 sequences: the item table would not fit in shared memory, so the forward runs one
     # CTA per item of the dense grid instead.
     ("grid_mode_many_sequences", _LENS_C, _LENS_C, 2, 1, 128, 128, True, -1, -1, "normal", "bf16"),
@@ -138,7 +143,10 @@ BWD_CASES = [
     ("fp16_varlen_gqa", [1, 129, 0, 257], [1, 129, 0, 257], 8, 2, 128, 128, True, -1, -1, "normal", "fp16"),
     ("fp16_dv64_window", [260], [300], 2, 1, 128, 64, True, 50, 0, "normal", "fp16"),
     ("fp16_dk64", [300, 131], [300, 131], 4, 1, 64, 64, True, -1, -1, "normal", "fp16"),
-    ("fp16_dv32_simt", [150, 90], [160, 90], 2, 1, 64, 32, True, 40, 0, "normal", "fp16"),
+    ("fp16_dv32", [150, 90], [160, 90], 2, 1, 64, 32, True, 40, 0, "normal", "fp16"),
+    ("dk64_dv32_varlen_gqa", [1, 129, 0, 257], [1, 129, 0, 300], 8, 2, 64, 32, True, -1, -1, "normal", "bf16"),
+    ("dk128_dv32_gqa_window", [300, 131], [333, 131], 4, 1, 128, 32, True, 100, 0, "normal", "bf16"),
+    ("dk128_dv32_full", [200, 65], [170, 65], 2, 2, 128, 32, False, -1, -1, "uniform", "fp16"),
     # head dim 256: the dQ / dK / dV tensor-core kernels (bf16, fp16); fp32 on the CUDA cores
     ("d256_causal_gqa", [1, 100, 0, 131], [1, 100, 0, 131], 4, 2, 256, 256, True, -1, -1, "normal", "bf16"),
     ("d256_fp16_window", [120], [150], 2, 2, 256, 256, True, 40, 0, "normal", "fp16"),
