@@ -422,7 +422,7 @@ def bench_fwd_d256(args, world, peaks, peak_kind):
                             steps, args.warmup, world, flush)
     achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
     pk = peaks["bf16_tflops"]
-    # backward (CUDA cores at this head dim): a few steps
+    # backward (preprocess + the tcgen05 dQ, dK and dV kernels of this head dim): a few steps
     do = torch.randn((tq, hq, d), generator=gen, device="cuda").to(torch.bfloat16)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dsink = torch.empty(hq, dtype=torch.float32, device="cuda")
@@ -475,6 +475,47 @@ def bench_fwd_d256(args, world, peaks, peak_kind):
                        "roofline": {"bound": "hbm", "achieved": round(da, 1), "peak": pb, "unit": "GB/s",
                                     "frac": round(da / pb, 4), "traffic": None,
                                     "kernels": "split + merge (two launches per step)"}}}
+
+
+def bench_small_configs(args, world, peaks, peak_kind):
+    """The two small forward configurations: 2 x 256 tokens, 4 heads, d 64, non-causal and
+    causal; and softmax_n (sink = log n, n in {1, 0.5, 3}) on 6 x (1024 queries, 1152 keys),
+    1 head, dk 64 / dv 32, bottom-right causal with a (512, 0) window.  Both launch far fewer
+    tiles than the GPU has SMs, so they measure launch latency and a short critical path,
+    not throughput; they are reported, not graded."""
+    import torch
+    import softmax_attn_sink_b200 as sab
+    flush = Flusher()
+    steps = max(10, min(args.steps, 100))
+    pk = peaks["bf16_tflops"]
+
+    def run(p, wl, wr):
+        td = torch.bfloat16
+        q, k, v = (torch.from_numpy(x).to(td).cuda() for x in (p.q, p.k, p.v))
+        cq, ck = torch.from_numpy(p.cu_seqlens_q).cuda(), torch.from_numpy(p.cu_seqlens_k).cuda()
+        sink = torch.from_numpy(p.sink).cuda()
+        out = torch.empty((q.shape[0], q.shape[1], v.shape[2]), dtype=td, device="cuda")
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device="cuda")
+        pairs = visible_pairs(p.cu_seqlens_q, p.cu_seqlens_k, q.shape[1], p.causal, wl, wr)
+        flops = 2 * (q.shape[2] + v.shape[2]) * pairs
+        per, total = time_steps(lambda: sab.attn_sink_fwd(q, k, v, cq, ck, p.max_seqlen_q, p.max_seqlen_k, sink,
+                                                          p.softmax_scale, p.causal, (wl, wr), out=out, lse=lse),
+                                steps, args.warmup, world, flush)
+        achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
+        return {"value": round(weak_scaling_value(flops, world, total, steps) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(total / steps, 5), "pairs": pairs, "flops": flops, "steps": steps,
+                "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": pk, "unit": "TFLOP/s",
+                             "frac": round(achieved / pk, 5), "traffic": None,
+                             "peak_source": f"bf16_tflops ({peak_kind}, burst)",
+                             "kernel": "fwd_sm100 (one launch per step; launch-latency bound)"}}
+
+    c1 = {"workload": "fixed2x256_h4_d64"}
+    for causal in (False, True):
+        c1["causal" if causal else "non_causal"] = run(W.config1(causal), -1, -1)
+    c4 = {"workload": "softmax_n_6x1024x1152_h1_dk64_dv32_causal_window512"}
+    for n in (1.0, 0.5, 3.0):
+        c4[f"n={n:g}"] = run(W.config4(n), 512, 0)
+    return {"config1": c1, "config4": c4}
 
 
 def bench_fwd_bwd(args, world, peaks, peak_kind):
@@ -694,7 +735,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all", "fwd", "fwd_fp16", "fwd_dropout", "fwd_d256", "fwd_bwd", "decode"],
+    ap.add_argument("--workload", choices=["all", "fwd", "fwd_fp16", "fwd_dropout", "fwd_d256", "fwd_bwd", "decode",
+                                           "small"],
                     default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", type=int, default=4, choices=[1, 2, 3, 4],
@@ -739,13 +781,17 @@ def main():
             extra["fwd_d256"] = bench_fwd_d256(args, world, peaks, peak_kind)
         if args.workload in ("all", "fwd_bwd"):
             extra["fwd_bwd"] = bench_fwd_bwd(args, world, peaks, peak_kind)
+        if args.workload in ("all", "small"):
+            extra.update(bench_small_configs(args, world, peaks, peak_kind))
         if args.workload in ("all", "decode"):
             extra["decode"] = bench_decode(args, world, peaks, peak_kind)
         if extra:
             line["extra"] = extra
         if "value" not in line:  # a single non-headline workload was asked for
-            key = args.workload
+            key = args.workload if args.workload != "small" else "config4"
             e = extra[key]
+            if key == "config4":
+                e = dict(e["n=1"], workload=e["workload"])
             v = e["fwd"]["value"] if key == "fwd_bwd" else e["value"]
             line.update({"value": v, "unit": e.get("unit", "TFLOP/s"),
                          "ms_per_step": e["fwd"]["ms_per_step"] if key == "fwd_bwd" else e["ms_per_step"],
