@@ -15,7 +15,8 @@
 // the K/V ring, the TMEM buffers and the mbarrier phases carry over from one item to the
 // next, so an item's Q load and first QK overlap the previous item's last tiles.  Warp roles:
 //   warp 0      TMA producer: Q_A, Q_B per item (once the previous item's last QK has read
-//               Q), then K and V tiles into a 2-stage ring.
+//               Q), then K and V tiles into a 2-stage ring; a stage's K and V are released
+//               together once both PVs of its tile are issued (one commit per tile).
 //   warp 1      TMEM allocation and the MMA issuer (one thread), in the order
 //                 PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1)
 //               so the tensor core works for one unit while the other unit's softmax runs;
@@ -37,7 +38,8 @@
 // over the first 64 columns of S_U once S_U has been read; the next QK_U into S_U is issued
 // after the PV_U that reads it, and MMAs from one thread execute in issue order.  Because a
 // commit tracks every earlier MMA of the thread, S_U(j) being ready also means PV_U(j-1) is
-// done.  Every mbarrier wait is bounded; a timeout sets the status word and the CTA drains
+// done: the lazy rescale of O needs no other wait, and pv_done is committed only after a
+// unit's last PV of an item, for its epilogue.  Every mbarrier wait is bounded; a timeout sets the status word and the CTA drains
 // and frees its TMEM instead of hanging.
 #include <cuda.h>
 
@@ -76,9 +78,9 @@ struct Layout {
   static constexpr int kOffK = kOffQ + 2 * kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKBytes;
   static constexpr int kOffBar = kOffV + kStages * kVBytes;
-  // q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-  // pv_done[2], drain, item_full[I], item_empty[I]
-  static constexpr int kNumBars = 2 + 4 * kStages + 7 + 2 * kItemSlots;
+  // q_full, q_empty, k_full[S], kv_empty[S], v_full[S], s_full[2], p_full[2], pv_done[2],
+  // drain, item_full[I], item_empty[I]
+  static constexpr int kNumBars = 2 + 3 * kStages + 7 + 2 * kItemSlots;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffItems = (kOffTmemSlot + 16 + 127) / 128 * 128;  // ItemDesc[kItemSlots]
   static constexpr int kOffTable = kOffItems + kItemSlots * 128;           // item list of a persistent launch
@@ -100,16 +102,16 @@ struct Bars {
   __device__ __forceinline__ uint32_t q_full() const { return base; }
   __device__ __forceinline__ uint32_t q_empty() const { return base + 8u; }
   __device__ __forceinline__ uint32_t k_full(int s) const { return base + 8u * (2 + s); }
-  __device__ __forceinline__ uint32_t k_empty(int s) const { return base + 8u * (2 + kStages + s); }
+  // K and V of a stage are released together, after the tile's last PV
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8u * (2 + kStages + s); }
   __device__ __forceinline__ uint32_t v_full(int s) const { return base + 8u * (2 + 2 * kStages + s); }
-  __device__ __forceinline__ uint32_t v_empty(int s) const { return base + 8u * (2 + 3 * kStages + s); }
-  __device__ __forceinline__ uint32_t s_full(int u) const { return base + 8u * (2 + 4 * kStages + u); }
-  __device__ __forceinline__ uint32_t p_full(int u) const { return base + 8u * (4 + 4 * kStages + u); }
-  __device__ __forceinline__ uint32_t pv_done(int u) const { return base + 8u * (6 + 4 * kStages + u); }
-  __device__ __forceinline__ uint32_t drain() const { return base + 8u * (8 + 4 * kStages); }
-  __device__ __forceinline__ uint32_t item_full(int s) const { return base + 8u * (9 + 4 * kStages + s); }
+  __device__ __forceinline__ uint32_t s_full(int u) const { return base + 8u * (2 + 3 * kStages + u); }
+  __device__ __forceinline__ uint32_t p_full(int u) const { return base + 8u * (4 + 3 * kStages + u); }
+  __device__ __forceinline__ uint32_t pv_done(int u) const { return base + 8u * (6 + 3 * kStages + u); }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * (8 + 3 * kStages); }
+  __device__ __forceinline__ uint32_t item_full(int s) const { return base + 8u * (9 + 3 * kStages + s); }
   __device__ __forceinline__ uint32_t item_empty(int s) const {
-    return base + 8u * (9 + 4 * kStages + kItemSlots + s);
+    return base + 8u * (9 + 3 * kStages + kItemSlots + s);
   }
 };
 
@@ -347,9 +349,8 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
     mbar_init(bar.q_empty(), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar.k_full(s), 1);
-      mbar_init(bar.k_empty(s), 1);
+      mbar_init(bar.kv_empty(s), 1);
       mbar_init(bar.v_full(s), 1);
-      mbar_init(bar.v_empty(s), 1);
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar.s_full(u), 1);
@@ -403,14 +404,10 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           const int st = kv % kStages;
           const uint32_t par = ((kv / kStages) & 1) ^ 1;
           const int row = k0 + lo + j * kBN;
-          if (!(ok = mbar_wait(bar.k_empty(st), par, a.status))) break;
+          if (!(ok = mbar_wait(bar.kv_empty(st), par, a.status))) break;
           mbar_arrive_expect_tx(bar.k_full(st), L::kKBytes);
           for (int hf = 0; hf < L::KH; ++hf)
             tma_load_3d(sK + st * L::kKBytes + hf * L::kHalfBytes, &tm_k, bar.k_full(st), hf * 64, g, row);
-          if (!(ok = mbar_wait(bar.v_empty(st), par, a.status))) {
-            ++kv;  // K of this tile is in flight
-            break;
-          }
           mbar_arrive_expect_tx(bar.v_full(st), L::kVBytes);
           for (int hf = 0; hf < L::VH; ++hf)
             tma_load_3d(sV + st * L::kVBytes + hf * L::kHalfBytes, &tm_v, bar.v_full(st), hf * 64, g, row);
@@ -497,7 +494,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
             mma_ts_lo(dO, aP + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), desc_hi, idesc_pv, (!first || kk > 0) ? 1u : 0u);
-          mma_commit(bar.pv_done(u));
+          if (j + 1 == (u ? jB1 : jA1)) mma_commit(bar.pv_done(u));
           return true;
         };
         auto active = [&](int u, int j) { return u ? (j >= jB0 && j < jB1) : (j >= jA0 && j < jA1); };
@@ -507,7 +504,6 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         if (!ok) break;
         qk0_issued = false;
         if (n == 1) mma_commit(bar.q_empty());  // every QK of the item is issued
-        mma_commit(bar.k_empty(kv % kStages));
         // V(j) is waited for one step ahead (while the previous QKs are still queued), so a
         // unit's P arrival finds this thread already waiting for it.
         if (!(ok = mbar_wait(bar.v_full(kv % kStages), (kv / kStages) & 1, a.status))) break;
@@ -517,7 +513,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
             if (active(u, j)) ok = issue_pv(u, j);
             if (!ok) break;
             if (u == 1) {
-              mma_commit(bar.v_empty(st));   // both PVs of tile j are issued
+              mma_commit(bar.kv_empty(st));   // both PVs of tile j are issued: K and V of tile j are free
               if (j + 1 < n && !(ok = mbar_wait(bar.v_full((p + 1) % kStages), ((p + 1) / kStages) & 1, a.status)))
                 break;
             }
@@ -540,7 +536,6 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           if (j + 1 < n) {
             // a tile no unit needs still has to be consumed for the producer's accounting
             if (!(ok = wait_k(j + 1))) break;
-            mma_commit(bar.k_empty((p + 1) % kStages));
           }
         }
         if (!ok) break;
@@ -601,7 +596,8 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
     const float scale2 = a.scale * kLog2e;
     // the staged store moves 64-column (128-byte) row segments
     const uint32_t stg = (DVO % 64 == 0 && sc.stage_off) ? base_u32 + (uint32_t)sc.stage_off + (uint32_t)(warp - 4) * L::kStageBytes : 0u;
-    int sc_u = 0;  // S tiles of this unit taken so far (s_full / pv_done phases)
+    int sc_u = 0;  // S tiles of this unit taken so far (s_full phases)
+    int ic_u = 0;  // items in which this unit had tiles (pv_done phases)
     constexpr int kChunks = DVO / 32;
     // Epilogue of an item: out = O / (l + 2^{sink2 - m}),  lse = (m + log2 l) ln 2.  Without
     // dropout it is deferred to the unit's next item: after that item's first softmax the
@@ -650,9 +646,10 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       if (e_row && a.lse) a.lse[(long long)e_h * a.total_q + e_grow] = e_lse;
     };
     // The pending epilogue, when the next item does not take its deferred path: wait for the
-    // unit's last PV (the sc_u-th pv_done phase), then read O and store it.
+    // unit's last PV (pv_done is committed once per item, after the unit's last PV), then
+    // read O and store it.
     auto flush = [&]() -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (sc_u - 1) & 1, a.status))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (ic_u - 1) & 1, a.status))) return false;
       tc_fence_after();
       uint32_t o[kChunks][32];
 #pragma unroll
@@ -686,7 +683,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         rhi = (int)(h_ - klo0);
       }
       float m = a.sink ? a.sink[h] * kLog2e : kNegInf, l = 0.f;
-      const int ph = sc_u - j0;                   // s_full / pv_done phase of tile j is ph + j
+      const int ph = sc_u - j0;                   // s_full phase of tile j is ph + j
       bool ok = true;
 
       for (int j = j0; j < j1; ++j) {
@@ -770,11 +767,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
 
         if (any_rescale && j > j0) {
           // O holds sum of the earlier P V: wait for the last of those MMAs, then scale rows
-          if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (ph + j - 1) & 1, a.status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+          // S(j) being ready means PV(j - 1) is complete (one issuing thread, commits in order)
 #pragma unroll
           for (int c = 0; c < DVO / 32; ++c) {
             uint32_t o[32];
@@ -810,6 +803,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       // ---- epilogue (see emit): record this item's output state -------------------------
       const bool have_o = j1 > j0;
       sc_u += j1 - j0;
+      ic_u += have_o ? 1 : 0;
       {
         const float sink2 = a.sink ? a.sink[h] * kLog2e : kNegInf;
         const float e_sink = (sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m);
@@ -827,7 +821,7 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
         continue;
       }
       if (have_o) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (sc_u - 1) & 1, a.status))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.pv_done(u), (ic_u - 1) & 1, a.status))) break;
         tc_fence_after();
       }
       // O 32 columns at a time with dropout (whose flag words take the room), else at once
