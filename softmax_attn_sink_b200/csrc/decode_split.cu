@@ -19,7 +19,9 @@
 // 3-stage cp.async pipeline (16-byte copies, XOR-swizzled rows so ldmatrix is
 // conflict-free).  The two contractions per 16 keys (S = Q K^T over the head dim and
 // O += P V over the keys) use m16n8k16 MMAs (bf16 or f16 inputs) with fp32 accumulation; the query
-// heads form the M dimension.  Scores are kept in the log2 domain (scale * log2 e folded
+// heads form the M dimension.  S is summed over the head dim in independent partial sums (short
+// dependency chains), and at head dim 256 two warps share each 16-key group, each computing the
+// scores and half of the output columns.  Scores are kept in the log2 domain (scale * log2 e folded
 // into one multiply) and exponentiated with ex2.approx.
 #include <type_traits>
 
@@ -28,13 +30,18 @@
 namespace attn_sink {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kStageKeys = 64;     // keys per pipeline stage (16 per warp)
+constexpr int kKeyGroups = 4;      // 16-key groups of a stage
+constexpr int kStageKeys = 64;     // keys per pipeline stage (16 per key group)
 // pipeline depth: 3 stages (at head dim 256 64 KB a stage, 192 KB, one CTA per SM)
 template <int DK, int DV>
 __host__ __device__ constexpr int stages_of() { return 3; }
 template <int DK, int DV>
 __host__ __device__ constexpr int ctas_per_sm() { return DK + DV > 256 ? 1 : 2; }
+// Warps of a CTA: one per key group, or at head dim 256 (one CTA per SM) two per key group,
+// each computing the group's scores and half of its output columns, so that two warps per
+// SM sub-partition hide each other's MMA and shared-memory latencies.
+template <int DK, int DV>
+__host__ __device__ constexpr int warps_of() { return DK + DV > 256 ? 8 : 4; }
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -117,12 +124,14 @@ __device__ __forceinline__ void decode_range(const DecodeArgs& a, int b, long lo
 enum KvMode { kPacked = 0, kPagedSmemTable = 1, kPagedGlobalTable = 2 };
 
 template <typename T, int DK, int DV, int MODE>
-__global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_split_kernel(const DecodeArgs a,
+__global__ void __launch_bounds__(warps_of<DK, DV>() * 32, ctas_per_sm<DK, DV>()) decode_split_kernel(const DecodeArgs a,
                                                                                         int chunk, int extra_off) {
   constexpr int kStages = stages_of<DK, DV>();
   constexpr bool PAGED = MODE != kPacked;
   constexpr int KCH = DK / 8, VCH = DV / 8;        // 16-byte chunks per row
-  constexpr int KSTEPS = DK / 16, VTILES = DV / 8;
+  constexpr int kThr = warps_of<DK, DV>() * 32;
+  constexpr int DVW = DV * kKeyGroups / warps_of<DK, DV>();   // output columns per warp
+  constexpr int KSTEPS = DK / 16, VTILES = DVW / 8;
   constexpr int STAGE_BYTES = kStageKeys * (DK + DV) * 2;
   extern __shared__ __align__(128) unsigned char smem[];
 
@@ -140,6 +149,7 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
   const int nstages = (nkeys + kStageKeys - 1) / kStageKeys;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kg = warp % kKeyGroups, dh = warp / kKeyGroups;   // key group, output-column half
   const int h_base = g * group + hb * 16;
   const int nh = (group - hb * 16) < 16 ? (group - hb * 16) : 16;
   const T* kp = static_cast<const T*>(a.k);
@@ -159,7 +169,7 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
   const int* trow = PAGED ? a.block_table + (long long)b * a.max_blocks : nullptr;
   if constexpr (MODE == kPagedSmemTable) {
     const int n_blk = (int)((c_hi - 1) / bs - blk_first + 1);
-    for (int i = tid; i < n_blk; i += kWarps * 32) s_blk[i] = trow[blk_first + i];
+    for (int i = tid; i < n_blk; i += kThr) s_blk[i] = trow[blk_first + i];
     __syncthreads();
   }
   auto compute_rows = [&](int st) {
@@ -190,23 +200,23 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
     const long long t0 = c_lo + (long long)st * kStageKeys;
     if constexpr (!PAGED && KCH == VCH) {
       // K and V rows of a key coincide: one address per copy pair
-      constexpr int NR = kStageKeys * KCH / (kWarps * 32);
+      constexpr int NR = kStageKeys * KCH / kThr;
 #pragma unroll
       for (int k = 0; k < NR; ++k) {
-        const int idx = tid + k * kWarps * 32, r = idx / KCH, ch = idx % KCH;
+        const int idx = tid + k * kThr, r = idx / KCH, ch = idx % KCH;
         const bool ok = t0 + r < c_hi;
         const long long base = ((k0 + t0 + r) * a.hkv + g) * DK + ch * 8;
         cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, ok ? kp + base : kp, ok);
         cp_async16(v_s + (r * VCH + swz<VCH>(r, ch)) * 16, ok ? vp + base : vp, ok);
       }
     } else if constexpr (!PAGED) {
-      for (int idx = tid; idx < kStageKeys * KCH; idx += kWarps * 32) {
+      for (int idx = tid; idx < kStageKeys * KCH; idx += kThr) {
         const int r = idx / KCH, ch = idx % KCH;
         const bool ok = t0 + r < c_hi;
         const T* src = ok ? kp + ((k0 + t0 + r) * a.hkv + g) * DK + ch * 8 : kp;
         cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, src, ok);
       }
-      for (int idx = tid; idx < kStageKeys * VCH; idx += kWarps * 32) {
+      for (int idx = tid; idx < kStageKeys * VCH; idx += kThr) {
         const int r = idx / VCH, ch = idx % VCH;
         const bool ok = t0 + r < c_hi;
         const T* src = ok ? vp + ((k0 + t0 + r) * a.hkv + g) * DV + ch * 8 : vp;
@@ -215,14 +225,14 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
     } else if constexpr (KCH == VCH && DK <= 128) {
       // K and V rows of a key coincide: every row this thread copies is read from shared
       // memory first, all loads before the first copy, then K and V are issued from them
-      constexpr int NR = kStageKeys * KCH / (kWarps * 32);
+      constexpr int NR = kStageKeys * KCH / kThr;
       const long long* rows = s_row + (st % kStages) * kStageKeys;
       long long rw[NR];
 #pragma unroll
-      for (int k = 0; k < NR; ++k) rw[k] = rows[(tid + k * kWarps * 32) / KCH];
+      for (int k = 0; k < NR; ++k) rw[k] = rows[(tid + k * kThr) / KCH];
 #pragma unroll
       for (int k = 0; k < NR; ++k) {
-        const int idx = tid + k * kWarps * 32, r = idx / KCH, ch = idx % KCH;
+        const int idx = tid + k * kThr, r = idx / KCH, ch = idx % KCH;
         const bool ok = rw[k] >= 0;
         const long long base = (rw[k] * a.hkv + g) * DK + ch * 8;
         cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, ok ? kp + base : kp, ok);
@@ -230,14 +240,14 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
       }
     } else {
       const long long* rows = s_row + (st % kStages) * kStageKeys;
-      for (int idx = tid; idx < kStageKeys * KCH; idx += kWarps * 32) {
+      for (int idx = tid; idx < kStageKeys * KCH; idx += kThr) {
         const int r = idx / KCH, ch = idx % KCH;
         const long long row = rows[r];
         const bool ok = row >= 0;
         const T* src = ok ? kp + (row * a.hkv + g) * DK + ch * 8 : kp;
         cp_async16(k_s + (r * KCH + swz<KCH>(r, ch)) * 16, src, ok);
       }
-      for (int idx = tid; idx < kStageKeys * VCH; idx += kWarps * 32) {
+      for (int idx = tid; idx < kStageKeys * VCH; idx += kThr) {
         const int r = idx / VCH, ch = idx % VCH;
         const long long row = rows[r];
         const bool ok = row >= 0;
@@ -289,12 +299,17 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
 
     const unsigned char* base = smem + (st % kStages) * STAGE_BYTES;
     const uint32_t k_s = smem_u32(base), v_s = smem_u32(base + kStageKeys * DK * 2);
-    const int key0 = warp * 16;                       // this warp's 16 keys of the stage
+    const int key0 = kg * 16;                         // this warp's 16 keys of the stage
     const long long t_abs = c_lo + (long long)st * kStageKeys + key0;
     if (t_abs >= c_hi) continue;                      // warp-uniform: nothing left for this warp
 
     // S = Q K^T  (two n8 tiles of 8 keys)
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    constexpr int NP = KSTEPS >= 8 ? 4 : 2;   // independent partial sums over the head dim
+    float sp[NP][2][4];
+#pragma unroll
+    for (int q_ = 0; q_ < NP; ++q_)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sp[q_][0][e] = sp[q_][1][e] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < KSTEPS; ++ks) {
       const int mi = lane >> 3, rr = lane & 7;
@@ -302,9 +317,19 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
       const int ch = ks * 2 + (mi & 1);
       uint32_t b0, b1, b2, b3;
       ldmatrix_x4(k_s + (row * KCH + swz<KCH>(row, ch)) * 16, b0, b1, b2, b3);
-      mma16816<T>(s[0], qa[ks], b0, b1);
-      mma16816<T>(s[1], qa[ks], b2, b3);
+      mma16816<T>(sp[ks % NP][0], qa[ks], b0, b1);
+      mma16816<T>(sp[ks % NP][1], qa[ks], b2, b3);
     }
+    float s[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float acc = sp[0][nt][e];
+#pragma unroll
+        for (int q_ = 1; q_ < NP; ++q_) acc += sp[q_][nt][e];
+        s[nt][e] = acc;
+      }
     // mask keys past the chunk end, online softmax in the log2 domain
     const int kc = (lane & 3) * 2;
     float mx[2] = {kNegInf, kNegInf};
@@ -354,7 +379,7 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
     for (int ntp = 0; ntp < VTILES / 2; ++ntp) {
       const int mi = lane >> 3, rr = lane & 7;
       const int row = key0 + (mi & 1) * 8 + rr;
-      const int ch = ntp * 2 + (mi >> 1);
+      const int ch = dh * (DVW / 8) + ntp * 2 + (mi >> 1);
       uint32_t b0, b1, b2, b3;
       ldmatrix_x4_trans(v_s + (row * VCH + swz<VCH>(row, ch)) * 16, b0, b1, b2, b3);
       mma16816<T>(o_acc[2 * ntp], pa, b0, b1);
@@ -364,39 +389,40 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm<DK, DV>()) decode_spl
   cp_async_wait<0>();
   __syncthreads();
 
-  // combine the 4 warps' states through shared memory (the stage buffers are free now)
-  float* s_o = reinterpret_cast<float*>(smem);                 // [kWarps][16][DV]
-  float* s_m = s_o + kWarps * 16 * DV;                          // [kWarps][16]
-  float* s_l = s_m + kWarps * 16;                               // [kWarps][16]
+  // combine the key groups' states through shared memory (the stage buffers are free now);
+  // the two warps of a key group at head dim 256 hold the same max and sum
+  float* s_o = reinterpret_cast<float*>(smem);                 // [kKeyGroups][16][DV]
+  float* s_m = s_o + kKeyGroups * 16 * DV;                      // [kKeyGroups][16]
+  float* s_l = s_m + kKeyGroups * 16;                           // [kKeyGroups][16]
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     float l = l_run[r];
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
     const int row = (lane >> 2) + r * 8;
-    if ((lane & 3) == 0) {
-      s_m[warp * 16 + row] = m_run[r];
-      s_l[warp * 16 + row] = l;
+    if ((lane & 3) == 0 && dh == 0) {
+      s_m[kg * 16 + row] = m_run[r];
+      s_l[kg * 16 + row] = l;
     }
   }
 #pragma unroll
   for (int nt = 0; nt < VTILES; ++nt) {
-    const int col = nt * 8 + (lane & 3) * 2, row = lane >> 2;
-    s_o[(warp * 16 + row) * DV + col] = o_acc[nt][0];
-    s_o[(warp * 16 + row) * DV + col + 1] = o_acc[nt][1];
-    s_o[(warp * 16 + row + 8) * DV + col] = o_acc[nt][2];
-    s_o[(warp * 16 + row + 8) * DV + col + 1] = o_acc[nt][3];
+    const int col = dh * DVW + nt * 8 + (lane & 3) * 2, row = lane >> 2;
+    s_o[(kg * 16 + row) * DV + col] = o_acc[nt][0];
+    s_o[(kg * 16 + row) * DV + col + 1] = o_acc[nt][1];
+    s_o[(kg * 16 + row + 8) * DV + col] = o_acc[nt][2];
+    s_o[(kg * 16 + row + 8) * DV + col + 1] = o_acc[nt][3];
   }
   __syncthreads();
-  for (int idx = tid; idx < nh * DV; idx += kWarps * 32) {
+  for (int idx = tid; idx < nh * DV; idx += kThr) {
     const int row = idx / DV, col = idx % DV;
     float m = kNegInf;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, s_m[w * 16 + row]);
+    for (int w = 0; w < kKeyGroups; ++w) m = fmaxf(m, s_m[w * 16 + row]);
     float o = 0.f, l = 0.f;
     if (m != kNegInf) {
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
+      for (int w = 0; w < kKeyGroups; ++w) {
         const float mw = s_m[w * 16 + row];
         const float f = (mw == kNegInf) ? 0.f : ex2(mw - m);
         o += f * s_o[(w * 16 + row) * DV + col];
@@ -463,7 +489,7 @@ cudaError_t launch_split(const DecodeArgs& a, int chunk, int smem, int extra_off
   if (e != cudaSuccess) return e;
   const int group = a.hq / a.hkv;
   dim3 grid(a.splits, a.hkv * ((group + 15) / 16), a.batch);
-  decode_split_kernel<T, DK, DV, MODE><<<grid, kWarps * 32, smem, s>>>(a, chunk, extra_off);
+  decode_split_kernel<T, DK, DV, MODE><<<grid, warps_of<DK, DV>() * 32, smem, s>>>(a, chunk, extra_off);
   return cudaGetLastError();
 }
 
@@ -476,7 +502,7 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t s) {
   constexpr int STAGE_BYTES = kStageKeys * (DK + DV) * 2;
   constexpr int kStages = stages_of<DK, DV>();
   constexpr int PIPE = kStages * STAGE_BYTES;
-  constexpr int COMBINE = kWarps * 16 * (DV + 2) * 4;
+  constexpr int COMBINE = kKeyGroups * 16 * (DV + 2) * 4;
   constexpr int SMEM = PIPE > COMBINE ? PIPE : COMBINE;
   (void)hblocks;
   const int ch = chunk > 0 ? chunk : 1;
