@@ -87,14 +87,16 @@ def source_digest(kernel_file: str) -> str:
     return h.hexdigest()[:16]
 
 
-def kernel_traffic(kernel_file: str):
-    """DRAM bytes per bench launch from profiles/traffic.txt, or None when the kernel's
-    sources have changed since that capture."""
+def kernel_traffic(kernel_file: str, leg: str = ""):
+    """DRAM bytes per bench launch from profiles/traffic.txt (the line labelled
+    ``kernel_file`` or ``kernel_file:leg``), or None when the kernel's sources have changed
+    since that capture."""
+    label = kernel_file + (":" + leg if leg else "")
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
             for line in f:
                 parts = line.split()
-                if parts and not line.startswith("#") and parts[0] == kernel_file:
+                if parts and not line.startswith("#") and parts[0] == label:
                     return int(parts[2]) if parts[1] == source_digest(kernel_file) else None
     except OSError:
         pass
@@ -473,7 +475,7 @@ def bench_fwd_d256(args, world, peaks, peak_kind):
             "decode": {"workload": "decode16_gqa32x4_d256_L8k-32k", "value": round(dbytes * world / (d_total / steps * 1e-3) / 1e9, 1),
                        "unit": "GB/s", "ms_per_step": round(d_total / steps, 4), "bytes_per_step": dbytes,
                        "roofline": {"bound": "hbm", "achieved": round(da, 1), "peak": pb, "unit": "GB/s",
-                                    "frac": round(da / pb, 4), "traffic": None,
+                                    "frac": round(da / pb, 4), "traffic": kernel_traffic("decode_split.cu", "d256"),
                                     "kernels": "split + merge (two launches per step)"}}}
 
 
