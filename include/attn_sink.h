@@ -123,7 +123,11 @@ typedef struct {
  * Forward (CANN doc, "Function" formula and softmax_lse formula; slime
  * learnable_softmax_flash_attn_varlen).  Writes out [total_q, Hq, dv] (dtype) and, when
  * `lse` is not NULL, lse [Hq, total_q] fp32.  sink may be NULL (= -inf).  The workspace
- * may be NULL when attn_sink_fwd_workspace_size() returns 0.
+ * (attn_sink_fwd_workspace_size() bytes, 16-byte aligned, contents ignored) holds the work
+ * counter the bf16/fp16 tensor-core forward's CTAs take their items from; the call zeroes
+ * it on `stream` first, so two forwards that overlap on the GPU need two workspaces.  A
+ * missing or smaller workspace returns ATTN_SINK_ERR_WORKSPACE on that path (the fp32 and
+ * head-dim-256 forwards do not read it).
  */
 int attn_sink_fwd(const attn_sink_params* params, const void* q, const void* k, const void* v,
                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const float* sink,
@@ -147,8 +151,8 @@ int attn_sink_bwd(const attn_sink_params* params, const void* q, const void* k, 
 
 /*
  * Forward and backward with dropout (see attn_sink_dropout); otherwise the arguments of
- * attn_sink_fwd / attn_sink_bwd.  Tensor-core paths only: bf16 or fp16 with head_dim_qk and
- * head_dim_v in {64, 128}, or 256 / 256 (ATTN_SINK_ERR_UNSUPPORTED
+ * attn_sink_fwd / attn_sink_bwd.  Tensor-core paths only: bf16 or fp16 with head_dim_qk in
+ * {64, 128} and head_dim_v in {32, 64, 128}, or 256 / 256 (ATTN_SINK_ERR_UNSUPPORTED
  * otherwise; ATTN_SINK_ERR_INVALID_ARG for a NULL dropout or p out of range).  The backward
  * takes the deterministic path (bit-identical results from run to run) and the workspace
  * attn_sink_bwd_workspace_size() gives.

@@ -36,6 +36,10 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // (dk, dv): 64 or 128 with 32, 64 or 128; and 256 with 256 (the CANN flash_attn doc lists
 // head dims 64, 128 and 256)
+// Forward workspace: one counter word of the persistent kernel's work queue, padded to 256
+// bytes.
+constexpr size_t kFwdWorkspaceBytes = 256;
+
 bool dims_supported(int dk, int dv) {
   return ((dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128)) || (dk == 256 && dv == 256);
 }
@@ -153,8 +157,6 @@ int run_fwd(const attn_sink_params* p, const void* q, const void* k, const void*
   for (const void* ptr : {q, k, v, (const void*)out})
     if (!aligned16(ptr)) return ATTN_SINK_ERR_INVALID_ARG;
   if ((lse && !aligned16(lse)) || (sink && !aligned16(sink))) return ATTN_SINK_ERR_INVALID_ARG;
-  (void)workspace;
-  (void)workspace_bytes;
   FwdArgs a{};
   if (!dropout_of(dropout, a.drop)) return ATTN_SINK_ERR_INVALID_ARG;
   a.q = q; a.k = k; a.v = v; a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k; a.sink = sink;
@@ -167,7 +169,12 @@ int run_fwd(const attn_sink_params* p, const void* q, const void* k, const void*
   a.status = status_ptr();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int dt = p->dtype;   // 0 bf16, 1 fp32, 2 fp16
-  if (fwd_sm100_supported(a, dt)) return from_cuda(launch_fwd_sm100(a, dt, s));
+  if (fwd_sm100_supported(a, dt)) {
+    // the persistent kernel's CTAs take their work items from a counter in the workspace
+    if (!workspace || workspace_bytes < kFwdWorkspaceBytes || !aligned16(workspace)) return ATTN_SINK_ERR_WORKSPACE;
+    a.work_counter = static_cast<unsigned*>(workspace);
+    return from_cuda(launch_fwd_sm100(a, dt, s));
+  }
   if (fwd_d256_sm100_supported(a, dt)) return from_cuda(launch_fwd_d256_sm100(a, dt, s));
   if (a.drop.threshold) return ATTN_SINK_ERR_UNSUPPORTED;   // dropout runs on the tensor-core path only
   return from_cuda(launch_fwd_simt(a, dt, s));
@@ -251,7 +258,7 @@ const char* attn_sink_status_string(int status) {
 
 size_t attn_sink_fwd_workspace_size(const attn_sink_params* p) {
   if (validate_params(p, false) != ATTN_SINK_OK) return SIZE_MAX;
-  return 0;
+  return kFwdWorkspaceBytes;
 }
 
 size_t attn_sink_bwd_workspace_size(const attn_sink_params* p) {

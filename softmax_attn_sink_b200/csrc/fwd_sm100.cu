@@ -119,13 +119,17 @@ struct Bars {
 //
 // A work item is one CTA's worth of work: a sequence b, a unit pair x (a head pair of a GQA
 // group when the group size is even, otherwise a head) and a level z (the row tile, or the
-// pair of row tiles, that the two units take).  Items are numbered level by level from the
-// deepest level down, and within a level by sequence and then unit pair.  Under a causal mask
-// an item's cost grows with its level, so this order is longest-first.
+// pair of row tiles, that the two units take).  In a persistent launch items are numbered
+// sequence by sequence, longest sequence first, and within a sequence from its deepest level
+// down, then by unit pair; the CTAs take them in that order from a shared counter, each
+// taking the next item as soon as it has room for one.  Under a causal mask an item's cost
+// grows with its level, so the first items are the longest and the ones that finish the
+// launch are short; and the CTAs working at any time read the K/V of one or two sequences,
+// which stay in L2 while every level of those sequences reads them.
 struct Sched {
   int zmax;        // levels of the longest sequence (bounded by max_seqlen_q)
   int width;       // unit pairs per (sequence, level)
-  int persistent;  // 1: the grid's CTAs walk the numbered list; 0: CTA i runs item i of the dense grid
+  int persistent;  // 1: the grid's CTAs take items from the counter; 0: CTA i runs item i of the dense grid
   int stage_off;   // byte offset of the output staging area from the aligned base; 0: none
 };
 
@@ -158,16 +162,19 @@ __device__ __forceinline__ void warp_suffix_sum(int* v, int n, int lane) {
 }
 
 // Item table of a persistent launch, built by one warp of every CTA (identical in all of them):
-//   cnt[z]   = sequences with more than z levels (the sequences present at level z),
-//   start[z] = number of the first item of level z,
-//   perm[j]  = the j-th sequence by descending level count (ties by index): the sequences
-//              present at level z are exactly perm[0, cnt[z]).
+//   start[j] = number of the first item of the j-th sequence of perm (start[j] = the total
+//              item count for j >= the number of sequences with rows),
+//   perm[j]  = the j-th sequence by descending level count (ties by index); sequences
+//              without rows are left out,
+// followed by two scratch arrays of the counting sort, cnt[z] (sequences with more than z
+// levels) and run[z].  Table ints: (B + 1) + B + 2 Z.
+constexpr long long table_ints(long long zmax, long long batch) { return 2 * batch + 1 + 2 * zmax; }
 __device__ void build_table(const FwdArgs& a, const Sched& sc, bool even, int* tbl, int lane) {
   const int Z = sc.zmax, B = a.batch, W = sc.width;
-  int* cnt = tbl;
-  int* start = tbl + Z;
-  int* run = tbl + 2 * Z;
-  int* perm = tbl + 3 * Z;
+  int* start = tbl;
+  int* perm = tbl + B + 1;
+  int* cnt = perm + B;
+  int* run = cnt + Z;
   for (int i = lane; i < Z; i += 32) cnt[i] = run[i] = 0;
   __syncwarp();
   for (int b = lane; b < B; b += 32) {
@@ -176,10 +183,6 @@ __device__ void build_table(const FwdArgs& a, const Sched& sc, bool even, int* t
   }
   __syncwarp();
   warp_suffix_sum(cnt, Z, lane);             // cnt[z] = sequences with more than z levels
-  for (int i = lane; i < Z; i += 32) start[i] = cnt[i];
-  __syncwarp();
-  warp_suffix_sum(start, Z, lane);
-  for (int i = lane; i < Z; i += 32) start[i] = W * (start[i] - cnt[i]);
   // stable counting sort of the sequences by descending level count
   for (int c0 = 0; c0 < B; c0 += 32) {
     const int b = c0 + lane;
@@ -191,36 +194,44 @@ __device__ void build_table(const FwdArgs& a, const Sched& sc, bool even, int* t
     if (nz > 0 && rank == 0) run[nz - 1] += __popc(peers);
     __syncwarp();
   }
+  // start[]: exclusive prefix sums of the sorted sequences' item counts, from an inclusive
+  // suffix sum: start[j] = total - sum_{k >= j} items(perm[k])
+  const int P = Z > 0 ? cnt[0] : 0;          // sequences with rows
+  for (int j = lane; j < P; j += 32) start[j] = W * levels_of(a, sc, even, perm[j]);
+  __syncwarp();
+  warp_suffix_sum(start, P, lane);
+  const int total = P > 0 ? start[0] : 0;
+  __syncwarp();
+  for (int j = lane; j <= B; j += 32) start[j] = j < P ? total - start[j] : total;
+  __syncwarp();
 }
 
-// Item of round r for this CTA.  Persistent CTAs walk the list in a snake: round r takes items
-// [r G, (r + 1) G), forward on even rounds and backward on odd ones, which keeps the
-// longest-first order balanced across the CTAs.  In grid mode CTA i runs item i only.
-__device__ __forceinline__ long long item_of_round(const Sched& sc, int r) {
-  const long long G = gridDim.x, c = blockIdx.x;
-  if (!sc.persistent) return r == 0 ? c : -1;
-  return (long long)r * G + ((r & 1) ? G - 1 - c : c);
+// The next item for this CTA: in a persistent launch the next number of the shared counter
+// (every CTA's scheduler takes its items one at a time, so they come in increasing order);
+// in grid mode CTA i runs item i only.
+__device__ __forceinline__ long long next_item(const Sched& sc, unsigned* counter, int r) {
+  if (!sc.persistent) return r == 0 ? (long long)blockIdx.x : -1;
+  return (long long)atomicAdd(counter, 1u);
 }
 
-// Decodes item t into (b, x, z).  `lvl` is a per-thread cursor over the levels (items of one
-// CTA come in increasing order, so it only moves down).  Returns false past the last item, or
-// for a grid-mode item whose sequence has no such level.
+// Decodes item t into (b, x, z).  `cur` is a per-thread cursor over perm (the items of one
+// CTA come in increasing order, so it only moves forward; start at 0).  Returns false past
+// the last item, or for a grid-mode item whose sequence has no such level.
 __device__ __forceinline__ bool decode_item(const FwdArgs& a, const Sched& sc, bool even, const int* tbl,
-                                            long long t, int& lvl, int& b, int& x, int& z) {
+                                            long long t, int& cur, int& b, int& x, int& z) {
   if (t < 0) return false;
   const int W = sc.width;
   if (sc.persistent) {
-    const int Z = sc.zmax;
-    const int* cnt = tbl;
-    const int* start = tbl + Z;
-    const int* perm = tbl + 3 * Z;
-    while (lvl >= 0 && t >= (long long)start[lvl] + (long long)W * cnt[lvl]) --lvl;
-    if (lvl < 0) return false;
-    const int r = (int)(t - start[lvl]);
-    const int j = r / W;
-    x = r - j * W;
-    b = perm[j];
-    z = lvl;
+    const int B = a.batch;
+    const int* start = tbl;
+    const int* perm = tbl + B + 1;
+    if (t >= (long long)start[B]) return false;
+    while (t >= (long long)start[cur + 1]) ++cur;
+    const int r = (int)(t - start[cur]);
+    const int lv = r / W;
+    x = r - lv * W;
+    b = perm[cur];
+    z = levels_of(a, sc, even, b) - 1 - lv;
     return true;
   }
   const long long per_level = (long long)a.batch * W;
@@ -331,8 +342,8 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
   const bool even = (group & 1) == 0;
   if (!sc.persistent) {
     // grid mode: a CTA whose item does not exist leaves before taking any resource
-    int lvl = 0, b, x, z;
-    if (!decode_item(a, sc, even, nullptr, blockIdx.x, lvl, b, x, z)) return;
+    int cur = 0, b, x, z;
+    if (!decode_item(a, sc, even, nullptr, blockIdx.x, cur, b, x, z)) return;
   }
   const uint32_t base_u32 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (base_u32 - smem_addr(smem_raw));
@@ -552,12 +563,12 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
     // ================================ scheduler ===========================================
     regs_dec<kRegsProducer>();
     if (lane == 0) {
-      int lvl = sc.zmax - 1;
+      int cur = 0;
       for (int r = 0;; ++r) {
         const int slot = r % kItemSlots;
         if (!mbar_wait(bar.item_empty(slot), ((r / kItemSlots) & 1) ^ 1, a.status)) break;
         int b, x, z;
-        const bool more = decode_item(a, sc, even, tbl, item_of_round(sc, r), lvl, b, x, z);
+        const bool more = decode_item(a, sc, even, tbl, next_item(sc, a.work_counter, r), cur, b, x, z);
         ItemDesc& d = items[slot];
         d.kind = more ? 1 : 0;
         if (more) {
@@ -911,7 +922,7 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
   const long long items_ub = (long long)zmax * a.batch * width;
   // The output staging area goes in when it fits beside the table (else rows are stored
   // directly from registers).
-  const long long tbl = 3LL * zmax + a.batch;
+  const long long tbl = table_ints(zmax, a.batch);
   Sched sc{zmax, width, 1, 0};
   long long smem;
   constexpr bool kStageable = DVO % 64 == 0;
@@ -927,6 +938,11 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t s) {
     smem = L::smem_bytes(0, st);
   }
   const long long grid = sc.persistent ? (items_ub < dev.sms ? items_ub : dev.sms) : items_ub;
+  if (sc.persistent) {
+    // the shared item counter starts at zero for every launch
+    if (a.work_counter == nullptr) return cudaErrorInvalidValue;
+    if ((e = cudaMemsetAsync(a.work_counter, 0, sizeof(unsigned), s)) != cudaSuccess) return e;
+  }
   auto kernel = a.drop.threshold ? fwd_sm100_kernel<T, DK, DV, DVO, true> : fwd_sm100_kernel<T, DK, DV, DVO, false>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -40,6 +40,7 @@ struct FwdArgs {
   int left, right;       // effective window (causal folded into right), kUnbounded = none
   unsigned* status;
   Dropout drop;          // threshold 0 = none (tensor-core path only)
+  unsigned* work_counter;  // workspace word the persistent forward's CTAs take items from (zeroed per launch)
 };
 
 struct BwdArgs {
