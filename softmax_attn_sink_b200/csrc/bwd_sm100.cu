@@ -737,10 +737,11 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     for (int t = 0; t < T; ++t) {
       const int h = head_of(t);
       const long long i0 = qbase_of(t);
-      // stage lse_tot * log2e and D of this tile's 128 queries (all 128 compute threads)
+      // stage -lse_tot * log2e and -D of this tile's 128 queries (all 128 compute threads);
+      // negated so that P's exponent and dP - D are single fused / packed operations
       named_bar_sync(1, 128);
-      s_lt[r] = pf_lt;
-      s_D[r] = pf_D;
+      s_lt[r] = -pf_lt;
+      s_D[r] = -pf_D;
       named_bar_sync(1, 128);
       if (t + 1 < T) prefetch(t + 1);   // in flight while this tile is computed
 #pragma unroll 1
@@ -772,18 +773,24 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(tmem + lane_off + cP + c * 32, dpv);
           tmem_wait_ld();
           const int qc = 64 * hh + 32 * c;           // first query of the chunk within the tile
-          float lt[32], dd[32];
+          float nlt[32], nd[32];   // -lse_tot * log2e, -D
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const float4 x = *reinterpret_cast<const float4*>(s_lt + qc + e);
             const float4 y = *reinterpret_cast<const float4*>(s_D + qc + e);
-            lt[e] = x.x; lt[e + 1] = x.y; lt[e + 2] = x.z; lt[e + 3] = x.w;
-            dd[e] = y.x; dd[e + 1] = y.y; dd[e + 2] = y.z; dd[e + 3] = y.w;
+            nlt[e] = x.x; nlt[e + 1] = x.y; nlt[e + 2] = x.z; nlt[e + 3] = x.w;
+            nd[e] = y.x; nd[e + 1] = y.y; nd[e + 2] = y.z; nd[e + 3] = y.w;
           }
           float p[32], ds[32];
           if (full) {
+            const float2 sc2 = make_float2(scale2, scale2);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) p[e] = ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e]));
+            for (int e = 0; e < 32; e += 2) {
+              const float2 x = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2,
+                                     make_float2(nlt[e], nlt[e + 1]));
+              p[e] = ex2(x.x);
+              p[e + 1] = ex2(x.y);
+            }
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -792,7 +799,7 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
               const long long d = j - (qi + off);
               if (a.right < kUnbounded) vis = vis && d <= a.right;
               if (a.left < kUnbounded) vis = vis && d >= -(long long)a.left;
-              p[e] = vis ? ex2(fmaf(__uint_as_float(sv[e]), scale2, -lt[e])) : 0.f;
+              p[e] = vis ? ex2(fmaf(__uint_as_float(sv[e]), scale2, nlt[e])) : 0.f;
             }
           }
           if constexpr (DROP) {
@@ -804,12 +811,18 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const uint32_t drop = prmt_sign_r(zb[e & 15], (e >> 4) ? sel1 : sel0);
-              ds[e] = p[e] * fmaf(__uint_as_float(dpv[e] & ~drop), zs, -dd[e]);
+              ds[e] = p[e] * fmaf(__uint_as_float(dpv[e] & ~drop), zs, nd[e]);
               p[e] = __uint_as_float(__float_as_uint(p[e]) & ~drop);
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ds[e] = p[e] * (__uint_as_float(dpv[e]) - dd[e]);
+            for (int e = 0; e < 32; e += 2) {
+              const float2 d = fmul2(make_float2(p[e], p[e + 1]),
+                                     fadd2(make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])),
+                                           make_float2(nd[e], nd[e + 1])));
+              ds[e] = d.x;
+              ds[e + 1] = d.y;
+            }
           }
           uint32_t pk[16], dk_[16];
 #pragma unroll
