@@ -326,10 +326,14 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                          : "memory");
           if (hh == 1) mbar_arrive(bar.rng_empty(j & 1));
         }
+        const float2 sc2 = make_float2(scale2, scale2), nlt2 = make_float2(neg_lt, neg_lt);
+        const float2 nD2 = make_float2(-Dr, -Dr);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), scale2, neg_lt));
-          const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), scale2, neg_lt));
+          // P's exponent for two keys in one packed fused multiply-add
+          const float2 x = ffma2(make_float2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sc2, nlt2);
+          const float p0 = ex2(x.x);
+          const float p1 = ex2(x.y);
           if constexpr (DROP) {
             // keys 2c, 2c + 1: bytes 0-1 (c even) or 2-3 (c odd) of flag word c / 2
             const uint4 w4 = kb4[c >> 3];
@@ -340,7 +344,9 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
             pk[c] = pack2<Elem>(p0 * fmaf(__uint_as_float(pv[2 * c] & ~d0), a.drop.scale, -Dr),
                                 p1 * fmaf(__uint_as_float(pv[2 * c + 1] & ~d1), a.drop.scale, -Dr));
           } else {
-            pk[c] = pack2<Elem>(p0 * (__uint_as_float(pv[2 * c]) - Dr), p1 * (__uint_as_float(pv[2 * c + 1]) - Dr));
+            const float2 d = fmul2(make_float2(p0, p1),
+                                   fadd2(make_float2(__uint_as_float(pv[2 * c]), __uint_as_float(pv[2 * c + 1])), nD2));
+            pk[c] = pack2<Elem>(d.x, d.y);
           }
         }
         // dS of keys [64 hh, 64 hh + 64) over S columns [32 hh, 32 hh + 32): half 0 goes over
