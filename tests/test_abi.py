@@ -161,16 +161,6 @@ def test_dropout_entry_points_validate_on_host(drop, change, status):
                                    a, ws, None) == status
 
 
-def test_bwd_dropout_needs_a_tensor_core_head_dim():
-    L = sab.lib()
-    p = _params(head_dim_qk=64, head_dim_v=32)   # dv = 32 runs on the CUDA cores
-    a = 1 << 20
-    d = sab.AttnSinkDropout(0.1, 1, 0)
-    ws = L.attn_sink_bwd_workspace_size(ctypes.byref(p))
-    assert L.attn_sink_bwd_dropout(ctypes.byref(p), a, a, a, a, a, a, a, a, None, ctypes.byref(d),
-                                   a, a, a, None, a, ws, None) == 2
-
-
 def test_dropout_struct_matches_header():
     text = open(HEADER).read()
     body = re.search(r"typedef struct \{([^{}]*)\} attn_sink_dropout;", text).group(1)
@@ -178,3 +168,31 @@ def test_dropout_struct_matches_header():
     names = re.findall(r"\b([a-z_]+)\s*;", body)
     assert names == [f[0] for f in sab.AttnSinkDropout._fields_]
     assert ctypes.sizeof(sab.AttnSinkDropout) == 24
+
+
+def test_fwd_workspace_size():
+    """The forward's workspace holds the work counter of the persistent tensor-core kernel."""
+    L = sab.lib()
+    assert L.attn_sink_fwd_workspace_size(ctypes.byref(_params())) == 256
+
+
+@pytest.mark.gpu
+def test_tensor_core_fwd_requires_its_workspace():
+    """Without the workspace attn_sink_fwd_workspace_size() asks for, the tensor-core
+    forward returns ATTN_SINK_ERR_WORKSPACE before any launch; with it, it runs."""
+    import torch
+    L = sab.lib()
+    q = torch.randn(64, 8, 128, device="cuda").to(torch.bfloat16)
+    k = torch.randn(64, 2, 128, device="cuda").to(torch.bfloat16)
+    cu = torch.tensor([0, 32, 64], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    p = _params()
+    stream = torch.cuda.current_stream().cuda_stream
+    args = (ctypes.byref(p), q.data_ptr(), k.data_ptr(), k.data_ptr(), cu.data_ptr(), cu.data_ptr(), None,
+            out.data_ptr(), None)
+    assert L.attn_sink_fwd(*args, None, 0, stream) == 3
+    ws = torch.empty(L.attn_sink_fwd_workspace_size(ctypes.byref(p)), dtype=torch.uint8, device="cuda")
+    assert L.attn_sink_fwd(*args, ws.data_ptr(), ws.numel() - 16, stream) == 3
+    assert L.attn_sink_fwd(*args, ws.data_ptr(), ws.numel(), stream) == 0
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
