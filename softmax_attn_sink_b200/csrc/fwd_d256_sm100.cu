@@ -72,17 +72,20 @@ struct Bars {
   __device__ __forceinline__ uint32_t o_done() const { return base + 8u * (7 + 4 * kStages); }
 };
 
-// CTA -> (row tile z, sequence b, q head h): the deepest row tiles first (under a causal mask
-// they see the most keys), heads fastest so that the CTAs of one GQA group run together and
-// share their K / V tiles in L2.  False for a row tile the sequence does not have.
+// CTA -> (sequence b, row tile z, q head h): sequence by sequence, within a sequence the
+// deepest row tiles first (under a causal mask they see the most keys), heads fastest so
+// that the CTAs of one GQA group run together.  The CTAs resident at any time then read the
+// K / V of one or two sequences, which stay in L2 while every row tile of those sequences
+// reads them; the hardware hands out CTAs in this order as SMs free up, which keeps the
+// load balanced.  False for a row tile the sequence does not have.
 __device__ __forceinline__ bool item_of(const FwdArgs& a, int zmax, int& z, int& b, int& h) {
   const long long id = blockIdx.x;
-  const long long per_level = (long long)a.batch * a.hq;
-  const int zr = (int)(id / per_level);
-  const int rem = (int)(id - (long long)zr * per_level);
+  const long long per_seq = (long long)zmax * a.hq;
+  b = (int)(id / per_seq);
+  const int rem = (int)(id - (long long)b * per_seq);
+  const int zr = rem / a.hq;
   z = zmax - 1 - zr;
-  b = rem / a.hq;
-  h = rem - b * a.hq;
+  h = rem - zr * a.hq;
   return (long long)z * kBM < (long long)(a.cu_q[b + 1] - a.cu_q[b]);
 }
 
