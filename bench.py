@@ -460,7 +460,7 @@ def bench_fwd_d256(args, world, peaks, peak_kind):
             "value": round(weak_scaling_value(flops, world, total, steps) / 1e12, 2),
             "ms_per_step": round(total / steps, 4), "flops": flops, "pairs": pairs,
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk, "unit": "TFLOP/s",
-                         "frac": round(achieved / pk, 4), "traffic": None,
+                         "frac": round(achieved / pk, 4), "traffic": kernel_traffic("fwd_d256_sm100.cu"),
                          "peak_source": f"bf16_tflops ({peak_kind}, burst)",
                          "kernel": "fwd_d256_sm100 (one launch per step)"},
             "bwd": {"value": round(bflops * world / (b_total / 3 * 1e-3) / 1e12, 2), "unit": "TFLOP/s",

@@ -268,9 +268,10 @@ const char* attn_sink_status_string(int status);
 /*
  * Synchronises `stream`, then reads and clears the calling device's status word.
  * Returns ATTN_SINK_OK, ATTN_SINK_ERR_TIMEOUT (a bounded wait ran out; bit 0),
- * ATTN_SINK_ERR_BAD_INDEX (an index or length outside its table was skipped, bit 1, or
- * attn_sink_check_seqlens found a broken cu_seqlens, bit 2) or ATTN_SINK_ERR_CUDA.  *bits
- * (if not NULL) receives the raw word.
+ * ATTN_SINK_ERR_BAD_INDEX (an index or length outside its table was skipped, bit 1;
+ * attn_sink_check_seqlens found a broken cu_seqlens, bit 2; or, in the debug build
+ * libattn_sink_debug.so only, a kernel skipped a store whose index range left the output
+ * it writes, bit 3) or ATTN_SINK_ERR_CUDA.  *bits (if not NULL) receives the raw word.
  */
 int attn_sink_get_device_status(attn_sink_stream_t stream, uint32_t* bits);
 

@@ -20,7 +20,9 @@ import os
 from typing import Optional, Sequence, Tuple
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libattn_sink.so")
+# ATTN_SINK_LIBRARY selects another build of the library (e.g. the bounds-checking
+# libattn_sink_debug.so); by default the in-tree release build is loaded.
+LIB_PATH = os.environ.get("ATTN_SINK_LIBRARY") or os.path.join(_HERE, "libattn_sink.so")
 
 ATTN_SINK_BF16, ATTN_SINK_FP32, ATTN_SINK_FP16 = 0, 1, 2
 STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE", 4: "ERR_CUDA",

@@ -2,10 +2,16 @@
 
     python -m softmax_attn_sink_b200.build          # incremental
     python -m softmax_attn_sink_b200.build --force  # rebuild everything
+    python -m softmax_attn_sink_b200.build --debug  # the bounds-checking debug library
 
 Each ``csrc/*.cu`` compiles to an object under ``_build/`` (in parallel), then nvcc
 links them into ``softmax_attn_sink_b200/libattn_sink.so`` with the CUDA runtime
 linked statically, so the library needs nothing but the driver at run time.
+
+``--debug`` builds the same sources with ``-DATTN_SINK_DEBUG`` into ``_build_debug/`` and
+``libattn_sink_debug.so``: every global store of an output checks its index range against
+the tensor it writes, skips a store that would leave it and sets bit 8 of the device status
+word.  Load it instead of the release library by setting ``ATTN_SINK_LIBRARY`` to its path.
 """
 from __future__ import annotations
 
@@ -22,6 +28,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libattn_sink.so")
+OBJ_DEBUG = os.path.join(HERE, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libattn_sink_debug.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -56,11 +64,16 @@ def _compile(src: str, obj: str, extra) -> str:
     return r.stderr
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile every CUDA source for sm_100a and link the shared library; returns its path."""
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = False) -> str:
+    """Compile every CUDA source for sm_100a and link the shared library; returns its path.
+
+    debug=True builds the bounds-checking library (``-DATTN_SINK_DEBUG``) beside the release one."""
+    obj_dir, lib = (OBJ_DEBUG, LIB_DEBUG) if debug else (OBJ, LIB)
+    if debug:
+        extra = list(extra) + ["-DATTN_SINK_DEBUG"]
+    os.makedirs(obj_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    objs = [os.path.join(OBJ, os.path.basename(s)[:-3] + ".o") for s in srcs]
+    objs = [os.path.join(obj_dir, os.path.basename(s)[:-3] + ".o") for s in srcs]
     todo = [(s, o) for s, o in zip(srcs, objs) if force or _stale(o, s)]
     if todo:
         with cf.ThreadPoolExecutor(max_workers=min(8, len(todo))) as ex:
@@ -69,21 +82,22 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
                 msg = f.result()
                 if verbose and msg.strip():
                     print(f"[{os.path.basename(futs[f])}]\n{msg}", file=sys.stderr)
-    if todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
+    if todo or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", lib] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{' '.join(cmd)}\n{r.stdout}{r.stderr}")
-    return LIB
+    return lib
 
 
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", "-v", action="store_true", help="print ptxas resource usage")
+    ap.add_argument("--debug", action="store_true", help="build the bounds-checking debug library")
     args = ap.parse_args()
     extra = ["-Xptxas", "-v"] if args.verbose else []
-    print(build(force=args.force or args.verbose, verbose=args.verbose, extra=extra))
+    print(build(force=args.force or args.verbose, verbose=args.verbose, extra=extra, debug=args.debug))
 
 
 if __name__ == "__main__":

@@ -13,7 +13,8 @@ using namespace attn_sink;
 namespace {
 
 // Bits set by kernels: a bounded wait ran out (kStatusTimeout), an index or length outside
-// its table was skipped (kStatusBadIndex).
+// its table was skipped (kStatusBadIndex), cu_seqlens broke their contract
+// (kStatusBadSeqlens), a debug build skipped a store outside its output (kStatusDebugBounds).
 __device__ unsigned int g_status_word;
 
 constexpr int kMaxDevices = 64;

@@ -324,7 +324,9 @@ bwd_dq_d256_kernel(const BwdArgs a, int mtiles, int band, const __grid_constant_
     tc_fence_after();
     if (ok)
       store_row<T>(tmem + lane_off + kColDQ, have, a.scale,
-                   static_cast<T*>(a.grad_q) + ((long long)(q0 + i) * a.hq + h) * D, row_ok);
+                   static_cast<T*>(a.grad_q) + ((long long)(q0 + i) * a.hq + h) * D,
+                   row_ok && store_ok(((long long)(q0 + i) * a.hq + h) * D, ((long long)(q0 + i) * a.hq + h) * D + D - 1,
+                                      (long long)a.total_q * a.hq * D, a.status));
   }
   tc_fence_before();
   __syncthreads();
@@ -577,7 +579,10 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
     tc_fence_after();
     if (ok)
       store_row<T>(tmem + lane_off + kColDV, have, DROP ? a.drop.scale : 1.f,
-                   static_cast<T*>(a.grad_v) + ((long long)(tl.k0 + j) * a.hkv + tl.g) * D, key_ok);
+                   static_cast<T*>(a.grad_v) + ((long long)(tl.k0 + j) * a.hkv + tl.g) * D,
+                   key_ok && store_ok(((long long)(tl.k0 + j) * a.hkv + tl.g) * D,
+                                      ((long long)(tl.k0 + j) * a.hkv + tl.g) * D + D - 1,
+                                      (long long)a.total_k * a.hkv * D, a.status));
   }
   tc_fence_before();
   __syncthreads();
@@ -799,7 +804,10 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
     tc_fence_after();
     if (ok)
       store_row<T>(tmem + lane_off + kColDK, have, a.scale,
-                   static_cast<T*>(a.grad_k) + ((long long)(tl.k0 + j) * a.hkv + tl.g) * D, key_ok);
+                   static_cast<T*>(a.grad_k) + ((long long)(tl.k0 + j) * a.hkv + tl.g) * D,
+                   key_ok && store_ok(((long long)(tl.k0 + j) * a.hkv + tl.g) * D,
+                                      ((long long)(tl.k0 + j) * a.hkv + tl.g) * D + D - 1,
+                                      (long long)a.total_k * a.hkv * D, a.status));
   }
   tc_fence_before();
   __syncthreads();

@@ -376,7 +376,8 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         const float x1 = (n > 0 && have) ? __uint_as_float(v[2 * e + 1]) * a.scale : 0.f;
         pk[e] = pack2<Elem>(x0, x1);
       }
-      if (row_ok) {
+      const long long e0 = ((q0 + i) * a.hq + h) * DK + c * 32;
+      if (row_ok && store_ok(e0, e0 + 31, (long long)a.total_q * a.hq * DK, a.status)) {
         uint4* dst = reinterpret_cast<uint4*>(dqp) + c * 4;
 #pragma unroll
         for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);

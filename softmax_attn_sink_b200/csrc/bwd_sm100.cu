@@ -382,7 +382,8 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
           const float x1 = (T > 0 && have) ? __uint_as_float(v[2 * e + 1]) * mul : 0.f;
           pk[e] = pack2<Elem>(x0, x1);
         }
-        if (key_ok) {
+        const long long e0 = ((k0 + j) * a.hkv + g) * ncol + c * 32;
+        if (key_ok && store_ok(e0, e0 + 31, (long long)a.total_k * a.hkv * ncol, a.status)) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) dst[c * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
@@ -442,8 +443,9 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
       __syncwarp();
       if (lane == 0) mbar_arrive(bar.dq_free());
       const long long qi = qbase_of(t) + r;
-      if (qi < sq) {
-        float* dst = a.dq_acc + ((q0 + qi) * a.hq + head_of(t)) * DK;
+      const long long a0 = ((q0 + qi) * a.hq + head_of(t)) * DK;
+      if (qi < sq && store_ok(a0, a0 + DK - 1, (long long)a.total_q * a.hq * DK, a.status)) {
+        float* dst = a.dq_acc + a0;
 #pragma unroll
         for (int e = 0; e < DK; e += 4)
           red_add_v4(dst + e, __uint_as_float(v[e]) * a.scale, __uint_as_float(v[e + 1]) * a.scale,
@@ -869,7 +871,8 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
           const float x1 = (T > 0 && have) ? __uint_as_float(v[2 * e + 1]) * mul : 0.f;
           pk[e] = pack2<Elem>(x0, x1);
         }
-        if (key_ok) {
+        const long long e0 = ((k0 + j) * a.hkv + g) * ncol + c * 32;
+        if (key_ok && store_ok(e0, e0 + 31, (long long)a.total_k * a.hkv * ncol, a.status)) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) dst[c * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
@@ -901,6 +904,9 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         const long long left = sq - qa;
         const int nval = left < 64 ? (int)left : 64;
         float* dst = a.dq_acc + ((long long)h * a.total_q + q0 + qa) * DK + d;
+        const long long a0 = ((long long)h * a.total_q + q0 + qa) * DK + d;
+        if (nval > 0 && !store_ok(a0, a0 + (long long)(nval - 1) * DK, (long long)a.hq * a.total_q * DK, a.status))
+          continue;
 #pragma unroll
         for (int e = 0; e < 64; ++e)
           if (e < nval) atomicAdd(dst + e * DK, __uint_as_float(v[e]) * a.scale);

@@ -201,4 +201,19 @@ __device__ __forceinline__ void set_status(unsigned* status, unsigned bit) {
   if (status) atomicOr(status, bit);
 }
 
+// Debug builds (compiled with -DATTN_SINK_DEBUG) check the element range [first, last] of a
+// global store against its tensor's element count n: a range outside it sets
+// kStatusDebugBounds in the device status word and the store is skipped.  This stands in
+// for a memory checker on machines where none can run.  Release builds compile it away.
+__device__ __forceinline__ bool store_ok(long long first, long long last, long long n, unsigned* status) {
+#ifdef ATTN_SINK_DEBUG
+  if (first >= 0 && first <= last && last < n) return true;
+  set_status(status, kStatusDebugBounds);
+  return false;
+#else
+  (void)first; (void)last; (void)n; (void)status;
+  return true;
+#endif
+}
+
 }  // namespace attn_sink

@@ -430,6 +430,8 @@ __global__ void __launch_bounds__(warps_of<DK, DV>() * 32, ctas_per_sm<DK, DV>()
       }
     }
     const long long pidx = ((long long)b * a.hq + h_base + row) * a.splits + c;
+    const long long nrows = (long long)a.batch * a.hq * a.splits;
+    if (!store_ok(pidx, pidx, nrows, a.status)) continue;
     a.part_o[pidx * DV + col] = o;
     if (col == 0) {
       a.part_ml[pidx * 2 + 0] = m;
@@ -476,6 +478,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, i
   const float den = lm + ((sink2 == kNegInf || m == kNegInf) ? 0.f : ex2(sink2 - m));
   const float inv = den > 0.f ? 1.f / den : 0.f;
   T* out = static_cast<T*>(a.out);
+  if (!store_ok(row * DV, row * DV + DV - 1, (long long)a.batch * a.hq * DV, a.status)) return;
 #pragma unroll
   for (int j = 0; j < VPL; ++j) out[row * DV + lane + 32 * j] = from_float<T>(o[j] * inv);
   if (a.lse && lane == 0)

@@ -363,12 +363,14 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack2<T>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        if (row_ok) {
+        const long long ob = ((long long)(q0 + i) * a.hq + h) * D + c * 32;
+        if (row_ok && store_ok(ob, ob + 31, (long long)a.total_q * a.hq * D, a.status)) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) orow[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (row_ok && a.lse)
+      // lse is [Hq, total_q]: the row itself must lie inside total_q
+      if (row_ok && a.lse && store_ok((long long)q0 + i, (long long)q0 + i, a.total_q, a.status))
         a.lse[(long long)h * a.total_q + q0 + i] = l > 0.f ? (m + __log2f(l)) * kLn2 : kNegInf;
     }
   }

@@ -641,12 +641,14 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
           for (int k = 0; k < 8; ++k) {
             const int rr = 4 * k + (lane >> 3), ch = lane & 7;
             const uint4 w = ld_shared_v4(stg + rr * 128 + ((ch ^ (rr & 7)) << 4));
-            if (rr < e_nrow)
-              *reinterpret_cast<uint4*>(out + ((e_grow - lane + rr) * a.hq + e_h) * DVO + (cc >> 1) * 64 + ch * 8) = w;
+            const long long o0 = ((e_grow - lane + rr) * a.hq + e_h) * DVO + (cc >> 1) * 64 + ch * 8;
+            if (rr < e_nrow && store_ok(o0, o0 + 7, (long long)a.total_q * a.hq * DVO, a.status))
+              *reinterpret_cast<uint4*>(out + o0) = w;
           }
           __syncwarp();
         }
-      } else if (e_row) {
+      } else if (e_row && store_ok((e_grow * a.hq + e_h) * DVO + cc * 32, (e_grow * a.hq + e_h) * DVO + cc * 32 + 31,
+                                   (long long)a.total_q * a.hq * DVO, a.status)) {
         uint4* orow = reinterpret_cast<uint4*>(out + (e_grow * a.hq + e_h) * DVO);
 #pragma unroll
         for (int v = 0; v < 4; ++v)
@@ -654,7 +656,9 @@ fwd_sm100_kernel(const FwdArgs a, const Sched sc, const __grid_constant__ CUtens
       }
     };
     auto emit_lse = [&]() {
-      if (e_row && a.lse) a.lse[(long long)e_h * a.total_q + e_grow] = e_lse;
+      // lse is [Hq, total_q]: the row itself must lie inside total_q
+      if (e_row && a.lse && store_ok(e_grow, e_grow, a.total_q, a.status))
+        a.lse[(long long)e_h * a.total_q + e_grow] = e_lse;
     };
     // The pending epilogue, when the next item does not take its deferred path: wait for the
     // unit's last PV (pv_done is committed once per item, after the unit's last PV), then

@@ -15,6 +15,7 @@ constexpr int kUnbounded = 1 << 30;
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBadIndex = 2u;  // a paged block id or key count outside its table
 constexpr unsigned kStatusBadSeqlens = 4u;  // cu_seqlens broke its contract (attn_sink_check_seqlens)
+constexpr unsigned kStatusDebugBounds = 8u;  // debug builds: a store outside its tensor was skipped
 
 // Dropout keep decisions: key j of packed query row r and q head h is kept when byte j % 16
 // of Philox4x32-10(counter = (j / 16, r, h, offset), key = (seed_lo, seed_hi)) is below the

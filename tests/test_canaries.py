@@ -4,8 +4,9 @@ elements.  Each output here is a view into a larger device buffer filled with 0x
 whose leading and trailing 4 KB are guards; after the call both guards must be intact, and
 no element of the output may still be all ones (every element must be written, including
 the zeros of rows or keys that see nothing).  All-ones is a NaN in bf16, fp16 and fp32,
-which no correct output is.  Values are compared with the
-oracle as well.
+which no correct output is.  Values are compared with the oracle as well, and the device
+status word must stay clear.  test_debug_build.py runs this file again against the
+bounds-checking debug library.
 
 The cu_seqlens contract is the caller's (CANN flash_attn doc, "SeqLengths Parameter
 Group"); with valid cu_seqlens every kernel must stay inside its outputs.  The cases span
@@ -13,6 +14,8 @@ varlen GQA with empty sequences and sq != sk, the persistent forward with and wi
 its output staging area, the one-CTA-per-item grid forward, head dims 64 / 128 / 256 and
 dv 32, fp16 and fp32, dropout, the atomic, deterministic and dropout backward, and the
 packed and paged decode."""
+import os
+
 import numpy as np
 import pytest
 
@@ -73,6 +76,26 @@ FWD_CASES = [
 ]
 
 
+def _status_clear():
+    """No kernel set a status bit (in the debug library: no store left its output)."""
+    assert sab.device_status() == (0, 0)
+
+
+@pytest.fixture(autouse=True)
+def _fresh_status():
+    sab.device_status()   # read and clear whatever an earlier test left
+    yield
+
+
+def test_library_in_use():
+    """Run with ATTN_SINK_EXPECT_LIBRARY set (the debug-library run), the package must have
+    loaded that file."""
+    want = os.environ.get("ATTN_SINK_EXPECT_LIBRARY")
+    sab.lib()
+    if want:
+        assert os.path.samefile(sab.LIB_PATH, want)
+
+
 def _fwd_guarded(p, dropout):
     td = tdtype(p)
     q, k, v = dev(p.q, td), dev(p.k, td), dev(p.v, td)
@@ -93,6 +116,7 @@ def test_fwd_stays_inside_its_outputs(case):
     _, go, gl = _fwd_guarded(p, drop)
     go.check()
     gl.check()
+    _status_clear()
     ro, rl = ref.fwd(p.q, p.k, p.v, p.cu_seqlens_q, p.cu_seqlens_k, p.sink, p.softmax_scale,
                      p.causal, wl, wr, dropout=drop)
     check_out(to_np(go.t), ro, dtype)
@@ -133,6 +157,7 @@ def test_bwd_stays_inside_its_outputs(case):
                       dk=gk.t, dv=gv.t, dsink=gs.t, deterministic=mode == "deterministic", dropout=drop)
     for g in (gq, gk, gv, gs):
         g.check()
+    _status_clear()
     a = (p.cu_seqlens_q, p.cu_seqlens_k, p.sink, p.softmax_scale, p.causal, wl, wr)
     rdq, rdk, rdv, rds = ref.bwd(p.q, p.k, p.v, p.dout, *a, dropout=drop)
     check_grad(to_np(gq.t), rdq, dtype, "dq")
@@ -153,6 +178,7 @@ def test_decode_stays_inside_its_outputs(dim, splits):
                          out=go.t, lse=gl.t)
     go.check()
     gl.check()
+    _status_clear()
     ro, rl = ref.decode(d.q, d.k, d.v, d.cu_seqlens_k, d.sink, d.softmax_scale)
     check_out(to_np(go.t), ro, "bf16")
     check_lse(to_np(gl.t), rl, "bf16")
@@ -172,6 +198,7 @@ def test_paged_decode_stays_inside_its_outputs():
                                dev(d.sink), d.softmax_scale, out=go.t, lse=gl.t)
     go.check()
     gl.check()
+    _status_clear()
     ro, rl = ref.decode_paged(d.q, kc, vc, table, used, 64, d.sink, d.softmax_scale)
     check_out(to_np(go.t), ro, "bf16")
     check_lse(to_np(gl.t), rl, "bf16")
