@@ -211,40 +211,41 @@ bwd_dq_d256_kernel(const BwdArgs a, int mtiles, int band, const __grid_constant_
         mbar_wait(bar.kv_full(p % kStages), (p / kStages) & 1, a.status);
     }
   } else if (warp == 1) {
-    if (lane == 0 && n > 0) {
+    // The whole warp runs the issue loop in step; elect.sync picks the issuing lane.
+    if (n > 0) {
       constexpr uint32_t id_s = idesc_of<T>(kBM, kBN, 0, 0);   // S, dP: K-major B
       constexpr uint32_t id_q = idesc_of<T>(kBM, D, 0, 1);     // dS (TMEM) x K (N-major)
       const uint64_t kO = smem_desc(sO, 16, 1024, kLayoutSwizzle128B);
       const uint64_t kK = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
       const uint64_t mK = smem_desc(sK, kBox64, 1024, kLayoutSwizzle128B);
       const uint64_t kV = smem_desc(sV, 16, 1024, kLayoutSwizzle128B);
-      bool ok = mbar_wait(bar.q_full(), 0, a.status) && mbar_wait(bar.o_full(), 0, a.status);
+      bool ok = mbar_wait_warp(bar.q_full(), 0, a.status) && mbar_wait_warp(bar.o_full(), 0, a.status);
       for (int j = 0; j < n && ok; ++j) {
         const int st = j % kStages;
-        if (!(ok = mbar_wait(bar.kv_full(st), (j / kStages) & 1, a.status))) break;
+        if (!(ok = mbar_wait_warp(bar.kv_full(st), (j / kStages) & 1, a.status))) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((st * kTile64) >> 4);
         // S = Q K^T (A = Q from TMEM); dS(j - 1) in S's columns was read by dQ(j - 1), issued
         // earlier by this thread
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_ts(tmem + kColS, tmem + kColQ + ks * 8, kK + so + kmaj_off(ks, kBox64), id_s, ks > 0 ? 1u : 0u);
+          mma_ts_elect(tmem + kColS, tmem + kColQ + ks * 8, kK + so + kmaj_off(ks, kBox64), id_s, ks > 0 ? 1u : 0u);
         // dP = dout V^T
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_ss(tmem + kColP, kO + kmaj_off(ks, kBox128), kV + so + kmaj_off(ks, kBox64), id_s, ks > 0 ? 1u : 0u);
-        mma_commit(bar.sdp_full());
-        if (!(ok = mbar_wait(bar.ds_full(), j & 1, a.status))) break;
+          mma_ss_elect(tmem + kColP, kO + kmaj_off(ks, kBox128), kV + so + kmaj_off(ks, kBox64), id_s, ks > 0 ? 1u : 0u);
+        mma_commit_elect(bar.sdp_full());
+        if (!(ok = mbar_wait_warp(bar.ds_full(), j & 1, a.status))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + kColDQ, tmem + kColS + kk * 8, mK + so + (uint64_t)((kk * 2048) >> 4), id_q,
+          mma_ts_elect(tmem + kColDQ, tmem + kColS + kk * 8, mK + so + (uint64_t)((kk * 2048) >> 4), id_q,
                  (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar.kv_empty(st));
+        mma_commit_elect(bar.kv_empty(st));
       }
-      if (ok) mma_commit(bar.dq_done());
-      mma_commit(bar.drain());
-      mbar_wait(bar.drain(), 0, a.status);
+      if (ok) mma_commit_elect(bar.dq_done());
+      mma_commit_elect(bar.drain());
+      mbar_wait_warp(bar.drain(), 0, a.status);
     }
   } else if (warp >= 4) {
     const int lg = warp & 3;
@@ -471,41 +472,42 @@ bwd_dv_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
         mbar_wait(bar.qd_full(p % kStages), (p / kStages) & 1, a.status);
     }
   } else if (warp == 1) {
-    if (lane == 0 && T_ > 0) {
+    // The whole warp runs the issue loop in step; elect.sync picks the issuing lane.
+    if (T_ > 0) {
       constexpr uint32_t id_s = idesc_of<T>(ks::kBN, kBM, 0, 0);   // K (TMEM) x Q (K-major)
       constexpr uint32_t id_v = idesc_of<T>(ks::kBN, D, 0, 1);     // P^T (TMEM) x dout (N-major)
       const uint64_t kQ = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
       const uint64_t mO = smem_desc(sO, kBox64, 1024, kLayoutSwizzle128B);
       auto issue_s = [&](int t) -> bool {
         const int st = t % kStages;
-        if (!mbar_wait(bar.qd_full(st), (t / kStages) & 1, a.status)) return false;
+        if (!mbar_wait_warp(bar.qd_full(st), (t / kStages) & 1, a.status)) return false;
         tc_fence_after();
         const uint64_t so = (uint64_t)((st * kTile64) >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ts(tmem + col_S(t & 1), tmem + kColK + k * 8, kQ + so + kmaj_off(k, kBox64), id_s, k > 0 ? 1u : 0u);
-        mma_commit(bar.s_full(t & 1));
+          mma_ts_elect(tmem + col_S(t & 1), tmem + kColK + k * 8, kQ + so + kmaj_off(k, kBox64), id_s, k > 0 ? 1u : 0u);
+        mma_commit_elect(bar.s_full(t & 1));
         return true;
       };
-      bool ok = mbar_wait(bar.k_full(), 0, a.status);
+      bool ok = mbar_wait_warp(bar.k_full(), 0, a.status);
       tc_fence_after();
       if (ok) ok = issue_s(0);
       if (ok && T_ > 1) ok = issue_s(1);
       for (int t = 0; t < T_ && ok; ++t) {
         const int st = t % kStages;
-        if (!(ok = mbar_wait(bar.p_full(t & 1), (t >> 1) & 1, a.status))) break;
+        if (!(ok = mbar_wait_warp(bar.p_full(t & 1), (t >> 1) & 1, a.status))) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((st * kTile64) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ts(tmem + kColDV, tmem + col_S(t & 1) + kk * 8, mO + so + (uint64_t)((kk * 2048) >> 4), id_v,
+          mma_ts_elect(tmem + kColDV, tmem + col_S(t & 1) + kk * 8, mO + so + (uint64_t)((kk * 2048) >> 4), id_v,
                  (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar.qd_empty(st));
+        mma_commit_elect(bar.qd_empty(st));
         if (t + 2 < T_) ok = issue_s(t + 2);
       }
-      if (ok) mma_commit(bar.dv_done());
-      mma_commit(bar.drain());
-      mbar_wait(bar.drain(), 0, a.status);
+      if (ok) mma_commit_elect(bar.dv_done());
+      mma_commit_elect(bar.drain());
+      mbar_wait_warp(bar.drain(), 0, a.status);
     }
   } else if (DROP && warp < 4) {
     // warps 2-3: the dropout flags of every tile, a tile ahead of the compute warps
@@ -687,39 +689,40 @@ bwd_dk_d256_kernel(const BwdArgs a, int ntiles, int band, const __grid_constant_
         mbar_wait(bar.qd_full(p % kStages), (p / kStages) & 1, a.status);
     }
   } else if (warp == 1) {
-    if (lane == 0 && T_ > 0) {
+    // The whole warp runs the issue loop in step; elect.sync picks the issuing lane.
+    if (T_ > 0) {
       constexpr uint32_t id_s = idesc_of<T>(ks::kBN, kBM, 0, 0);   // S^T, dP^T: K-major B
       constexpr uint32_t id_k = idesc_of<T>(ks::kBN, D, 0, 1);     // dS^T (TMEM) x Q (N-major)
       const uint64_t kV = smem_desc(sV, 16, 1024, kLayoutSwizzle128B);
       const uint64_t kQ = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
       const uint64_t mQ = smem_desc(sQ, kBox64, 1024, kLayoutSwizzle128B);
       const uint64_t kO = smem_desc(sO, 16, 1024, kLayoutSwizzle128B);
-      bool ok = mbar_wait(bar.k_full(), 0, a.status) && mbar_wait(bar.v_full(), 0, a.status);
+      bool ok = mbar_wait_warp(bar.k_full(), 0, a.status) && mbar_wait_warp(bar.v_full(), 0, a.status);
       for (int t = 0; t < T_ && ok; ++t) {
         const int st = t % kStages;
-        if (!(ok = mbar_wait(bar.qd_full(st), (t / kStages) & 1, a.status))) break;
+        if (!(ok = mbar_wait_warp(bar.qd_full(st), (t / kStages) & 1, a.status))) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((st * kTile64) >> 4);
         // S^T = K Q^T (A = K from TMEM); dS^T(t - 1) in S^T's columns was read by dK(t - 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ts(tmem + kColS, tmem + kColK + k * 8, kQ + so + kmaj_off(k, kBox64), id_s, k > 0 ? 1u : 0u);
+          mma_ts_elect(tmem + kColS, tmem + kColK + k * 8, kQ + so + kmaj_off(k, kBox64), id_s, k > 0 ? 1u : 0u);
         // dP^T = V dout^T
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + kColP, kV + kmaj_off(k, kBox128), kO + so + kmaj_off(k, kBox64), id_s, k > 0 ? 1u : 0u);
-        mma_commit(bar.sdp_full());
-        if (!(ok = mbar_wait(bar.ds_full(), t & 1, a.status))) break;
+          mma_ss_elect(tmem + kColP, kV + kmaj_off(k, kBox128), kO + so + kmaj_off(k, kBox64), id_s, k > 0 ? 1u : 0u);
+        mma_commit_elect(bar.sdp_full());
+        if (!(ok = mbar_wait_warp(bar.ds_full(), t & 1, a.status))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ts(tmem + kColDK, tmem + kColS + kk * 8, mQ + so + (uint64_t)((kk * 2048) >> 4), id_k,
+          mma_ts_elect(tmem + kColDK, tmem + kColS + kk * 8, mQ + so + (uint64_t)((kk * 2048) >> 4), id_k,
                  (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar.qd_empty(st));
+        mma_commit_elect(bar.qd_empty(st));
       }
-      if (ok) mma_commit(bar.dk_done());
-      mma_commit(bar.drain());
-      mbar_wait(bar.drain(), 0, a.status);
+      if (ok) mma_commit_elect(bar.dk_done());
+      mma_commit_elect(bar.drain());
+      mbar_wait_warp(bar.drain(), 0, a.status);
     }
   } else if (DROP && warp < 4) {
     // warps 2-3: the dropout flags of every tile, a tile ahead of the compute warps

@@ -206,7 +206,8 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
     if constexpr (DROP) regs_dec<kRegsLowD>();
-    if (lane == 0 && n > 0) {
+    // The whole warp runs the issue loop in step; elect.sync picks the issuing lane.
+    if (n > 0) {
       constexpr uint32_t id_s = idesc_of<Elem>(kBM, kBN, 0, 0);   // S, dP: K-major A and B
       constexpr uint32_t id_q = idesc_of<Elem>(kBM, DK, 0, 1);    // dS (TMEM) x K (MN-major)
       // Shared-memory descriptors, built once; offsets add to the start field.  "k" = K-major
@@ -220,37 +221,37 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       // issued earlier by this thread
       auto issue_s = [&](int j) -> bool {
         const int sk_ = j % L::KS;
-        if (!mbar_wait(bar.k_full(sk_), (j / L::KS) & 1, a.status)) return false;
+        if (!mbar_wait_warp(bar.k_full(sk_), (j / L::KS) & 1, a.status)) return false;
         tc_fence_after();
         const uint64_t koff = (uint64_t)((sk_ * L::kKBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + col_S(j & 1), kQ + off16, kK + koff + off16, id_s, ks > 0);
+          mma_ss_elect(tmem + col_S(j & 1), kQ + off16, kK + koff + off16, id_s, ks > 0);
         }
         return true;
       };
       // dP(j) = dout V_j^T; then V_j's stage is free and tile j's S and dP are announced
       auto issue_p = [&](int j) -> bool {
         const int sv_ = j & 1;
-        if (!mbar_wait(bar.v_full(sv_), (j >> 1) & 1, a.status)) return false;
+        if (!mbar_wait_warp(bar.v_full(sv_), (j >> 1) & 1, a.status)) return false;
         tc_fence_after();
         const uint64_t voff = (uint64_t)((sv_ * L::kVBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < DV / 16; ++ks) {
           const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + kColP, kO + off16, kV + voff + off16, id_s, ks > 0);
+          mma_ss_elect(tmem + kColP, kO + off16, kV + voff + off16, id_s, ks > 0);
         }
-        mma_commit(bar.v_empty(sv_));
-        mma_commit(bar.sdp_full());
+        mma_commit_elect(bar.v_empty(sv_));
+        mma_commit_elect(bar.sdp_full());
         return true;
       };
-      bool ok = mbar_wait(bar.qd_full(), 0, a.status);
+      bool ok = mbar_wait_warp(bar.qd_full(), 0, a.status);
       if (ok) ok = issue_s(0) && issue_p(0);
       for (int j = 0; j < n && ok; ++j) {
         if (j + 1 < n && !(ok = issue_s(j + 1))) break;   // overlaps the compute warps' tile j
         // the compute warps have written dS(j) and are done reading dP(j)
-        if (!(ok = mbar_wait(bar.ds_full(), j & 1, a.status))) break;
+        if (!(ok = mbar_wait_warp(bar.ds_full(), j & 1, a.status))) break;
         tc_fence_after();
         if (j + 1 < n && !(ok = issue_p(j + 1))) break;
         // dQ += dS(j) K_j, then K_j's stage is free
@@ -258,14 +259,14 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
         const uint64_t koff = (uint64_t)((sk_ * L::kKBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + kColQ, tmem + col_S(j & 1) + kk * 8, mK + koff + (uint64_t)((kk * 2048) >> 4), id_q,
+          mma_ts_elect(tmem + kColQ, tmem + col_S(j & 1) + kk * 8, mK + koff + (uint64_t)((kk * 2048) >> 4), id_q,
                  (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar.k_empty(sk_));
+        mma_commit_elect(bar.k_empty(sk_));
       }
-      if (ok) mma_commit(bar.dq_done());
+      if (ok) mma_commit_elect(bar.dq_done());
       // every MMA must be complete before the TMEM is freed
-      mma_commit(bar.drain());
-      mbar_wait(bar.drain(), 0, a.status);
+      mma_commit_elect(bar.drain());
+      mbar_wait_warp(bar.drain(), 0, a.status);
     }
   } else if (warp < 4) {
     if constexpr (DROP) regs_dec<kRegsLowD>();   // warps 2-3: no role, but part of the first warpgroup

@@ -210,57 +210,59 @@ bwd_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q, cons
     }
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
-    if (lane == 0 && T > 0) {
+    // The whole warp runs the issue loop in step and elect.sync picks the issuing lane
+    // (an MMA costs the warp 5-10 cycles this way, against about 50 from a lone lane).
+    if (T > 0) {
       constexpr uint32_t id_s = idesc_of<Elem>(kBN, kBM, 0, 0);   // S^T, dP^T: K-major A and B
       constexpr uint32_t id_dv = idesc_of<Elem>(kBN, DV, 0, 1);   // A from TMEM, B = dout MN-major
       constexpr uint32_t id_dk = idesc_of<Elem>(kBN, DK, 0, 1);   // A = dS^T K-major, B = Q MN-major
       constexpr uint32_t id_dq = idesc_of<Elem>(kBM, DK, 1, 1);   // A = dS MN-major, B = K MN-major
-      bool ok = mbar_wait(bar.kv_full(), 0, a.status);
+      bool ok = mbar_wait_warp(bar.kv_full(), 0, a.status);
       for (int t = 0; t < T && ok; ++t) {
         const int st = t & 1;
         const uint32_t q_s = sQ + st * L::kQBytes, o_s = sO + st * L::kOBytes;
-        ok = mbar_wait(bar.qd_full(st), (t >> 1) & 1, a.status);
-        if (ok && t >= 1) ok = mbar_wait(bar.dv_done(), (t - 1) & 1, a.status);   // R0 free
+        ok = mbar_wait_warp(bar.qd_full(st), (t >> 1) & 1, a.status);
+        if (ok && t >= 1) ok = mbar_wait_warp(bar.dv_done(), (t - 1) & 1, a.status);   // R0 free
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
-          mma_ss(tmem + kColR0, smem_desc(sK + off, 16, 1024, kLayoutSwizzle128B),
+          mma_ss_elect(tmem + kColR0, smem_desc(sK + off, 16, 1024, kLayoutSwizzle128B),
                  smem_desc(q_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
         }
-        if (DQ && t >= 1 && !(ok = mbar_wait(bar.dq_free(), (t - 1) & 1, a.status))) break;   // R1 free
+        if (DQ && t >= 1 && !(ok = mbar_wait_warp(bar.dq_free(), (t - 1) & 1, a.status))) break;   // R1 free
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DV / 16; ++ks) {
           const uint32_t off = (ks >> 2) * L::kHalf + (ks & 3) * 32;
-          mma_ss(tmem + kColR1, smem_desc(sV + off, 16, 1024, kLayoutSwizzle128B),
+          mma_ss_elect(tmem + kColR1, smem_desc(sV + off, 16, 1024, kLayoutSwizzle128B),
                  smem_desc(o_s + off, 16, 1024, kLayoutSwizzle128B), id_s, ks > 0);
         }
-        mma_commit(bar.sdp_full());
-        if (!(ok = mbar_wait(bar.compute_done(), t & 1, a.status))) break;
+        mma_commit_elect(bar.sdp_full());
+        if (!(ok = mbar_wait_warp(bar.compute_done(), t & 1, a.status))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ts(tmem + kColDV, tmem + kColR0 + kk * 8,
+          mma_ts_elect(tmem + kColDV, tmem + kColR0 + kk * 8,
                  smem_desc(o_s + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dv, (t > 0 || kk > 0));
-        mma_commit(bar.dv_done());
+        mma_commit_elect(bar.dv_done());
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ss(tmem + kColDK, smem_desc(sDS + (kk >> 2) * L::kHalf + (kk & 3) * 32, 16, 1024, kLayoutSwizzle128B),
+          mma_ss_elect(tmem + kColDK, smem_desc(sDS + (kk >> 2) * L::kHalf + (kk & 3) * 32, 16, 1024, kLayoutSwizzle128B),
                  smem_desc(q_s + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dk, (t > 0 || kk > 0));
         if (DQ) {
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ss(tmem + kColR1, smem_desc(sDS + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B),
+            mma_ss_elect(tmem + kColR1, smem_desc(sDS + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B),
                    smem_desc(sK + kk * 2048, L::kHalf, 1024, kLayoutSwizzle128B), id_dq, kk > 0);
-          mma_commit(bar.dq_full());
+          mma_commit_elect(bar.dq_full());
         }
-        mma_commit(bar.ds_free());
-        mma_commit(bar.qd_empty(st));
+        mma_commit_elect(bar.ds_free());
+        mma_commit_elect(bar.qd_empty(st));
       }
-      mma_commit(bar.drain());
-      mbar_wait(bar.drain(), 0, a.status);
+      mma_commit_elect(bar.drain());
+      mbar_wait_warp(bar.drain(), 0, a.status);
     }
   } else if (warp < 6) {
     // ================================ compute warps (thread = key row) ===================
@@ -609,7 +611,27 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
     regs_dec<kRegsLow>();
-    if (lane == 0 && T > 0) {
+    // Without the dQ part the whole warp runs the issue loop in step and elect.sync picks the
+    // issuing lane (an MMA costs the warp 5-10 cycles this way, against about 50 from a lone
+    // lane): +1.5-3% on the deterministic and dropout backward.  With dQ (the atomic
+    // backward) that measured 0.5-1% slower, so there one lane issues.
+    constexpr bool kElect = !DQ;
+    if ((kElect || lane == 0) && T > 0) {
+      auto wait_ = [&](uint32_t b, uint32_t par) -> bool {
+        return kElect ? mbar_wait_warp(b, par, a.status) : mbar_wait(b, par, a.status);
+      };
+      auto mma_ss_ = [&](uint32_t d, uint32_t al, uint32_t bl, uint32_t hi, uint32_t id, uint32_t acc) {
+        if constexpr (kElect) mma_ss_lo_elect(d, al, bl, hi, id, acc);
+        else mma_ss_lo(d, al, bl, hi, id, acc);
+      };
+      auto mma_ts_ = [&](uint32_t d, uint32_t at, uint32_t bl, uint32_t hi, uint32_t id, uint32_t acc) {
+        if constexpr (kElect) mma_ts_lo_elect(d, at, bl, hi, id, acc);
+        else mma_ts_lo(d, at, bl, hi, id, acc);
+      };
+      auto commit_ = [&](uint32_t b) {
+        if constexpr (kElect) mma_commit_elect(b);
+        else mma_commit(b);
+      };
       constexpr uint32_t id_s = idesc_of<Elem>(kBN, 64, 0, 0);    // S_h, dP_h: 128 keys x 64 queries
       constexpr uint32_t id_dv = idesc_of<Elem>(kBN, DV, 0, 1);   // P^T_h (TMEM) x dout_h (MN-major)
       constexpr uint32_t id_dk = idesc_of<Elem>(kBN, DK, 0, 1);   // dS^T_h (K-major) x Q_h (MN-major)
@@ -618,75 +640,79 @@ bwd_sm100_d128_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
       // Shared-memory descriptors, built once: an address offset is an addition to the start
       // field (addresses stay below 2^18 bytes, so the 14-bit field never carries).  "k" =
       // K-major view (LBO unused), "m" = MN-major view (LBO = the 16 KB between 64-column halves).
-      const uint64_t kK = smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
-      const uint64_t mK = smem_desc(sK, L::kHalf, 1024, kLayoutSwizzle128B);
-      const uint64_t kV = smem_desc(sV, 16, 1024, kLayoutSwizzle128B);
-      const uint64_t kQ = smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
-      const uint64_t mQ = smem_desc(sQ, L::kHalf, 1024, kLayoutSwizzle128B);
-      const uint64_t kO = smem_desc(sO, 16, 1024, kLayoutSwizzle128B);
-      const uint64_t mO = smem_desc(sO, L::kHalf, 1024, kLayoutSwizzle128B);
-      const uint64_t kDS = smem_desc(sDS, 16, 1024, kLayoutSwizzle128B);
-      const uint64_t mDS = smem_desc(sDS, L::kHalf, 1024, kLayoutSwizzle128B);
+      // Start address and LBO sit in the low word; every descriptor shares the high word
+      // (1024-byte stride, SW128), kept once in desc_hi, so each costs one register.
+      const uint32_t desc_hi = (uint32_t)(smem_desc(sK, 16, 1024, kLayoutSwizzle128B) >> 32);
+      const uint32_t kK = (uint32_t)smem_desc(sK, 16, 1024, kLayoutSwizzle128B);
+      const uint32_t mK = (uint32_t)smem_desc(sK, L::kHalf, 1024, kLayoutSwizzle128B);
+      const uint32_t kV = (uint32_t)smem_desc(sV, 16, 1024, kLayoutSwizzle128B);
+      const uint32_t kQ = (uint32_t)smem_desc(sQ, 16, 1024, kLayoutSwizzle128B);
+      const uint32_t mQ = (uint32_t)smem_desc(sQ, L::kHalf, 1024, kLayoutSwizzle128B);
+      const uint32_t kO = (uint32_t)smem_desc(sO, 16, 1024, kLayoutSwizzle128B);
+      const uint32_t mO = (uint32_t)smem_desc(sO, L::kHalf, 1024, kLayoutSwizzle128B);
+      const uint32_t kDS = (uint32_t)smem_desc(sDS, 16, 1024, kLayoutSwizzle128B);
+      const uint32_t mDS = (uint32_t)smem_desc(sDS, L::kHalf, 1024, kLayoutSwizzle128B);
       auto issue_sdp = [&](int t, int hh) -> bool {
         const int st = t & 1;
-        const uint64_t qoff = (uint64_t)((st * L::kQBytes + hh * 8192) >> 4);
-        const uint64_t ooff = (uint64_t)((st * L::kOBytes + hh * 8192) >> 4);
+        const uint32_t qoff = (uint32_t)((st * L::kQBytes + hh * 8192) >> 4);
+        const uint32_t ooff = (uint32_t)((st * L::kOBytes + hh * 8192) >> 4);
         const uint32_t cS = tmem + (hh ? kColSb : kColSa), cP = tmem + (hh ? kColDPb : kColDPa);
-        if (hh == 0 && !mbar_wait(bar.qd_full(st), (t >> 1) & 1, a.status)) return false;
-        if (t >= 1 && !mbar_wait(bar.dv_done(hh), (t - 1) & 1, a.status)) return false;   // P^T_h read
+        if (hh == 0 && !wait_(bar.qd_full(st), (t >> 1) & 1)) return false;
+        if (t >= 1 && !wait_(bar.dv_done(hh), (t - 1) & 1)) return false;   // P^T_h read
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
-          mma_ss(cS, kK + off16, kQ + qoff + off16, id_s, ks > 0);
+          mma_ss_(cS, kK + off16, kQ + qoff + off16, desc_hi, id_s, ks > 0);
         }
-        if (DQ && t >= 1 && !mbar_wait(bar.dq_free(hh), (t - 1) & 1, a.status)) return false;   // dQ^T_h read
+        if (DQ && t >= 1 && !wait_(bar.dq_free(hh), (t - 1) & 1)) return false;   // dQ^T_h read
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DV / 16; ++ks) {
           const uint32_t off16 = ((ks >> 2) * L::kHalf + (ks & 3) * 32) >> 4;
-          mma_ss(cP, kV + off16, kO + ooff + off16, id_s, ks > 0);
+          mma_ss_(cP, kV + off16, kO + ooff + off16, desc_hi, id_s, ks > 0);
         }
-        mma_commit(bar.sdp_full(hh));
+        commit_(bar.sdp_full(hh));
         return true;
       };
       auto issue_grads = [&](int t, int hh) {
         const int st = t & 1;
-        const uint64_t qoff = (uint64_t)((st * L::kQBytes) >> 4), ooff = (uint64_t)((st * L::kOBytes) >> 4);
-        const uint64_t dsoff = (uint64_t)((hh * L::kHalf) >> 4);
+        const uint32_t qoff = (uint32_t)((st * L::kQBytes) >> 4), ooff = (uint32_t)((st * L::kOBytes) >> 4);
+        const uint32_t dsoff = (uint32_t)((hh * L::kHalf) >> 4);
         const uint32_t cS = tmem + (hh ? kColSb : kColSa), cP = tmem + (hh ? kColDPb : kColDPa);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kColDV, cS + kk * 8, mO + ooff + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_dv,
-                 (t > 0 || hh > 0 || kk > 0));
-        mma_commit(bar.dv_done(hh));
+          mma_ts_(tmem + kColDV, cS + kk * 8, mO + ooff + (uint32_t)(((4 * hh + kk) * 2048) >> 4), desc_hi,
+                          id_dv, (t > 0 || hh > 0 || kk > 0));
+        commit_(bar.dv_done(hh));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kColDK, kDS + dsoff + (uint64_t)((kk * 32) >> 4),
-                 mQ + qoff + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_dk, (t > 0 || hh > 0 || kk > 0));
+          mma_ss_(tmem + kColDK, kDS + dsoff + (uint32_t)((kk * 32) >> 4),
+                          mQ + qoff + (uint32_t)(((4 * hh + kk) * 2048) >> 4), desc_hi, id_dk, (t > 0 || hh > 0 || kk > 0));
         if (DQ) {
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ss(cP, mK + (uint64_t)((kk * 2048) >> 4), mDS + dsoff + (uint64_t)((kk * 2048) >> 4), id_dq, kk > 0);
-          mma_commit(bar.dq_full(hh));
+            mma_ss_(cP, mK + (uint32_t)((kk * 2048) >> 4), mDS + dsoff + (uint32_t)((kk * 2048) >> 4), desc_hi, id_dq,
+                            kk > 0);
+          commit_(bar.dq_full(hh));
         }
-        mma_commit(bar.ds_free(hh));
+        commit_(bar.ds_free(hh));
       };
-      bool ok = mbar_wait(bar.kv_full(), 0, a.status);
+      bool ok = wait_(bar.kv_full(), 0);
       if (ok) ok = issue_sdp(0, 0) && issue_sdp(0, 1);
       for (int t = 0; t < T && ok; ++t) {
-        if (!(ok = mbar_wait(bar.compute_done(0), t & 1, a.status))) break;
+        if (!(ok = wait_(bar.compute_done(0), t & 1))) break;
         tc_fence_after();
         issue_grads(t, 0);
-        if (!(ok = mbar_wait(bar.compute_done(1), t & 1, a.status))) break;
+        if (!(ok = wait_(bar.compute_done(1), t & 1))) break;
         tc_fence_after();
         if (t + 1 < T && !(ok = issue_sdp(t + 1, 0))) break;
         issue_grads(t, 1);
-        mma_commit(bar.qd_empty(t & 1));
+        commit_(bar.qd_empty(t & 1));
         if (t + 1 < T && !(ok = issue_sdp(t + 1, 1))) break;
       }
-      mma_commit(bar.drain());
-      mbar_wait(bar.drain(), 0, a.status);
+      commit_(bar.drain());
+      wait_(bar.drain(), 0);
     }
   } else if (warp < 4) {
     regs_dec<kRegsLow>();   // warps 2-3: dropout keep flags (below), else no role

@@ -171,7 +171,8 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
     }
   } else if (warp == 1) {
     // ================================ MMA issuer =========================================
-    if (lane == 0 && n > 0) {
+    // The whole warp runs the issue loop in step; elect.sync picks the issuing lane.
+    if (n > 0) {
       constexpr uint32_t idesc_s = idesc_of<T>(kBM, kBN, 0, 0);   // Q (TMEM) x K (K-major)
       constexpr uint32_t idesc_pv = idesc_of<T>(kBM, D, 0, 1);    // P (TMEM) x V (MN-major)
       // Shared-memory descriptors, built once; an address offset adds to the start field.
@@ -180,40 +181,40 @@ fwd_d256_sm100_kernel(const FwdArgs a, int zmax, const __grid_constant__ CUtenso
       // S(j) = Q K_j^T into buffer j % 2, then K_j's stage is free
       auto issue_s = [&](int j) -> bool {
         const int st = j % kStages;
-        if (!mbar_wait(bar.k_full(st), (j / kStages) & 1, a.status)) return false;
+        if (!mbar_wait_warp(bar.k_full(st), (j / kStages) & 1, a.status)) return false;
         tc_fence_after();
         const uint64_t dk = dK0 + (uint64_t)((st * kTileBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off16 = ((ks >> 2) * kBox + (ks & 3) * 32) >> 4;
-          mma_ts(tmem + col_S(j & 1), tmem + kColQ + ks * 8, dk + off16, idesc_s, ks > 0 ? 1u : 0u);
+          mma_ts_elect(tmem + col_S(j & 1), tmem + kColQ + ks * 8, dk + off16, idesc_s, ks > 0 ? 1u : 0u);
         }
-        mma_commit(bar.s_full(j & 1));
-        mma_commit(bar.k_empty(st));
+        mma_commit_elect(bar.s_full(j & 1));
+        mma_commit_elect(bar.k_empty(st));
         return true;
       };
-      bool ok = mbar_wait(bar.q_full(), 0, a.status);
+      bool ok = mbar_wait_warp(bar.q_full(), 0, a.status);
       tc_fence_after();
       if (ok) ok = issue_s(0);
       if (ok && n > 1) ok = issue_s(1);
       for (int j = 0; j < n && ok; ++j) {
         const int st = j % kStages;
-        if (!(ok = mbar_wait(bar.p_full(j & 1), (j >> 1) & 1, a.status))) break;
-        if (!(ok = mbar_wait(bar.v_full(st), (j / kStages) & 1, a.status))) break;
+        if (!(ok = mbar_wait_warp(bar.p_full(j & 1), (j >> 1) & 1, a.status))) break;
+        if (!(ok = mbar_wait_warp(bar.v_full(st), (j / kStages) & 1, a.status))) break;
         tc_fence_after();
         const uint64_t dv = dV0 + (uint64_t)((st * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + kColO, tmem + col_S(j & 1) + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+          mma_ts_elect(tmem + kColO, tmem + col_S(j & 1) + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                  (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar.pv_done());
-        mma_commit(bar.v_empty(st));
+        mma_commit_elect(bar.pv_done());
+        mma_commit_elect(bar.v_empty(st));
         if (j + 2 < n) ok = issue_s(j + 2);
       }
-      if (ok) mma_commit(bar.o_done());
+      if (ok) mma_commit_elect(bar.o_done());
       // every MMA must be complete before the TMEM is freed
-      mma_commit(bar.drain());
-      mbar_wait(bar.drain(), 0, a.status);
+      mma_commit_elect(bar.drain());
+      mbar_wait_warp(bar.drain(), 0, a.status);
     }
   } else if (warp >= 4) {
     // ================================ softmax warps ======================================
