@@ -20,7 +20,8 @@
 //       dP^T [192,256) dK [256,512); per 64-query tile: S^T = K Q^T (TS),
 //       dP^T = V dout^T (SS), dS^T over S^T's columns, dK += dS^T Q (TS).
 // None of them needs atomics, so the result is the same bits on every run.  Warps: 0 TMA
-// producer, 1 TMEM allocation and MMA issuer (one thread), 2-3 idle, 4-7 compute (thread t =
+// producer, 1 TMEM allocation and MMA issuer (the warp in step, one elected lane issuing),
+// 2-3 idle, 4-7 compute (thread t =
 // stationary row t = TMEM lane t).  Every mbarrier wait is bounded; a timeout sets the status
 // word and the CTA drains and frees its TMEM instead of hanging.  Named barriers (the per-tile
 // lse_tot / D staging of the key-stationary kernels) are passed by every compute warp in

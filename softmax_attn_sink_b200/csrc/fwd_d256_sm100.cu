@@ -12,7 +12,8 @@
 // reads only the 2 KB K slice from shared memory.
 //
 // TMEM columns: Q [0,128), S/P buffer 0 [128,192), buffer 1 [192,256), O [256,512).
-// Warps: 0 TMA producer (K / V ring), 1 TMEM allocation and MMA issuer (one thread), 2-3 idle,
+// Warps: 0 TMA producer (K / V ring), 1 TMEM allocation and MMA issuer (the warp runs the loop
+// in step; elect.sync over the full warp picks the same issuing lane every time), 2-3 idle,
 // 4-7 softmax (thread t = query row t = TMEM lane t), which first copy their Q rows into TMEM
 // and finally write out and lse.
 // MMA issue order: S(0), S(1), then per tile j: PV(j), S(j+2).  S(j+2) goes into the buffer

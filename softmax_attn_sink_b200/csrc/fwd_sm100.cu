@@ -17,8 +17,11 @@
 //   warp 0      TMA producer: Q_A, Q_B per item (once the previous item's last QK has read
 //               Q), then K and V tiles into a 2-stage ring; a stage's K and V are released
 //               together once both PVs of its tile are issued (one commit per tile).
-//   warp 1      TMEM allocation and the MMA issuer (one thread), in the order
+//   warp 1      TMEM allocation and the MMA issuer, in the order
 //                 PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1)
+//               Without dropout the whole warp runs the loop in step and elect.sync over the
+//               full warp picks the issuing lane (the same lane every time, so every MMA and
+//               commit still comes from one thread); with dropout lane 0 alone runs it.
 //               so the tensor core works for one unit while the other unit's softmax runs;
 //               on an item's last tile the QKs of the next item's first tile follow the
 //               PVs directly.  QK: S_U = Q_U K^T (A, B from shared memory); PV: O_U += P_U V
