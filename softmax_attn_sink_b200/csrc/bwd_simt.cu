@@ -56,6 +56,112 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
   }
 }
 
+// The same pass with 16-byte loads, for head dims that are a multiple of one load: a row of
+// out / dout is split over L lanes (L = DV / elements per load, at most 32), each warp covers
+// its 8 rows in 8 L / 32 passes whose loads are all issued before any product is summed, and
+// the L lanes of a row reduce with xor shuffles.  Same grid, rows and partial layout as above.
+__device__ __forceinline__ float dot16(uint4 x, uint4 y, const __nv_bfloat16*) {
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+  float d = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 u = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[k]));
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[k]));
+    d = fmaf(u.x, v.x, d);
+    d = fmaf(u.y, v.y, d);
+  }
+  return d;
+}
+__device__ __forceinline__ float dot16(uint4 x, uint4 y, const __half*) {
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+  float d = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 u = __half22float2(*reinterpret_cast<const __half2*>(&xs[k]));
+    const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&ys[k]));
+    d = fmaf(u.x, v.x, d);
+    d = fmaf(u.y, v.y, d);
+  }
+  return d;
+}
+__device__ __forceinline__ float dot16(uint4 x, uint4 y, const float*) {
+  float d = __uint_as_float(x.x) * __uint_as_float(y.x);
+  d = fmaf(__uint_as_float(x.y), __uint_as_float(y.y), d);
+  d = fmaf(__uint_as_float(x.z), __uint_as_float(y.z), d);
+  return fmaf(__uint_as_float(x.w), __uint_as_float(y.w), d);
+}
+
+template <typename T, int DV>
+__global__ void __launch_bounds__(256) bwd_preprocess_vec_kernel(const BwdArgs a) {
+  constexpr int kEpv = 16 / (int)sizeof(T);      // elements per 16-byte load
+  constexpr int kNv = DV / kEpv;                 // loads per row
+  constexpr int kL = kNv < 32 ? kNv : 32;        // lanes per row
+  constexpr int kVpl = kNv / kL;                 // loads per lane and row
+  constexpr int kR = 32 / kL;                    // rows per pass
+  constexpr int kP = 8 / kR;                     // passes over the warp's 8 rows
+  static_assert(kNv * kEpv == DV && kL * kVpl == kNv && kR * kP == 8, "row split");
+  const int h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % kL, rsub = lane / kL;
+  const float sink = a.sink ? a.sink[h] : kNegInf;
+  const uint4* out = static_cast<const uint4*>(a.out);
+  const uint4* dout = static_cast<const uint4*>(a.dout);
+  const long long r0 = ((long long)blockIdx.x * 8 + warp) * 8;
+  uint4 xo[kP][kVpl], xd[kP][kVpl];
+#pragma unroll
+  for (int p = 0; p < kP; ++p) {
+    const long long i = r0 + p * kR + rsub;
+    const long long base = (i * a.hq + h) * kNv;   // in 16-byte loads
+#pragma unroll
+    for (int v = 0; v < kVpl; ++v) {
+      if (i < a.total_q) {
+        xo[p][v] = __ldg(out + base + sub + v * kL);
+        xd[p][v] = __ldg(dout + base + sub + v * kL);
+      } else {
+        xo[p][v] = make_uint4(0u, 0u, 0u, 0u);
+        xd[p][v] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  float ds_acc = 0.f;
+#pragma unroll
+  for (int p = 0; p < kP; ++p) {
+    float d = 0.f;
+#pragma unroll
+    for (int v = 0; v < kVpl; ++v) d += dot16(xo[p][v], xd[p][v], static_cast<const T*>(nullptr));
+#pragma unroll
+    for (int o = kL / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    const long long i = r0 + p * kR + rsub;
+    if (sub == 0 && i < a.total_q) {
+      const long long k = (long long)h * a.total_q + i;
+      const float lt = logaddexp(a.lse[k], sink);
+      a.D[k] = d;
+      a.lse_tot[k] = lt;
+      if (sink != kNegInf && lt != kNegInf) ds_acc -= __expf(sink - lt) * d;
+    }
+  }
+  ds_acc = warp_sum(ds_acc);
+  __shared__ float red[8];
+  if (lane == 0) red[warp] = ds_acc;
+  __syncthreads();
+  if (threadIdx.x == 0 && a.dsink) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += red[w];
+    a.dsink_part[(long long)h * gridDim.x + blockIdx.x] = s;   // summed in a fixed order later
+  }
+}
+
+template <typename T>
+void launch_preprocess_typed(const BwdArgs& a, dim3 grid, cudaStream_t s) {
+  switch (a.dv) {
+    case 32: bwd_preprocess_vec_kernel<T, 32><<<grid, 256, 0, s>>>(a); return;
+    case 64: bwd_preprocess_vec_kernel<T, 64><<<grid, 256, 0, s>>>(a); return;
+    case 128: bwd_preprocess_vec_kernel<T, 128><<<grid, 256, 0, s>>>(a); return;
+    case 256: bwd_preprocess_vec_kernel<T, 256><<<grid, 256, 0, s>>>(a); return;
+    default: bwd_preprocess_kernel<T><<<grid, 256, 0, s>>>(a); return;
+  }
+}
+
 // d_sink[h] = sum over the preprocess blocks of their partials, one warp per head: lane l
 // adds blocks l, l + 32, ... in order, then a fixed butterfly combines the lanes, so the
 // result does not depend on the order in which blocks ran.
@@ -333,11 +439,11 @@ cudaError_t dispatch_dims(const BwdArgs& a, cudaStream_t s) {
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, int dtype, cudaStream_t s) {
   dim3 grid((a.total_q + 63) / 64, a.hq);
   if (dtype == 1)
-    bwd_preprocess_kernel<float><<<grid, 256, 0, s>>>(a);
+    launch_preprocess_typed<float>(a, grid, s);
   else if (dtype == 2)
-    bwd_preprocess_kernel<__half><<<grid, 256, 0, s>>>(a);
+    launch_preprocess_typed<__half>(a, grid, s);
   else
-    bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
+    launch_preprocess_typed<__nv_bfloat16>(a, grid, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.dsink) return e;
   dsink_reduce_kernel<<<a.hq, 32, 0, s>>>(a, (int)grid.x);
