@@ -47,11 +47,12 @@ constexpr int kBN = 128;       // keys per tile
 constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 compute
 // With dropout a fourth warpgroup (warps 8-11, one warp per SM sub-partition) draws the keep
 // bytes of each key tile one tile ahead of the compute warps, into a two-stage shared-memory
-// ring.  Launched at 168 registers (384 x 168 = 64512): the first and the dropout warpgroups
-// drop to 136, the compute warps take 232 (128 x (136 + 136 + 232) = 64512).
+// ring.  Launched at 168 registers (384 x 168 = 64512): the first warpgroup drops to 136, the
+// dropout warpgroup to 120, the compute warps take 248 (128 x (136 + 120 + 248) = 64512; no
+// spills, where 136 / 136 / 232 spilled 24 bytes).
 constexpr int kThreadsDrop = 384;
-constexpr int kRegsLowD = 136, kRegsHighD = 232;
-static_assert(128 * (2 * kRegsLowD + kRegsHighD) <= kThreadsDrop * 168, "register split");
+constexpr int kRegsLowD = 136, kRegsFlagD = 120, kRegsHighD = 248;
+static_assert(128 * (kRegsLowD + kRegsFlagD + kRegsHighD) <= kThreadsDrop * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColP = 128, kColQ = 256;
 __host__ __device__ constexpr uint32_t col_S(int b) { return b ? 384u : 0u; }
@@ -389,7 +390,7 @@ bwd_dq_sm100_kernel(const BwdArgs a, const __grid_constant__ CUtensorMap tm_q,
     // Philox keep bytes of row r for the 8 16-key blocks of key tile j (counter: key block,
     // packed row, q head, offset), turned into drop flags (bit 7 of a byte set = dropped) and
     // stored for the compute thread of the same row.
-    regs_dec<kRegsLowD>();
+    regs_dec<kRegsFlagD>();
     const int r = (warp - 8) * 32 + lane;
     const uint32_t row = (uint32_t)(q0 + m0 + r);
     const uint32_t t4 = (a.drop.threshold - 1u) * 0x01010101u, t4h = t4 | 0x80808080u;
