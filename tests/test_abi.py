@@ -27,6 +27,24 @@ def test_library_exports_every_declared_symbol():
     assert set(sab._SYMBOLS) <= set(declared)
 
 
+def test_debug_library_exports_the_same_symbols():
+    """The bounds-checking build (libattn_sink_debug.so, built beside the release library)
+    exports every declared function too, and ATTN_SINK_LIBRARY makes the binding load it."""
+    import subprocess
+    import sys
+    from softmax_attn_sink_b200 import build as B
+    if not os.path.exists(B.LIB_DEBUG):
+        pytest.skip("debug library not built (python -m softmax_attn_sink_b200.build --debug)")
+    D = ctypes.CDLL(B.LIB_DEBUG)
+    for name in _declared_functions():
+        assert hasattr(D, name), f"{name} missing from the debug library"
+    code = "import softmax_attn_sink_b200 as s; s.lib(); print(s.LIB_PATH)"
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       env=dict(os.environ, ATTN_SINK_LIBRARY=B.LIB_DEBUG), timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert os.path.samefile(r.stdout.strip().splitlines()[-1], B.LIB_DEBUG)
+
+
 def test_params_struct_matches_header_field_order():
     text = open(HEADER).read()
     body = re.search(r"typedef struct \{(.*?)\} attn_sink_params;", text, flags=re.S).group(1)
